@@ -1,0 +1,234 @@
+"""Pins of the oracle's routing, grouping, forward and backward (CPU only)."""
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from grouped_nf4_expert_b200 import inputs
+
+
+def _experts(prob, lora_dtype=np.float64):
+    f = lambda b: inputs.bits_to_f32(b).astype(lora_dtype)  # noqa: E731
+    return oracle.Experts(prob.gate_up_nf4, prob.gate_up_absmax, prob.down_nf4,
+                          prob.down_absmax, f(prob.A_gu), f(prob.B_gu), f(prob.A_d), f(prob.B_d))
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    prob = inputs.make_problem(inputs.CONFIGS["tiny"])
+    return prob, _experts(prob), inputs.bits_to_f32(prob.x).astype(np.float64)
+
+
+# ---------------------------------------------------------------- routing
+
+def test_route_matches_torch_topk_softmax():
+    rng = np.random.default_rng(0)
+    logits = rng.standard_normal((500, 37)).astype(np.float32)
+    ids, w = oracle.route_topk(logits, 5)
+    tl = torch.from_numpy(logits)
+    vals, idx = torch.topk(tl, 5, dim=1, sorted=True)
+    assert np.array_equal(ids, idx.numpy().astype(np.int32))
+    ref = torch.softmax(vals.double(), dim=1).numpy()
+    np.testing.assert_allclose(w, ref, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-14)
+
+
+def test_route_ties_go_to_lower_id_and_order_is_descending():
+    logits = np.array([[0.5, 2.0, 2.0, -1.0, 2.0],
+                       [0.0, 0.0, 0.0, 0.0, 0.0],
+                       [-0.0, 0.0, 1.0, -3.0, 0.0]], dtype=np.float32)
+    ids, w = oracle.route_topk(logits, 3)
+    assert ids.tolist() == [[1, 2, 4], [0, 1, 2], [2, 0, 1]]
+    np.testing.assert_allclose(w[1], [1 / 3] * 3, rtol=1e-15)
+
+
+def test_route_rejects_bad_k():
+    with pytest.raises(ValueError):
+        oracle.route_topk(np.zeros((2, 3), np.float32), 4)
+
+
+def test_grouping_is_a_stable_sort():
+    rng = np.random.default_rng(1)
+    ids = rng.integers(0, 9, (300, 3)).astype(np.int32)
+    ids[:, 1] = (ids[:, 0] + 1) % 9  # distinct within a token like real routing
+    g = oracle.group_by_expert(ids, 10)
+    flat = ids.reshape(-1)
+    ref = np.argsort(flat, kind="stable")
+    assert np.array_equal(g["slots"], ref)
+    assert np.array_equal(g["counts"], np.bincount(flat, minlength=10))
+    assert g["counts"][9] == 0 and g["starts"][-1] == flat.size
+    assert np.array_equal(np.sort(g["slots"]), np.arange(flat.size))
+    for f in range(flat.size):
+        assert g["slots"][g["starts"][flat[f]] + g["rank"][f]] == f
+
+
+# ---------------------------------------------------------------- forward pins
+
+def test_b_zero_gives_base_block_exactly():
+    prob = inputs.make_problem(inputs.CONFIGS["tiny_b0"])
+    ex = _experts(prob)
+    base = oracle.Experts(ex.gate_up_nf4, ex.gate_up_absmax, ex.down_nf4, ex.down_absmax,
+                          np.zeros_like(ex.A_gu), ex.B_gu, np.zeros_like(ex.A_d), ex.B_d)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    a = oracle.moe_forward(x, prob.logits, ex, 2, 16.0)
+    b = oracle.moe_forward(x, prob.logits, base, 2, 16.0)
+    assert np.any(ex.A_gu != 0)
+    assert np.array_equal(a["y"], b["y"])
+
+
+def _silu(v):
+    return v / (1 + np.exp(-v))
+
+
+def test_bruteforce_per_token_per_expert_loop(tiny):
+    prob, ex, x = tiny
+    cfg = prob.cfg
+    s = cfg.alpha / cfg.r
+    out = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha)
+    # Independent brute force: every token against every expert, a dense
+    # gate over all E with zeros outside the top-k, matrix-vector products.
+    T, E, I = cfg.T, cfg.E, cfg.I
+    W = [oracle.expert_weights(ex, e) for e in range(E)]
+    y = np.zeros((T, cfg.H))
+    for t in range(T):
+        lg = prob.logits[t].astype(np.float64)
+        top = sorted(range(E), key=lambda e: (-prob.logits[t, e], e))[: cfg.top_k]
+        z = np.array([np.exp(lg[e] - lg[top[0]]) for e in top])
+        gate = np.zeros(E)
+        gate[top] = z / z.sum()
+        for e in range(E):
+            wgu, wd = W[e]
+            hv = wgu.dot(x[t]) + s * ex.B_gu[e].dot(ex.A_gu[e].dot(x[t]))
+            av = _silu(hv[:I]) * hv[I:]
+            yv = wd.dot(av) + s * ex.B_d[e].dot(ex.A_d[e].dot(av))
+            y[t] += gate[e] * yv
+    np.testing.assert_allclose(out["y"], y, rtol=1e-11, atol=1e-13)
+
+
+def test_dense_delta_equivalence_with_torch(tiny):
+    prob, ex, x = tiny
+    cfg = prob.cfg
+    s = cfg.alpha / cfg.r
+    out = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha)
+    ids, w = out["ids"], out["w"]
+    xt = torch.from_numpy(x)
+    y = torch.zeros(cfg.T, cfg.H, dtype=torch.float64)
+    for e in range(cfg.E):
+        wgu, wd = (torch.from_numpy(m) for m in oracle.expert_weights(ex, e))
+        wgu = wgu + s * torch.from_numpy(ex.B_gu[e]) @ torch.from_numpy(ex.A_gu[e])
+        wd = wd + s * torch.from_numpy(ex.B_d[e]) @ torch.from_numpy(ex.A_d[e])
+        h = F.linear(xt, wgu)
+        yd = F.linear(F.silu(h[:, : cfg.I]) * h[:, cfg.I:], wd)
+        gate = torch.from_numpy(((ids == e) * w).sum(1))
+        y += gate[:, None] * yd
+    np.testing.assert_allclose(out["y"], y.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_token_subset_matches_full(tiny):
+    prob, ex, x = tiny
+    full = oracle.moe_forward(x, prob.logits, ex, 2, 16.0)
+    sub = oracle.moe_forward(x, prob.logits, ex, 2, 16.0, tokens=[3, 17, 30])
+    np.testing.assert_allclose(sub["y"][[3, 17, 30]], full["y"][[3, 17, 30]], rtol=1e-12, atol=1e-15)
+    assert np.all(sub["y"][0] == 0)
+
+
+# ---------------------------------------------------------------- backward pins
+
+def _dense_torch_block(x, ex, s, I):
+    """E = 1, k = 1: the block is a dense SwiGLU MLP with LoRA on both projections."""
+    wgu, wd = (torch.from_numpy(m) for m in oracle.expert_weights(ex, 0))
+    X = torch.from_numpy(x).requires_grad_(True)
+    A_gu = torch.from_numpy(ex.A_gu[0].copy()).requires_grad_(True)
+    B_gu = torch.from_numpy(ex.B_gu[0].copy()).requires_grad_(True)
+    A_d = torch.from_numpy(ex.A_d[0].copy()).requires_grad_(True)
+    B_d = torch.from_numpy(ex.B_d[0].copy()).requires_grad_(True)
+    h = F.linear(X, wgu) + s * F.linear(F.linear(X, A_gu), B_gu)
+    a = F.silu(h[:, :I]) * h[:, I:]
+    y = F.linear(a, wd) + s * F.linear(F.linear(a, A_d), B_d)
+    return y, (X, A_gu, B_gu, A_d, B_d)
+
+
+def test_single_expert_reduces_to_dense_swiglu_mlp_with_torch_autograd():
+    cfg = inputs.Config("e1k1", E=1, H=64, I=128, top_k=1, T=24, r=8, alpha=16.0,
+                        routing="normal", seed=21)
+    prob = inputs.make_problem(cfg)
+    ex = _experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    s = cfg.alpha / cfg.r
+    y, leaves = _dense_torch_block(x, ex, s, cfg.I)
+    (y * torch.from_numpy(dY)).sum().backward()
+    fo = oracle.moe_forward(x, prob.logits, ex, 1, cfg.alpha)
+    bo = oracle.moe_backward(x, prob.logits, dY, ex, 1, cfg.alpha)
+    np.testing.assert_allclose(fo["y"], y.detach().numpy(), rtol=1e-11, atol=1e-13)
+    X, A_gu, B_gu, A_d, B_d = leaves
+    for mine, ref in [(bo["dx"], X.grad), (bo["dA_gu"][0], A_gu.grad), (bo["dB_gu"][0], B_gu.grad),
+                      (bo["dA_d"][0], A_d.grad), (bo["dB_d"][0], B_d.grad)]:
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-13)
+
+
+def _loss(x, logits, dY, ex, k, alpha):
+    return float(np.sum(oracle.moe_forward(x, logits, ex, k, alpha)["y"] * dY))
+
+
+def test_finite_differences_all_gradients(tiny):
+    prob, ex, x = tiny
+    cfg = prob.cfg
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    bo = oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha)
+    rng = np.random.default_rng(7)
+    eps = 1e-4
+
+    def check(name, grad, perturb):
+        v = rng.standard_normal(grad.shape)
+        v /= np.linalg.norm(v)  # unit direction: truncation error O(eps^2)
+        lp = perturb(eps * v)
+        lm = perturb(-eps * v)
+        fd = (lp - lm) / (2 * eps)
+        an = float(np.sum(grad * v))
+        assert np.linalg.norm(grad) > 1e-3, name
+        assert abs(fd - an) <= 1e-7 * np.linalg.norm(grad), (name, fd, an)
+
+    def with_lora(key, dv):
+        kw = {f: getattr(ex, f) for f in ("gate_up_nf4", "gate_up_absmax", "down_nf4", "down_absmax",
+                                          "A_gu", "B_gu", "A_d", "B_d")}
+        kw[key] = kw[key] + dv
+        return _loss(x, prob.logits, dY, oracle.Experts(**kw), cfg.top_k, cfg.alpha)
+
+    check("dx", bo["dx"], lambda dv: _loss(x + dv, prob.logits, dY, ex, cfg.top_k, cfg.alpha))
+    check("dA_gu", bo["dA_gu"], lambda dv: with_lora("A_gu", dv))
+    check("dB_gu", bo["dB_gu"], lambda dv: with_lora("B_gu", dv))
+    check("dA_d", bo["dA_d"], lambda dv: with_lora("A_d", dv))
+    check("dB_d", bo["dB_d"], lambda dv: with_lora("B_d", dv))
+    # and a few single coordinates of dx
+    for (t, h) in [(0, 0), (5, 33), (31, 63)]:
+        d = np.zeros_like(x)
+        d[t, h] = eps
+        fd = (_loss(x + d, prob.logits, dY, ex, 2, 16.0) - _loss(x - d, prob.logits, dY, ex, 2, 16.0)) / (2 * eps)
+        assert abs(fd - bo["dx"][t, h]) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_b_zero_gives_zero_dA_and_empty_expert_zero_grads():
+    prob = inputs.make_problem(inputs.CONFIGS["tiny_b0"])
+    ex = _experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    logits = prob.logits.copy()
+    logits[:, 3] = -1e30  # expert 3 never routed
+    bo = oracle.moe_backward(x, logits, dY, ex, 2, 16.0)
+    assert np.all(bo["dA_gu"] == 0) and np.all(bo["dA_d"] == 0)
+    assert np.any(bo["dB_gu"][0] != 0) and np.any(bo["dB_d"][0] != 0)
+    for key in ("dB_gu", "dB_d"):
+        assert np.all(bo[key][3] == 0)
+
+
+def test_backward_subsets_match_full(tiny):
+    prob, ex, x = tiny
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    full = oracle.moe_backward(x, prob.logits, dY, ex, 2, 16.0)
+    sub = oracle.moe_backward(x, prob.logits, dY, ex, 2, 16.0, tokens=[1, 2], grad_experts=[2])
+    np.testing.assert_allclose(sub["dx"][[1, 2]], full["dx"][[1, 2]], rtol=1e-12, atol=1e-15)
+    for key in ("dA_gu", "dB_gu", "dA_d", "dB_d"):
+        np.testing.assert_allclose(sub[key][2], full[key][2], rtol=1e-12, atol=1e-15)
