@@ -1,0 +1,476 @@
+// C-ABI entry points (include/e4b.h): host-side validation, buffer sizes,
+// workspace layout, tensor-map encoding and the launch sequence of each call.
+// No entry point allocates device memory; only e4b_check_device_error
+// synchronises.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "e4b_device.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_num_sms[kMaxDevices] = {0};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cudaError_t device_sms(int* out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    g_num_sms[dev] = n;
+  }
+  *out = g_num_sms[dev];
+  return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int r_padded(int r) { return r <= 16 ? 16 : (r <= 32 ? 32 : 64); }
+
+e4b_status check_dims(const e4b_moe_dims* d, int32_t T) {
+  if (d == nullptr || T < 0) return E4B_ERR_INVALID_ARG;
+  if (d->E < 1 || d->E > E4B_MAX_EXPERTS) return E4B_ERR_UNSUPPORTED;
+  if (d->H <= 0 || d->H % 64 || d->I <= 0 || d->I % 64) return E4B_ERR_UNSUPPORTED;
+  if (d->top_k < 1 || d->top_k > d->E || d->top_k > E4B_MAX_TOP_K) return E4B_ERR_UNSUPPORTED;
+  if (d->r < 8 || d->r > E4B_MAX_RANK || d->r % 8) return E4B_ERR_UNSUPPORTED;
+  if (d->blocksize != 64) return E4B_ERR_UNSUPPORTED;
+  if (d->act != E4B_ACT_SILU_GLU) return E4B_ERR_UNSUPPORTED;
+  if (!isfinite(d->alpha)) return E4B_ERR_INVALID_ARG;
+  // 32-bit row and element indices inside the kernels
+  const int64_t N = (int64_t)T * d->top_k;
+  const int64_t rc = rows_cap(N, d->E);
+  if (rc * (int64_t)(2 * d->I > d->H ? 2 * d->I : d->H) >= ((int64_t)1 << 40) || rc >= ((int64_t)1 << 30))
+    return E4B_ERR_UNSUPPORTED;
+  return E4B_OK;
+}
+
+size_t workspace_bytes(const e4b_moe_dims* d, int32_t T) {
+  const int64_t nblk = ((int64_t)T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock;
+  const size_t route = (size_t)2 * nblk * d->E * sizeof(int32_t);
+  return sizeof(DeviceError) + ((route + 255) / 256) * 256;
+}
+
+e4b_status check_ws(const e4b_moe_dims* d, int32_t T, const void* ws, size_t ws_bytes) {
+  if (!aligned16(ws)) return E4B_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(d, T)) return E4B_ERR_WORKSPACE_TOO_SMALL;
+  return E4B_OK;
+}
+
+e4b_status check_routing(const e4b_routing* r) {
+  if (r == nullptr) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(r->topk_ids) || !aligned16(r->topk_w) || !aligned16(r->counts) || !aligned16(r->offsets) ||
+      !aligned16(r->row_of_slot) || !aligned16(r->slot_of_row) || !aligned16(r->tiles))
+    return E4B_ERR_INVALID_ARG;
+  return E4B_OK;
+}
+
+e4b_status check_base(const e4b_nf4_experts* b) {
+  if (b == nullptr || !aligned16(b->gate_up_nf4) || !aligned16(b->gate_up_absmax) || !aligned16(b->down_nf4) ||
+      !aligned16(b->down_absmax))
+    return E4B_ERR_INVALID_ARG;
+  return E4B_OK;
+}
+
+e4b_status check_lora(const e4b_lora* l) {
+  if (l == nullptr || !aligned16(l->A_gu) || !aligned16(l->B_gu) || !aligned16(l->A_d) || !aligned16(l->B_d))
+    return E4B_ERR_INVALID_ARG;
+  return E4B_OK;
+}
+
+e4b_status check_fwd(const e4b_fwd_buffers* f) {
+  if (f == nullptr || !aligned16(f->x_perm) || !aligned16(f->p_gu) || !aligned16(f->gu) || !aligned16(f->act) ||
+      !aligned16(f->p_d) || !aligned16(f->y_perm))
+    return E4B_ERR_INVALID_ARG;
+  return E4B_OK;
+}
+
+e4b_status check_bwd(const e4b_bwd_buffers* b) {
+  if (b == nullptr || !aligned16(b->dyw) || !aligned16(b->q_d) || !aligned16(b->dgu) || !aligned16(b->q_gu) ||
+      !aligned16(b->dx_perm))
+    return E4B_ERR_INVALID_ARG;
+  return E4B_OK;
+}
+
+#define E4B_TRY(expr)                     \
+  do {                                    \
+    const e4b_status _s = (expr);         \
+    if (_s != E4B_OK) return _s;          \
+  } while (0)
+
+#define E4B_CUDA(expr)                      \
+  do {                                      \
+    if ((expr) != cudaSuccess) {            \
+      (void)cudaGetLastError();             \
+      return E4B_ERR_CUDA;                  \
+    }                                       \
+  } while (0)
+
+}  // namespace
+
+cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                              CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, []() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr) return cudaErrorNotSupported;
+  cuuint64_t d[5];
+  cuuint64_t s[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) s[i] = strides_bytes[i];
+  }
+  const CUresult r = g_encode(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), d, s, b, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace e4b
+
+using namespace e4b;
+
+extern "C" {
+
+const char* e4b_status_string(e4b_status s) {
+  switch (s) {
+    case E4B_OK: return "E4B_OK";
+    case E4B_ERR_INVALID_ARG: return "E4B_ERR_INVALID_ARG: null or misaligned pointer, or inconsistent sizes";
+    case E4B_ERR_UNSUPPORTED: return "E4B_ERR_UNSUPPORTED: shape, rank, block size or epilogue not supported";
+    case E4B_ERR_WORKSPACE_TOO_SMALL: return "E4B_ERR_WORKSPACE_TOO_SMALL: workspace below e4b_get_sizes()";
+    case E4B_ERR_CUDA: return "E4B_ERR_CUDA: a CUDA call or kernel launch failed";
+    case E4B_ERR_DEVICE_TIMEOUT: return "E4B_ERR_DEVICE_TIMEOUT: a device-side wait ran out";
+  }
+  return "E4B_ERR_UNKNOWN";
+}
+
+const char* e4b_version(void) { return "e4b-b200 0.1.0 (sm_100a)"; }
+
+void e4b_nf4_levels(float out[16]) {
+  if (out != nullptr)
+    for (int c = 0; c < 16; ++c) out[c] = nf4_level(c);
+}
+
+e4b_status e4b_get_sizes(const e4b_moe_dims* dims, int32_t T, e4b_sizes* out) {
+  E4B_TRY(check_dims(dims, T));
+  if (out == nullptr) return E4B_ERR_INVALID_ARG;
+  const int64_t N = (int64_t)T * dims->top_k;
+  out->slots = N;
+  out->rows_cap = rows_cap(N, dims->E);
+  out->tiles_cap = tiles_cap(N, dims->E);
+  out->workspace_bytes = workspace_bytes(dims, T);
+  return E4B_OK;
+}
+
+e4b_status e4b_workspace_init(void* ws, size_t ws_bytes, e4b_stream_t stream) {
+  if (!aligned16(ws) || ws_bytes < sizeof(DeviceError)) return E4B_ERR_INVALID_ARG;
+  E4B_CUDA(cudaMemsetAsync(ws, 0, sizeof(DeviceError), (cudaStream_t)stream));
+  return E4B_OK;
+}
+
+e4b_status e4b_check_device_error(const void* ws, e4b_stream_t stream) {
+  if (!aligned16(ws)) return E4B_ERR_INVALID_ARG;
+  DeviceError host;
+  E4B_CUDA(cudaMemcpyAsync(&host, ws, sizeof(DeviceError), cudaMemcpyDeviceToHost, (cudaStream_t)stream));
+  E4B_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  if (host.code == E4B_ERR_DEVICE_TIMEOUT) return E4B_ERR_DEVICE_TIMEOUT;
+  if (host.code != 0) return E4B_ERR_CUDA;
+  return E4B_OK;
+}
+
+e4b_status e4b_route_permute(const e4b_moe_dims* dims, int32_t T, const float* logits, const e4b_bf16* x,
+                             const e4b_routing* routing, e4b_bf16* x_perm, void* ws, size_t ws_bytes,
+                             e4b_stream_t stream) {
+  E4B_TRY(check_dims(dims, T));
+  E4B_TRY(check_ws(dims, T, ws, ws_bytes));
+  E4B_TRY(check_routing(routing));
+  if (!aligned16(logits) || !aligned16(x) || !aligned16(x_perm)) return E4B_ERR_INVALID_ARG;
+  if (T == 0) return E4B_OK;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  const int64_t N = (int64_t)T * dims->top_k;
+  int32_t* scratch = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sizeof(DeviceError));
+  E4B_CUDA(launch_route(logits, x, T, dims->E, dims->H, dims->top_k, routing->topk_ids, routing->topk_w,
+                        routing->counts, routing->offsets, routing->row_of_slot, routing->slot_of_row, routing->tiles,
+                        mtiles_cap(N, dims->E), x_perm, rows_cap(N, dims->E), scratch, sms,
+                        (cudaStream_t)stream));
+  return E4B_OK;
+}
+
+e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e4b_routing* routing,
+                                    const e4b_nf4_experts* base, const e4b_lora* lora, const e4b_fwd_buffers* fwd,
+                                    e4b_bf16* y, void* ws, size_t ws_bytes, e4b_stream_t stream) {
+  E4B_TRY(check_dims(dims, T));
+  E4B_TRY(check_ws(dims, T, ws, ws_bytes));
+  E4B_TRY(check_routing(routing));
+  E4B_TRY(check_base(base));
+  E4B_TRY(check_lora(lora));
+  E4B_TRY(check_fwd(fwd));
+  if (!aligned16(y)) return E4B_ERR_INVALID_ARG;
+  if (T == 0) return E4B_OK;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int E = dims->E, H = dims->H, I = dims->I, r = dims->r, k = dims->top_k;
+  const int64_t N = (int64_t)T * k;
+  const float s = dims->alpha / (float)r;
+  DeviceError* err = static_cast<DeviceError*>(ws);
+
+  LoraProjHost lp{};
+  lp.E = E;
+  lp.r = r;
+  lp.r_pad = r_padded(r);
+  lp.scale = s;
+  lp.tiles = routing->tiles;
+  lp.rows_cap = rows_cap(N, E);
+  lp.mt_cap = mtiles_cap(N, E);
+  lp.err = err;
+  lp.timeout_ns = kDefaultTimeoutNs;
+
+  Nf4GemmHost g{};
+  g.E = E;
+  g.H = H;
+  g.I = I;
+  g.r = r;
+  g.r_pad = r_padded(r);
+  g.tiles = routing->tiles;
+  g.rows_cap = lp.rows_cap;
+  g.mt_cap = lp.mt_cap;
+  g.err = err;
+  g.timeout_ns = kDefaultTimeoutNs;
+
+  // p_gu = s * x_perm A_gu^T
+  lp.act_in = fwd->x_perm;
+  lp.K = H;
+  lp.w = lora->A_gu;
+  lp.w_mn_major = false;
+  lp.out = fwd->p_gu;
+  E4B_CUDA(launch_lora_proj(lp, sms, st));
+  // gu = W_gu x + p_gu B_gu^T ; act = silu(gate) * up
+  g.mode = kFwdGateUp;
+  g.nf4 = base->gate_up_nf4;
+  g.absmax = base->gate_up_absmax;
+  g.stored_rows = 2 * I;
+  g.stored_cols = H;
+  g.act_in = fwd->x_perm;
+  g.K = H;
+  g.n_dim = 2 * I;
+  g.lora_a_rows = fwd->p_gu;
+  g.lora_w = lora->B_gu;
+  g.out0 = fwd->gu;
+  g.out1 = fwd->act;
+  g.aux = nullptr;
+  E4B_CUDA(launch_nf4_gemm(g, sms, st));
+  // p_d = s * act A_d^T
+  lp.act_in = fwd->act;
+  lp.K = I;
+  lp.w = lora->A_d;
+  lp.out = fwd->p_d;
+  E4B_CUDA(launch_lora_proj(lp, sms, st));
+  // y_perm = W_d act + p_d B_d^T
+  g.mode = kFwdDown;
+  g.nf4 = base->down_nf4;
+  g.absmax = base->down_absmax;
+  g.stored_rows = H;
+  g.stored_cols = I;
+  g.act_in = fwd->act;
+  g.K = I;
+  g.n_dim = H;
+  g.lora_a_rows = fwd->p_d;
+  g.lora_w = lora->B_d;
+  g.out0 = fwd->y_perm;
+  g.out1 = nullptr;
+  E4B_CUDA(launch_nf4_gemm(g, sms, st));
+  // y[t] = sum_j w[t,j] y_perm[row(t,j)]
+  E4B_CUDA(launch_combine(fwd->y_perm, routing->row_of_slot, routing->topk_w, T, k, H, y, sms, st));
+  return E4B_OK;
+}
+
+e4b_status e4b_grouped_nf4_lora_dgrad(const e4b_moe_dims* dims, int32_t T, const e4b_routing* routing,
+                                      const e4b_nf4_experts* base, const e4b_lora* lora,
+                                      const e4b_fwd_buffers* fwd, const e4b_bf16* dY, const e4b_bwd_buffers* bwd,
+                                      e4b_bf16* dx, void* ws, size_t ws_bytes, e4b_stream_t stream) {
+  E4B_TRY(check_dims(dims, T));
+  E4B_TRY(check_ws(dims, T, ws, ws_bytes));
+  E4B_TRY(check_routing(routing));
+  E4B_TRY(check_base(base));
+  E4B_TRY(check_lora(lora));
+  E4B_TRY(check_fwd(fwd));
+  E4B_TRY(check_bwd(bwd));
+  if (!aligned16(dY) || !aligned16(dx)) return E4B_ERR_INVALID_ARG;
+  if (T == 0) return E4B_OK;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int E = dims->E, H = dims->H, I = dims->I, r = dims->r, k = dims->top_k;
+  const int64_t N = (int64_t)T * k;
+  const float s = dims->alpha / (float)r;
+  DeviceError* err = static_cast<DeviceError*>(ws);
+
+  // dyw[row] = w(slot) * dY[token]
+  E4B_CUDA(launch_gather_rows(dY, routing->slot_of_row, routing->tiles, routing->topk_w, H, k, rows_cap(N, E),
+                              bwd->dyw, sms, st));
+  LoraProjHost lp{};
+  lp.E = E;
+  lp.r = r;
+  lp.r_pad = r_padded(r);
+  lp.scale = s;
+  lp.tiles = routing->tiles;
+  lp.rows_cap = rows_cap(N, E);
+  lp.mt_cap = mtiles_cap(N, E);
+  lp.err = err;
+  lp.timeout_ns = kDefaultTimeoutNs;
+  Nf4GemmHost g{};
+  g.E = E;
+  g.H = H;
+  g.I = I;
+  g.r = r;
+  g.r_pad = r_padded(r);
+  g.tiles = routing->tiles;
+  g.rows_cap = lp.rows_cap;
+  g.mt_cap = lp.mt_cap;
+  g.err = err;
+  g.timeout_ns = kDefaultTimeoutNs;
+
+  // q_d = s * dyw B_d
+  lp.act_in = bwd->dyw;
+  lp.K = H;
+  lp.w = lora->B_d;
+  lp.w_mn_major = true;
+  lp.out = bwd->q_d;
+  E4B_CUDA(launch_lora_proj(lp, sms, st));
+  // dact = dyw W_d + q_d A_d ; dgu = SwiGLU backward(dact, gu)
+  g.mode = kDgradDown;
+  g.nf4 = base->down_nf4;
+  g.absmax = base->down_absmax;
+  g.stored_rows = H;
+  g.stored_cols = I;
+  g.act_in = bwd->dyw;
+  g.K = H;
+  g.n_dim = I;
+  g.lora_a_rows = bwd->q_d;
+  g.lora_w = lora->A_d;
+  g.out0 = bwd->dgu;
+  g.out1 = nullptr;
+  g.aux = fwd->gu;
+  E4B_CUDA(launch_nf4_gemm(g, sms, st));
+  // q_gu = s * dgu B_gu
+  lp.act_in = bwd->dgu;
+  lp.K = 2 * I;
+  lp.w = lora->B_gu;
+  lp.out = bwd->q_gu;
+  E4B_CUDA(launch_lora_proj(lp, sms, st));
+  // dx_perm = dgu W_gu + q_gu A_gu
+  g.mode = kDgradGateUp;
+  g.nf4 = base->gate_up_nf4;
+  g.absmax = base->gate_up_absmax;
+  g.stored_rows = 2 * I;
+  g.stored_cols = H;
+  g.act_in = bwd->dgu;
+  g.K = 2 * I;
+  g.n_dim = H;
+  g.lora_a_rows = bwd->q_gu;
+  g.lora_w = lora->A_gu;
+  g.out0 = bwd->dx_perm;
+  g.aux = nullptr;
+  E4B_CUDA(launch_nf4_gemm(g, sms, st));
+  // dx[t] = sum_j dx_perm[row(t,j)]
+  E4B_CUDA(launch_combine(bwd->dx_perm, routing->row_of_slot, nullptr, T, k, H, dx, sms, st));
+  return E4B_OK;
+}
+
+e4b_status e4b_lora_wgrad(const e4b_moe_dims* dims, int32_t T, const e4b_routing* routing,
+                          const e4b_fwd_buffers* fwd, const e4b_bwd_buffers* bwd, e4b_bf16* dA_gu, e4b_bf16* dB_gu,
+                          e4b_bf16* dA_d, e4b_bf16* dB_d, void* ws, size_t ws_bytes, e4b_stream_t stream) {
+  E4B_TRY(check_dims(dims, T));
+  E4B_TRY(check_ws(dims, T, ws, ws_bytes));
+  E4B_TRY(check_routing(routing));
+  E4B_TRY(check_fwd(fwd));
+  E4B_TRY(check_bwd(bwd));
+  if (!aligned16(dA_gu) || !aligned16(dB_gu) || !aligned16(dA_d) || !aligned16(dB_d)) return E4B_ERR_INVALID_ARG;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  const int E = dims->E, H = dims->H, I = dims->I, r = dims->r;
+  const int64_t N = (int64_t)T * dims->top_k;
+  if (T == 0) {
+    // No tokens: every gradient is exactly zero.
+    const cudaStream_t st = (cudaStream_t)stream;
+    E4B_CUDA(cudaMemsetAsync(dB_gu, 0, (size_t)E * 2 * I * r * 2, st));
+    E4B_CUDA(cudaMemsetAsync(dA_gu, 0, (size_t)E * r * H * 2, st));
+    E4B_CUDA(cudaMemsetAsync(dB_d, 0, (size_t)E * H * r * 2, st));
+    E4B_CUDA(cudaMemsetAsync(dA_d, 0, (size_t)E * r * I * 2, st));
+    return E4B_OK;
+  }
+  WgradHost w{};
+  w.act[0] = bwd->dgu;  // dB_gu = dgu^T p_gu
+  w.low[0] = fwd->p_gu;
+  w.out[0] = dB_gu;
+  w.F[0] = 2 * I;
+  w.transposed[0] = false;
+  w.act[1] = fwd->x_perm;  // dA_gu = (x^T q_gu)^T
+  w.low[1] = bwd->q_gu;
+  w.out[1] = dA_gu;
+  w.F[1] = H;
+  w.transposed[1] = true;
+  w.act[2] = bwd->dyw;  // dB_d = dyw^T p_d
+  w.low[2] = fwd->p_d;
+  w.out[2] = dB_d;
+  w.F[2] = H;
+  w.transposed[2] = false;
+  w.act[3] = fwd->act;  // dA_d = (act^T q_d)^T
+  w.low[3] = bwd->q_d;
+  w.out[3] = dA_d;
+  w.F[3] = I;
+  w.transposed[3] = true;
+  w.E = E;
+  w.r = r;
+  w.r_pad = r_padded(r);
+  w.counts = routing->counts;
+  w.offsets = routing->offsets;
+  w.tiles = routing->tiles;
+  w.rows_cap = rows_cap(N, E);
+  w.mt_cap = mtiles_cap(N, E);
+  w.err = static_cast<DeviceError*>(ws);
+  w.timeout_ns = kDefaultTimeoutNs;
+  E4B_CUDA(launch_wgrad(w, sms, (cudaStream_t)stream));
+  return E4B_OK;
+}
+
+e4b_status e4b_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n, e4b_bf16* out,
+                           e4b_stream_t stream) {
+  if (n < 0 || n % 64) return E4B_ERR_INVALID_ARG;
+  if (n == 0) return E4B_OK;
+  if (!aligned16(packed) || absmax == nullptr || (reinterpret_cast<uintptr_t>(absmax) & 3u) || !aligned16(out))
+    return E4B_ERR_INVALID_ARG;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  E4B_CUDA(launch_nf4_dequant(packed, absmax, n, out, sms, (cudaStream_t)stream));
+  return E4B_OK;
+}
+
+e4b_status e4b_debug_watchdog(void* ws, size_t ws_bytes, int64_t timeout_ns, e4b_stream_t stream) {
+  if (!aligned16(ws) || ws_bytes < sizeof(DeviceError) || timeout_ns <= 0 || timeout_ns > 10000000000LL)
+    return E4B_ERR_INVALID_ARG;
+  E4B_CUDA(launch_watchdog(static_cast<DeviceError*>(ws), (long long)timeout_ns, (cudaStream_t)stream));
+  return E4B_OK;
+}
+
+}  // extern "C"

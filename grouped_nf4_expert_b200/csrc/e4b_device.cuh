@@ -1,0 +1,341 @@
+// Device-side building blocks for sm_100a: mbarriers with bounded waits,
+// TMA tile loads, tcgen05 (TMEM allocation, UMMA, commit, TMEM loads),
+// shared-memory matrix descriptors, and the NF4 block decoder.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/e4b.h"
+
+namespace e4b {
+
+// ----------------------------------------------------------------------------
+// Device error word (first bytes of the caller's workspace).
+// ----------------------------------------------------------------------------
+struct DeviceError {
+  int code;       // 0 or an e4b_status
+  int site;       // which wait gave up (kernel-specific id)
+  int block;      // blockIdx.x of the first CTA that gave up
+  int pad[61];    // keeps the rest of the workspace 256-byte aligned
+};
+static_assert(sizeof(DeviceError) == 256, "error word block must be 256 bytes");
+
+// Waits give up after this many nanoseconds by default (about a second).
+constexpr long long kDefaultTimeoutNs = 2000000000LL;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_error(DeviceError* err, int code, int site) {
+  if (err != nullptr) {
+    if (atomicCAS(&err->code, 0, code) == 0) {
+      err->site = site;
+      err->block = blockIdx.x;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ----------------------------------------------------------------------------
+// mbarrier
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Shared control block of a CTA: an abort flag that every bounded wait
+// watches, so that when one role gives up the others stop too.
+struct CtaControl {
+  volatile int abort;
+  int pad;
+};
+
+// Waits for the phase with `parity` of `bar` to complete.  Gives up (returns
+// false) when `timeout_ns` elapses or another thread of the CTA has given up;
+// a thread that gives up records E4B_ERR_DEVICE_TIMEOUT with `site`.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, CtaControl* ctl,
+                                          DeviceError* err, long long timeout_ns, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (ctl->abort) return false;
+    if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
+      ctl->abort = 1;
+      record_error(err, E4B_ERR_DEVICE_TIMEOUT, site);
+      return false;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Proxy fences
+// ----------------------------------------------------------------------------
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor core reads through UMMA descriptors).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), tile mode, no multicast.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// tcgen05: TMEM allocation, UMMA, commit, TMEM -> registers
+// ----------------------------------------------------------------------------
+// Whole warp: allocates `ncols` TMEM columns (power of two >= 32) and writes
+// the base address to `dst`.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulation.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives once on `bar` when every UMMA this thread issued so far completes.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// Each thread of a warp reads 16 consecutive fp32 columns of its TMEM lane.
+// The warp may only address lanes 32*(warp%4) .. +31.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ----------------------------------------------------------------------------
+// UMMA descriptors
+// ----------------------------------------------------------------------------
+// Swizzle modes of the shared-memory matrix descriptor (bits 61-63).
+enum : uint32_t { kSwNone = 0, kSw128 = 2, kSw64 = 4, kSw32 = 6 };
+
+// Shared-memory matrix descriptor.  `lbo` and `sbo` are byte offsets:
+//  K-major, swizzled: sbo = stride between 8-row groups; lbo unused.
+//  MN-major, swizzled: lbo = stride between MN atoms (atom = swizzle width),
+//                      sbo = stride between 8-row K groups.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t swz) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)(swz & 7u) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                   // D format: f32
+         | (1u << 7)                                 // A format: bf16
+         | (1u << 10)                                // B format: bf16
+         | ((a_mn_major ? 1u : 0u) << 15)            // A major-ness
+         | ((b_mn_major ? 1u : 0u) << 16)            // B major-ness
+         | ((uint32_t)(N >> 3) << 17)                // N / 8
+         | ((uint32_t)(M >> 4) << 24);               // M / 16
+}
+
+// Swizzle mode for a row of `row_bytes` (32, 64 or 128).
+__host__ __device__ constexpr uint32_t swz_for_row_bytes(int row_bytes) {
+  return row_bytes == 128 ? kSw128 : (row_bytes == 64 ? kSw64 : kSw32);
+}
+
+// ----------------------------------------------------------------------------
+// bf16 helpers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (bits 0-15), .y = hi
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// ----------------------------------------------------------------------------
+// NF4 decode.
+// A weight is bf16_rn(float32(level[code]) * float32(absmax)).  For one block
+// of 64 codes the 16 possible products are formed once (16 float32 multiplies,
+// rounded to bf16), split into a low-byte plane and a high-byte plane, and
+// every code then becomes a byte-permute lookup: exact by construction.
+// ----------------------------------------------------------------------------
+// The NF4 levels (QLoRA's NormalFloat-4 code book, as printed in its appendix).
+__host__ __device__ __forceinline__ float nf4_level(int c) {
+  constexpr float kLevels[16] = {-1.0f,
+                                 -0.6961928009986877f,
+                                 -0.5250730514526367f,
+                                 -0.39491748809814453f,
+                                 -0.28444138169288635f,
+                                 -0.18477343022823334f,
+                                 -0.09105003625154495f,
+                                 0.0f,
+                                 0.07958029955625534f,
+                                 0.16093020141124725f,
+                                 0.24611230194568634f,
+                                 0.33791524171829224f,
+                                 0.44070982933044434f,
+                                 0.5626170039176941f,
+                                 0.7229568362236023f,
+                                 1.0f};
+  return kLevels[c];
+}
+
+struct Nf4Planes {
+  uint32_t lo[4];  // lo[g] = low bytes of the bf16 products of levels 4g..4g+3
+  uint32_t hi[4];  // hi[g] = high bytes of the same
+};
+
+__device__ __forceinline__ Nf4Planes nf4_block_planes(float absmax) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = __fmul_rn(nf4_level(2 * i), absmax);
+    const float b = __fmul_rn(nf4_level(2 * i + 1), absmax);
+    pk[i] = pack_bf16x2(a, b);
+  }
+  Nf4Planes p;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    p.lo[g] = prmt(pk[2 * g], pk[2 * g + 1], 0x6420u);
+    p.hi[g] = prmt(pk[2 * g], pk[2 * g + 1], 0x7531u);
+  }
+  return p;
+}
+
+// Decodes the 8 codes of one little-endian 32-bit word (bytes b0..b3,
+// element 2m = high nibble of byte m) into 4 bf16x2 words holding elements
+// (0,1), (2,3), (4,5), (6,7) -- lower element in the low half.
+__device__ __forceinline__ void nf4_decode_word(uint32_t w, const Nf4Planes& p, uint32_t* out) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    // Selector nibbles i = 0..3 hold the codes of elements 1, 0, 3, 2 of this half.
+    const uint32_t s = (h == 0) ? w : (w >> 16);
+    const uint32_t s_hi = s ^ 0x8888u;                       // codes 8..15 -> 0..7
+    const uint32_t pick = ((s >> 1) & 0x4444u) | 0x3210u;    // byte i from the 0..7 or 8..15 lookup
+    const uint32_t xl = prmt(p.lo[0], p.lo[1], s);
+    const uint32_t yl = prmt(p.lo[2], p.lo[3], s_hi);
+    const uint32_t xh = prmt(p.hi[0], p.hi[1], s);
+    const uint32_t yh = prmt(p.hi[2], p.hi[3], s_hi);
+    const uint32_t fl = prmt(xl, yl, pick);
+    const uint32_t fh = prmt(xh, yh, pick);
+    out[2 * h] = prmt(fl, fh, 0x4051u);
+    out[2 * h + 1] = prmt(fl, fh, 0x6273u);
+  }
+}
+
+// Decodes one block: 32 bytes of codes (as 8 words) -> 64 bf16 (32 words).
+__device__ __forceinline__ void nf4_decode_block(const uint32_t (&codes)[8], float absmax, uint32_t (&out)[32]) {
+  const Nf4Planes p = nf4_block_planes(absmax);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) nf4_decode_word(codes[i], p, &out[4 * i]);
+}
+
+// Writes 64 bf16 (one 128-byte row of a 128B-swizzled atom) to shared memory:
+// row `row` of the 8-row group starting at `base` + (row/8)*1024; 16-byte chunk
+// c goes to chunk c ^ (row % 8).
+__device__ __forceinline__ void st_swizzled_row128(uint8_t* base, int row, const uint32_t (&v)[32]) {
+  uint8_t* rp = base + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 q = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = q;
+  }
+}
+
+}  // namespace e4b

@@ -1,0 +1,108 @@
+// Internal interface between the C-ABI layer (e4b_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/e4b.h"
+
+namespace e4b {
+
+// Tokens handled by one CTA of the routing kernels.
+constexpr int kRouteTokensPerBlock = 256;
+// Header ints at the front of the tile list: [0] = m-tiles, [1] = rows used.
+constexpr int kTileHeader = 8;
+
+// Tile list layout (int32): header, then (expert, first row) per 128-row
+// m-tile, then the experts ordered by descending token count.
+inline int64_t mtiles_cap(int64_t N, int E) { return (N + 127) / 128 + E; }
+inline int64_t tiles_cap(int64_t N, int E) { return kTileHeader + 2 * mtiles_cap(N, E) + E; }
+inline int64_t rows_cap(int64_t N, int E) { return ((N + (int64_t)E * 127) + 127) / 128 * 128; }
+
+struct DeviceError;
+
+// ---- routing (route.cu)
+cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, int H, int k,
+                         int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
+                         int32_t* row_of_slot, int32_t* slot_of_row, int32_t* tiles, int64_t mt_cap,
+                         uint16_t* x_perm, int64_t rows_cap, int32_t* scratch, int num_sms,
+                         cudaStream_t stream);
+
+// dst[row] = src[token of row] (optionally scaled by the slot's routing weight), zero for padding rows.
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, const int32_t* tiles,
+                               const float* scale_w, int H, int k, int64_t rows_cap, uint16_t* dst,
+                               int num_sms, cudaStream_t stream);
+
+// out[t] = sum_j (w[t,j] or 1) * src_perm[row(t,j)] in float32, rounded once to bf16.
+cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot, const float* topk_w, int T,
+                           int k, int H, uint16_t* out, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n, uint16_t* out,
+                               int num_sms, cudaStream_t stream);
+
+cudaError_t launch_watchdog(DeviceError* err, long long timeout_ns, cudaStream_t stream);
+
+// ---- grouped GEMMs (gemm.cu)
+enum Nf4Mode { kFwdGateUp = 0, kFwdDown = 1, kDgradDown = 2, kDgradGateUp = 3 };
+
+struct Nf4GemmHost {
+  int mode;
+  int E, H, I, r, r_pad;
+  const uint8_t* nf4;      // stored stack [E, rows, cols/2]
+  const float* absmax;     // [E, rows, cols/64]
+  int stored_rows, stored_cols;
+  const uint16_t* act_in;  // A operand [rows_cap, K]
+  int K;                   // reduction length
+  int n_dim;               // output columns
+  const uint16_t* lora_a_rows;  // p or q [rows_cap, r]
+  const uint16_t* lora_w;       // LoRA weight used as the B operand of the K = r step
+  uint16_t* out0;          // gu | y_perm | dgu | dx_perm
+  uint16_t* out1;          // act (forward gate_up) or nullptr
+  const uint16_t* aux;     // saved gu (down dgrad) or nullptr
+  const int32_t* tiles;
+  int64_t rows_cap, mt_cap;
+  DeviceError* err;
+  long long timeout_ns;
+};
+cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stream);
+
+struct LoraProjHost {
+  const uint16_t* act_in;  // [rows_cap, K]
+  int K;
+  const uint16_t* w;       // LoRA factor: A [E, r, K] (k_major) or B [E, K, r] (mn_major)
+  bool w_mn_major;
+  int E, r, r_pad;
+  float scale;
+  uint16_t* out;           // [rows_cap, r]
+  const int32_t* tiles;
+  int64_t rows_cap, mt_cap;
+  DeviceError* err;
+  long long timeout_ns;
+};
+cudaError_t launch_lora_proj(const LoraProjHost& h, int num_sms, cudaStream_t stream);
+
+struct WgradHost {
+  // four products dOut_g[e] = Act_g[e rows]^T * Low_g[e rows]
+  const uint16_t* act[4];  // [rows_cap, F_g]
+  const uint16_t* low[4];  // [rows_cap, r]
+  uint16_t* out[4];        // [E, F_g, r] (transposed = false) or [E, r, F_g] (transposed = true)
+  int F[4];
+  bool transposed[4];
+  int E, r, r_pad;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* tiles;
+  int64_t rows_cap, mt_cap;
+  DeviceError* err;
+  long long timeout_ns;
+};
+cudaError_t launch_wgrad(const WgradHost& h, int num_sms, cudaStream_t stream);
+
+// Tensor-map encoding through the driver entry point (no link-time libcuda).
+cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                              CUtensorMapSwizzle swizzle);
+
+}  // namespace e4b

@@ -1,0 +1,951 @@
+// Grouped GEMMs on the 5th-generation tensor cores (tcgen05, TMEM
+// accumulators, TMA-fed shared memory) for the NF4 expert block:
+//
+//  * nf4_gemm_kernel: one 128x128 output tile per work unit of a grouped
+//    GEMM whose B operand is a frozen NF4 expert matrix, dequantised into
+//    shared memory by a decode warpgroup (bit-exact bf16 weights), with the
+//    LoRA term as an extra K = r MMA into the same TMEM accumulator.  Four
+//    modes: forward gate_up (SiLU-gated epilogue), forward down, down dgrad
+//    (transposed base, SwiGLU backward epilogue), gate_up dgrad.
+//  * lora_proj_kernel: s * (rows x LoRA factor) -> [rows, r], the low-rank
+//    projections p = s x A^T and q = s dy B.
+//  * wgrad_kernel: variable-K grouped GEMM for the LoRA weight gradients
+//    (K = the rows of one expert).
+//
+// Pages: "How do I QLoRA-train the fused experts of a MoE", section "The
+// abstraction that fails" (pre-activation per-expert delta over the fused
+// stacks), section "Why it happens" (scaling * (x @ A.T) @ B.T; the base is
+// re-dequantised in backward), section "Which project solves it" (grouped
+// forward and a dgrad kernel); package METADATA "The package family"
+// (in-register decode of 4-bit stacks, fp32 accumulation).
+#include <math.h>
+
+#include "e4b_device.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+
+__device__ __forceinline__ void store_bf16x16(uint16_t* dst, const uint32_t (&w)[8]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+__device__ __forceinline__ void load_bf16x16(const uint16_t* src, float (&v)[16]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  const uint4 a = __ldg(s), b = __ldg(s + 1);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = bf16lo_to_f32(w[i]);
+    v[2 * i + 1] = bf16hi_to_f32(w[i]);
+  }
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+}  // namespace
+
+// =============================================================================
+// NF4 grouped GEMM
+// =============================================================================
+namespace nf4g {
+constexpr int BM = 128, BN = 128, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                        // activation tile, K-major SW128
+constexpr int B_BYTES = BN * BK * 2;                        // dequantised weight tile
+constexpr int RAW_BYTES = BN * BK / 2;                      // NF4 codes as loaded
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;  // 36 KB, 1024-aligned
+constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;             // p or q tile
+constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;             // LoRA weight tile
+constexpr int BAR_BYTES = 1024;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LA_BYTES + LB_BYTES + BAR_BYTES + 1024;
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-7 decode, warps 8-11 epilogue
+constexpr int kTmemCols = 128;
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+}  // namespace nf4g
+
+struct Nf4GemmParams {
+  const float* absmax;
+  const int32_t* tiles;
+  uint16_t* out0;
+  uint16_t* out1;
+  const uint16_t* aux;
+  DeviceError* err;
+  long long timeout_ns;
+  int K, n_dim, I, r_pad;
+  int stored_rows, stored_cols;
+  int n_nt;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(nf4g::kThreads, 1)
+    nf4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_raw,
+                    const __grid_constant__ CUtensorMap map_la, const __grid_constant__ CUtensorMap map_lb,
+                    const Nf4GemmParams p) {
+  using namespace nf4g;
+  constexpr bool kMN = (MODE == kDgradDown || MODE == kDgradGateUp);  // B operand N-contiguous
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = align1024(smem_dyn);
+  uint8_t* stages = smem;
+  uint8_t* la = smem + STAGES * STAGE_BYTES;
+  uint8_t* lb = la + LA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lb + LB_BYTES);
+  uint64_t* full = bars;                 // TMA: activation tile + NF4 codes landed
+  uint64_t* bfull = bars + STAGES;       // decode: dequantised tile written
+  uint64_t* empty = bars + 2 * STAGES;   // MMA: stage consumed
+  uint64_t* lfull = bars + 3 * STAGES;   // TMA: LoRA operands landed
+  uint64_t* lempty = lfull + 1;          // MMA: LoRA operands consumed
+  uint64_t* accfull = lfull + 2;         // MMA: accumulator complete
+  uint64_t* accempty = lfull + 3;        // epilogue: accumulator drained
+  uint64_t* drain = lfull + 4;           // MMA: all issued UMMAs finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 5);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 6);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&bfull[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(lfull, 1);
+    mbar_init(lempty, 1);
+    mbar_init(accfull, 1);
+    mbar_init(accempty, 4);
+    mbar_init(drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_units = p.tiles[0] * p.n_nt;
+  const int kchunks = p.K / BK;
+
+  // Stored rows of the B tile (row-major stacks, K-major modes): two 64-row halves.
+  auto kmajor_rows = [&](int nt, int& rA, int& rB) {
+    if (MODE == kFwdGateUp) {
+      rA = nt * 64;
+      rB = p.I + nt * 64;
+    } else {
+      rA = nt * 128;
+      rB = nt * 128 + 64;
+    }
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_raw);
+      tma_prefetch_desc(&map_la);
+      tma_prefetch_desc(&map_lb);
+      int s = 0;
+      uint32_t ph = 0, tph = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int mt = u / p.n_nt, nt = u % p.n_nt;
+        const int e = p.tiles[kTileHeader + 2 * mt], row0 = p.tiles[kTileHeader + 2 * mt + 1];
+        int rA = 0, rB = 0;
+        if (!kMN) kmajor_rows(nt, rA, rB);
+        if (!(ok = mbar_wait(lempty, tph ^ 1, ctl, p.err, p.timeout_ns, 10))) break;
+        mbar_arrive_expect_tx(lfull, 512u * p.r_pad);
+        tma_load_2d(la, &map_la, lfull, 0, row0);
+        if (!kMN) {
+          tma_load_3d(lb, &map_lb, lfull, 0, rA, e);
+          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, 0, rB, e);
+        } else {
+          tma_load_3d(lb, &map_lb, lfull, nt * 128, 0, e);
+          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, nt * 128 + 64, 0, e);
+        }
+        tph ^= 1;
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 11))) break;
+          uint8_t* st = stages + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], A_BYTES + RAW_BYTES);
+          tma_load_2d(st, &map_a, &full[s], kc * BK, row0);
+          if (!kMN) {
+            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, &full[s], kc * (BK / 2), rA, e);
+            tma_load_3d(st + A_BYTES + B_BYTES + RAW_BYTES / 2, &map_raw, &full[s], kc * (BK / 2), rB, e);
+          } else {
+            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, &full[s], nt * (BN / 2), kc * BK, e);
+          }
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let copies already issued land before the CTA's shared memory goes away.
+        for (int i = 0; i < STAGES; ++i)
+          if (issued & (1u << i)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
+                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(BM, BN, false, kMN);
+      const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
+      const uint32_t la_u = smem_u32(la), lb_u = smem_u32(lb);
+      int s = 0;
+      uint32_t ph = 0, tph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        if (!(ok = mbar_wait(accempty, tph ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
+        tc_fence_after();
+        if (!(ok = mbar_wait(lfull, tph, ctl, p.err, p.timeout_ns, 21))) break;
+        tc_fence_after();
+        // LoRA step first: acc = (s*p) * B_lora^T over K = r (overwrites the accumulator).
+        for (int ks = 0; ks < p.r_pad / 16; ++ks) {
+          const uint64_t ad = make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz);
+          const uint64_t bd = kMN ? make_sdesc(lb_u + 2048 * ks, 128 * p.r_pad, 1024, kSw128)
+                                  : make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz);
+          umma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(lempty);
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 22))) break;
+          if (!(ok = mbar_wait(&bfull[s], ph, ctl, p.err, p.timeout_ns, 23))) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(stages + s * STAGE_BYTES);
+          const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = make_sdesc(a0 + 32 * kk, 16, 1024, kSw128);
+            const uint64_t bd =
+                kMN ? make_sdesc(b0 + 2048 * kk, 8192, 1024, kSw128) : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
+            umma_bf16(tmem, ad, bd, idesc, 1u);
+          }
+          umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(accfull);
+        tph ^= 1;
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ NF4 decode
+    const int t = threadIdx.x - 128;
+    const int blocks_per_row = p.stored_cols / 64;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int mt = u / p.n_nt, nt = u % p.n_nt;
+      const int e = p.tiles[kTileHeader + 2 * mt];
+      int rA = 0, rB = 0;
+      if (!kMN) kmajor_rows(nt, rA, rB);
+      for (int kc = 0; kc < kchunks; ++kc) {
+        int srow, sblk;
+        bool valid;
+        if (!kMN) {
+          srow = (t < 64) ? rA + t : rB + (t - 64);
+          sblk = kc;
+          valid = srow < p.stored_rows;
+        } else {
+          srow = kc * BK + (t & 63);
+          sblk = nt * 2 + (t >> 6);
+          valid = sblk < blocks_per_row;
+        }
+        const float amax =
+            valid ? __ldg(p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk) : 0.0f;
+        ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 30);
+        ok = __all_sync(kFull, ok);
+        if (!ok) break;
+        uint8_t* st = stages + s * STAGE_BYTES;
+        const uint8_t* raw = st + A_BYTES + B_BYTES + (kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32);
+        uint32_t v[32];
+        if (valid) {
+          const uint4 q0 = *reinterpret_cast<const uint4*>(raw);
+          const uint4 q1 = *reinterpret_cast<const uint4*>(raw + 16);
+          const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          nf4_decode_block(codes, amax, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (!kMN)
+          st_swizzled_row128(st + A_BYTES, t, v);
+        else
+          st_swizzled_row128(st + A_BYTES + (t >> 6) * 8192, t & 63, v);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bfull[s]);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ epilogue
+    const int q = threadIdx.x - 256;  // tile row == TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint32_t tph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int mt = u / p.n_nt, nt = u % p.n_nt;
+      const size_t row = (size_t)p.tiles[kTileHeader + 2 * mt + 1] + q;
+      ok = mbar_wait(accfull, tph, ctl, p.err, p.timeout_ns, 40);
+      ok = __all_sync(kFull, ok);
+      if (!ok) break;
+      tc_fence_after();
+      if (MODE == kFwdGateUp) {
+        const int I2 = 2 * p.I, c0 = nt * 64;
+#pragma unroll 1
+        for (int j = 0; j < 64; j += 16) {
+          float g[16], up[16];
+          tmem_ld16(tl + j, g);
+          tmem_ld16(tl + 64 + j, up);
+          uint32_t gw[8], uw[8], aw[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            gw[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+            uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
+            aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
+          }
+          store_bf16x16(p.out0 + row * I2 + c0 + j, gw);
+          store_bf16x16(p.out0 + row * I2 + p.I + c0 + j, uw);
+          store_bf16x16(p.out1 + row * p.I + c0 + j, aw);
+        }
+      } else if (MODE == kDgradDown) {
+        const int I2 = 2 * p.I, c0 = nt * 128;
+#pragma unroll 1
+        for (int j = 0; j < 128; j += 16) {
+          if (c0 + j >= p.I) break;
+          float da[16], g[16], up[16];
+          tmem_ld16(tl + j, da);
+          load_bf16x16(p.aux + row * I2 + c0 + j, g);
+          load_bf16x16(p.aux + row * I2 + p.I + c0 + j, up);
+          uint32_t dgw[8], duw[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float dg[2], du[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float gg = g[2 * i + h], uu = up[2 * i + h], d = da[2 * i + h];
+              const float sg = 1.0f / (1.0f + __expf(-gg));
+              dg[h] = d * uu * sg * (1.0f + gg * (1.0f - sg));
+              du[h] = d * gg * sg;
+            }
+            dgw[i] = pack_bf16x2(dg[0], dg[1]);
+            duw[i] = pack_bf16x2(du[0], du[1]);
+          }
+          store_bf16x16(p.out0 + row * I2 + c0 + j, dgw);
+          store_bf16x16(p.out0 + row * I2 + p.I + c0 + j, duw);
+        }
+      } else {
+        const int c0 = nt * 128;
+#pragma unroll 1
+        for (int j = 0; j < 128; j += 16) {
+          if (c0 + j >= p.n_dim) break;
+          float v[16];
+          tmem_ld16(tl + j, v);
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          store_bf16x16(p.out0 + row * p.n_dim + c0 + j, w);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty);
+      tph ^= 1;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// =============================================================================
+// LoRA projection: out[rows, r] = bf16(scale * act[rows, K] . W_e)
+// =============================================================================
+namespace lproj {
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BK * E4B_MAX_RANK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 24 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kTmemCols = 64;
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+}  // namespace lproj
+
+struct LoraProjParams {
+  const int32_t* tiles;
+  uint16_t* out;
+  DeviceError* err;
+  long long timeout_ns;
+  float scale;
+  int K, r, r_pad;
+};
+
+template <bool W_MN>
+__global__ void __launch_bounds__(lproj::kThreads)
+    lora_proj_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_w,
+                     const LoraProjParams p) {
+  using namespace lproj;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = align1024(smem_dyn);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* accfull = bars + 2 * STAGES;
+  uint64_t* accempty = accfull + 1;
+  uint64_t* drain = accfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 3);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accempty, 4);
+    mbar_init(drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_units = p.tiles[0];
+  const int kchunks = p.K / BK;
+  const uint32_t b_bytes = BK * p.r_pad * 2;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&map_act);
+      tma_prefetch_desc(&map_w);
+      int s = 0;
+      uint32_t ph = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int e = p.tiles[kTileHeader + 2 * u], row0 = p.tiles[kTileHeader + 2 * u + 1];
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 110))) break;
+          uint8_t* st = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], A_BYTES + b_bytes);
+          tma_load_2d(st, &map_act, &full[s], kc * BK, row0);
+          if (W_MN)
+            tma_load_3d(st + A_BYTES, &map_w, &full[s], 0, kc * BK, e);
+          else
+            tma_load_3d(st + A_BYTES, &map_w, &full[s], kc * BK, 0, e);
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < STAGES; ++i)
+          if (issued & (1u << i)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
+                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(BM, p.r_pad, false, W_MN);
+      const uint32_t wswz = swz_for_row_bytes(2 * p.r_pad);
+      int s = 0;
+      uint32_t ph = 0, tph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        if (!(ok = mbar_wait(accempty, tph ^ 1, ctl, p.err, p.timeout_ns, 120))) break;
+        tc_fence_after();
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 121))) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES), b0 = a0 + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = make_sdesc(a0 + 32 * kk, 16, 1024, kSw128);
+            const uint64_t bd = W_MN ? make_sdesc(b0 + 32 * p.r_pad * kk, b_bytes, 16 * p.r_pad, wswz)
+                                     : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
+            umma_bf16(tmem, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(accfull);
+        tph ^= 1;
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+      }
+    }
+  } else {
+    const int q = ((warp & 3) << 5) | lane;  // TMEM lane of this thread
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint32_t tph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const size_t row = (size_t)p.tiles[kTileHeader + 2 * u + 1] + q;
+      ok = mbar_wait(accfull, tph, ctl, p.err, p.timeout_ns, 130);
+      ok = __all_sync(kFull, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int j = 0; j < p.r_pad; j += 16) {
+        float v[16];
+        tmem_ld16(tl + j, v);
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(p.scale * v[2 * i], p.scale * v[2 * i + 1]);
+        uint4* d = reinterpret_cast<uint4*>(p.out + row * p.r + j);
+        if (j < p.r) d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (j + 8 < p.r) d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty);
+      tph ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// =============================================================================
+// LoRA weight gradients: out_g[e] = act_g[rows of e]^T . low_g[rows of e]
+// =============================================================================
+namespace wg {
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BK * BM * 2;            // 64 rows x 128 features, MN-major SW128
+constexpr int B_BYTES = BK * E4B_MAX_RANK * 2;  // 64 rows x r_pad, MN-major
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 64;
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+}  // namespace wg
+
+struct WgradParams {
+  uint16_t* out[4];
+  int F[4];
+  int n_ft[4];
+  int transposed_mask;
+  int units_per_expert;
+  int E, r, r_pad;
+  int64_t mt_cap;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* tiles;
+  DeviceError* err;
+  long long timeout_ns;
+};
+
+struct WgradUnit {
+  int g, ft, e, nk;
+};
+
+__device__ __forceinline__ WgradUnit wgrad_unit(const WgradParams& p, int u) {
+  WgradUnit w;
+  const int erank = u / p.units_per_expert;
+  int rem = u - erank * p.units_per_expert;
+  w.g = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+    if (w.g == i && rem >= p.n_ft[i]) {
+      rem -= p.n_ft[i];
+      w.g = i + 1;
+    }
+  w.ft = rem;
+  w.e = p.tiles[kTileHeader + 2 * p.mt_cap + erank];
+  w.nk = ((p.counts[w.e] + 127) / 128) * 2;  // 64-row K chunks over the padded group
+  return w;
+}
+
+__global__ void __launch_bounds__(wg::kThreads)
+    wgrad_kernel(const __grid_constant__ CUtensorMap act0, const __grid_constant__ CUtensorMap act1,
+                 const __grid_constant__ CUtensorMap act2, const __grid_constant__ CUtensorMap act3,
+                 const __grid_constant__ CUtensorMap low0, const __grid_constant__ CUtensorMap low1,
+                 const __grid_constant__ CUtensorMap low2, const __grid_constant__ CUtensorMap low3,
+                 const WgradParams p) {
+  using namespace wg;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = align1024(smem_dyn);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* accfull = bars + 2 * STAGES;
+  uint64_t* accempty = accfull + 1;
+  uint64_t* drain = accfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 3);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accempty, 4);
+    mbar_init(drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_units = p.E * p.units_per_expert;
+  const uint32_t b_bytes = BK * p.r_pad * 2;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const CUtensorMap* amaps[4] = {&act0, &act1, &act2, &act3};
+      const CUtensorMap* lmaps[4] = {&low0, &low1, &low2, &low3};
+      int s = 0;
+      uint32_t ph = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const WgradUnit w = wgrad_unit(p, u);
+        const int row0 = p.offsets[w.e];
+        for (int kc = 0; kc < w.nk; ++kc) {
+          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 210))) break;
+          uint8_t* st = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], A_BYTES + b_bytes);
+          tma_load_2d(st, amaps[w.g], &full[s], w.ft * BM, row0 + kc * BK);
+          tma_load_2d(st + A_BYTES / 2, amaps[w.g], &full[s], w.ft * BM + 64, row0 + kc * BK);
+          tma_load_2d(st + A_BYTES, lmaps[w.g], &full[s], 0, row0 + kc * BK);
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < STAGES; ++i)
+          if (issued & (1u << i)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
+                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(BM, p.r_pad, true, true);
+      const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
+      int s = 0;
+      uint32_t ph = 0, tph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const WgradUnit w = wgrad_unit(p, u);
+        if (!(ok = mbar_wait(accempty, tph ^ 1, ctl, p.err, p.timeout_ns, 220))) break;
+        tc_fence_after();
+        for (int kc = 0; kc < w.nk; ++kc) {
+          if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 221))) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES), b0 = a0 + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = make_sdesc(a0 + 2048 * kk, A_BYTES / 2, 1024, kSw128);
+            const uint64_t bd = make_sdesc(b0 + 32 * p.r_pad * kk, b_bytes, 16 * p.r_pad, lswz);
+            umma_bf16(tmem, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(accfull);
+        tph ^= 1;
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+      }
+    }
+  } else {
+    const int q = ((warp & 3) << 5) | lane;
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint32_t tph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const WgradUnit w = wgrad_unit(p, u);
+      ok = mbar_wait(accfull, tph, ctl, p.err, p.timeout_ns, 230);
+      ok = __all_sync(kFull, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int F = p.F[w.g];
+      const int m = w.ft * BM + q;
+      const bool tr = (p.transposed_mask >> w.g) & 1;
+      uint16_t* out = p.out[w.g];
+#pragma unroll 1
+      for (int j = 0; j < p.r_pad; j += 16) {
+        float v[16];
+        if (w.nk > 0) {
+          tmem_ld16(tl + j, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+        }
+        if (m < F) {
+          if (!tr) {
+            uint32_t pw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pw[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            uint4* d = reinterpret_cast<uint4*>(out + ((size_t)w.e * F + m) * p.r + j);
+            if (j < p.r) d[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            if (j + 8 < p.r) d[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (j + i < p.r) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(v[i]);
+                out[((size_t)w.e * p.r + j + i) * F + m] = *reinterpret_cast<const uint16_t*>(&b);
+              }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty);
+      tph ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// =============================================================================
+// Host-side launchers
+// =============================================================================
+namespace {
+
+CUtensorMapSwizzle swizzle_for_bytes(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// 2-D bf16 matrix [rows, cols] row-major.
+cudaError_t map_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                        uint32_t box_rows, CUtensorMapSwizzle swz) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 2};
+  const uint32_t box[2] = {box_cols, box_rows};
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, swz);
+}
+
+// 3-D bf16 stack [E, rows, cols].
+cudaError_t map_bf16_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
+                        uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  const uint64_t dims[3] = {cols, rows, E};
+  const uint64_t strides[2] = {cols * 2, cols * rows * 2};
+  const uint32_t box[3] = {box_cols, box_rows, 1};
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, swz);
+}
+
+// 3-D byte stack [E, rows, bytes].
+cudaError_t map_u8_3d(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t rows, uint64_t E,
+                      uint32_t box_bytes, uint32_t box_rows) {
+  const uint64_t dims[3] = {bytes, rows, E};
+  const uint64_t strides[2] = {bytes, bytes * rows};
+  const uint32_t box[3] = {box_bytes, box_rows, 1};
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stream) {
+  const bool mn = (h.mode == kDgradDown || h.mode == kDgradGateUp);
+  CUtensorMap ma, mraw, mla, mlb;
+  cudaError_t err;
+  if ((err = map_bf16_2d(&ma, h.act_in, h.K, h.rows_cap, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+    return err;
+  if (!mn)
+    err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 32, 64);
+  else
+    err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 64, 64);
+  if (err != cudaSuccess) return err;
+  const CUtensorMapSwizzle rswz = swizzle_for_bytes(2 * h.r_pad);
+  if ((err = map_bf16_2d(&mla, h.lora_a_rows, h.r, h.rows_cap, h.r_pad, 128, rswz)) != cudaSuccess) return err;
+  if (!mn)  // B_lora [E, stored_rows, r], K-major rows
+    err = map_bf16_3d(&mlb, h.lora_w, h.r, h.stored_rows, h.E, h.r_pad, 64, rswz);
+  else  // A_lora [E, r, stored_cols], rows are the K = r dimension
+    err = map_bf16_3d(&mlb, h.lora_w, h.stored_cols, h.r, h.E, 64, h.r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (err != cudaSuccess) return err;
+
+  Nf4GemmParams p;
+  p.absmax = h.absmax;
+  p.tiles = h.tiles;
+  p.out0 = h.out0;
+  p.out1 = h.out1;
+  p.aux = h.aux;
+  p.err = h.err;
+  p.timeout_ns = h.timeout_ns;
+  p.K = h.K;
+  p.n_dim = h.n_dim;
+  p.I = h.I;
+  p.r_pad = h.r_pad;
+  p.stored_rows = h.stored_rows;
+  p.stored_cols = h.stored_cols;
+  p.n_nt = (h.mode == kFwdGateUp) ? h.I / 64 : (h.n_dim + 127) / 128;
+  const int64_t units_max = h.mt_cap * p.n_nt;
+  const int grid = (int)(units_max < num_sms ? units_max : num_sms);
+  const int smem = nf4g::SMEM_BYTES;
+  switch (h.mode) {
+    case kFwdGateUp:
+      if ((err = set_smem(nf4_gemm_kernel<kFwdGateUp>, smem)) != cudaSuccess) return err;
+      nf4_gemm_kernel<kFwdGateUp><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      break;
+    case kFwdDown:
+      if ((err = set_smem(nf4_gemm_kernel<kFwdDown>, smem)) != cudaSuccess) return err;
+      nf4_gemm_kernel<kFwdDown><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      break;
+    case kDgradDown:
+      if ((err = set_smem(nf4_gemm_kernel<kDgradDown>, smem)) != cudaSuccess) return err;
+      nf4_gemm_kernel<kDgradDown><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      break;
+    default:
+      if ((err = set_smem(nf4_gemm_kernel<kDgradGateUp>, smem)) != cudaSuccess) return err;
+      nf4_gemm_kernel<kDgradGateUp><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_proj(const LoraProjHost& h, int num_sms, cudaStream_t stream) {
+  CUtensorMap mact, mw;
+  cudaError_t err;
+  if ((err = map_bf16_2d(&mact, h.act_in, h.K, h.rows_cap, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+    return err;
+  if (h.w_mn_major)  // B [E, K, r]: K rows of r values
+    err = map_bf16_3d(&mw, h.w, h.r, h.K, h.E, h.r_pad, 64, swizzle_for_bytes(2 * h.r_pad));
+  else  // A [E, r, K]: r rows of K values
+    err = map_bf16_3d(&mw, h.w, h.K, h.r, h.E, 64, h.r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (err != cudaSuccess) return err;
+  LoraProjParams p;
+  p.tiles = h.tiles;
+  p.out = h.out;
+  p.err = h.err;
+  p.timeout_ns = h.timeout_ns;
+  p.scale = h.scale;
+  p.K = h.K;
+  p.r = h.r;
+  p.r_pad = h.r_pad;
+  const int64_t cap = (int64_t)num_sms * 2;
+  const int grid = (int)(h.mt_cap < cap ? h.mt_cap : cap);
+  const int smem = lproj::SMEM_BYTES;
+  if (h.w_mn_major) {
+    if ((err = set_smem(lora_proj_kernel<true>, smem)) != cudaSuccess) return err;
+    lora_proj_kernel<true><<<grid, lproj::kThreads, smem, stream>>>(mact, mw, p);
+  } else {
+    if ((err = set_smem(lora_proj_kernel<false>, smem)) != cudaSuccess) return err;
+    lora_proj_kernel<false><<<grid, lproj::kThreads, smem, stream>>>(mact, mw, p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wgrad(const WgradHost& h, int num_sms, cudaStream_t stream) {
+  CUtensorMap ma[4], ml[4];
+  cudaError_t err;
+  WgradParams p;
+  p.units_per_expert = 0;
+  p.transposed_mask = 0;
+  for (int g = 0; g < 4; ++g) {
+    if ((err = map_bf16_2d(&ma[g], h.act[g], h.F[g], h.rows_cap, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+        cudaSuccess)
+      return err;
+    if ((err = map_bf16_2d(&ml[g], h.low[g], h.r, h.rows_cap, h.r_pad, 64, swizzle_for_bytes(2 * h.r_pad))) !=
+        cudaSuccess)
+      return err;
+    p.out[g] = h.out[g];
+    p.F[g] = h.F[g];
+    p.n_ft[g] = (h.F[g] + 127) / 128;
+    p.units_per_expert += p.n_ft[g];
+    if (h.transposed[g]) p.transposed_mask |= 1 << g;
+  }
+  p.E = h.E;
+  p.r = h.r;
+  p.r_pad = h.r_pad;
+  p.mt_cap = h.mt_cap;
+  p.counts = h.counts;
+  p.offsets = h.offsets;
+  p.tiles = h.tiles;
+  p.err = h.err;
+  p.timeout_ns = h.timeout_ns;
+  const int64_t units = (int64_t)h.E * p.units_per_expert;
+  const int64_t cap = (int64_t)num_sms * 2;
+  const int grid = (int)(units < cap ? units : cap);
+  const int smem = wg::SMEM_BYTES;
+  if ((err = set_smem(wgrad_kernel, smem)) != cudaSuccess) return err;
+  wgrad_kernel<<<grid, wg::kThreads, smem, stream>>>(ma[0], ma[1], ma[2], ma[3], ml[0], ml[1], ml[2], ml[3], p);
+  return cudaGetLastError();
+}
+
+}  // namespace e4b

@@ -1,0 +1,357 @@
+// Routing and permutation kernels: top-k + softmax, expert histogram, prefix
+// sums with per-expert padding, the device work list, a deterministic stable
+// scatter, row gathers and the weighted un-permute combine.  Also the NF4
+// dequantisation test kernel and the watchdog self-test.
+//
+// Pages: "How do I QLoRA-train the fused experts of a MoE", section "Which
+// project solves it" (grouped execution of the routed experts) and section
+// "The abstraction that fails" (router frozen: its logits are inputs).
+#include <math.h>
+
+#include "e4b_device.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+
+// NaN ranks lowest; equal values go to the lower expert id.
+__device__ __forceinline__ bool route_better(float av, int ae, float bv, int be) {
+  const bool an = isnan(av), bn = isnan(bv);
+  if (an || bn) return (an && bn) ? (ae < be) : bn;
+  return av > bv || (av == bv && ae < be);
+}
+
+// One warp per token: k rounds of a warp-wide argmax over the unpicked
+// experts, then a softmax over the k selected logits.  The CTA also counts
+// the slots it produced per expert (order-independent shared counters).
+template <int EPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                         int32_t* __restrict__ topk_ids,
+                                                         float* __restrict__ topk_w,
+                                                         int32_t* __restrict__ block_counts) {
+  extern __shared__ int s_cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int t0 = blockIdx.x * kRouteTokensPerBlock;
+  const int t1 = min(T, t0 + kRouteTokensPerBlock);
+  for (int t = t0 + warp; t < t1; t += nwarps) {
+    const float* row = logits + (size_t)t * E;
+    float v[EPL];
+    uint32_t picked = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = (e < E) ? row[e] : 0.0f;
+      if (e >= E) picked |= 1u << i;
+    }
+    float my_v = 0.0f;
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = __int_as_float(0x7fc00000);  // NaN: loses to everything
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        if (!(picked & (1u << i)) && route_better(v[i], lane + 32 * i, bv, be)) {
+          bv = v[i];
+          be = lane + 32 * i;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (route_better(ov, oe, bv, be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) picked |= 1u << (be >> 5);
+      if (lane == j) {
+        my_v = bv;
+        my_e = be;
+      }
+    }
+    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const float z = (lane < k) ? expf(my_v - vmax) : 0.0f;
+    float sum = z;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) {
+      topk_ids[(size_t)t * k + lane] = my_e;
+      topk_w[(size_t)t * k + lane] = z / sum;
+      atomicAdd(&s_cnt[my_e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = s_cnt[e];
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_warp[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += y;
+    }
+    s_warp[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const int before = (warp > 0) ? s_warp[warp - 1] : 0;
+  __syncthreads();
+  return before + x - v;
+}
+
+// One CTA of 1024 threads, one thread per expert: counts, 128-aligned group
+// offsets, per-(CTA, expert) scatter bases, padding markers, the m-tile list
+// and the experts in descending-count order.
+__global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ block_counts, int nblk,
+                                                          int E, int32_t* __restrict__ block_base,
+                                                          int32_t* __restrict__ counts,
+                                                          int32_t* __restrict__ offsets,
+                                                          int32_t* __restrict__ slot_of_row,
+                                                          int32_t* __restrict__ tiles, int64_t mt_cap) {
+  __shared__ int s_warp[32];
+  __shared__ int s_cnt[E4B_MAX_EXPERTS];
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < E)
+    for (int b = 0; b < nblk; ++b) cnt += block_counts[(size_t)b * E + e];
+  const int padded = (cnt + 127) / 128 * 128;
+  const int off = block_exclusive_scan(e < E ? padded : 0, s_warp);
+  const int mt_off = block_exclusive_scan(e < E ? padded / 128 : 0, s_warp);
+  if (e < E) {
+    s_cnt[e] = cnt;
+    counts[e] = cnt;
+    offsets[e] = off;
+    int run = off;
+    for (int b = 0; b < nblk; ++b) {
+      block_base[(size_t)b * E + e] = run;
+      run += block_counts[(size_t)b * E + e];
+    }
+    for (int r = off + cnt; r < off + padded; ++r) slot_of_row[r] = -1;
+    for (int i = 0; i < padded / 128; ++i) {
+      tiles[kTileHeader + 2 * (mt_off + i)] = e;
+      tiles[kTileHeader + 2 * (mt_off + i) + 1] = off + 128 * i;
+    }
+    if (e == E - 1) {
+      offsets[E] = off + padded;
+      tiles[0] = mt_off + padded / 128;
+      tiles[1] = off + padded;
+    }
+  }
+  __syncthreads();
+  if (e < E) {
+    int rank = 0;
+    for (int o = 0; o < E; ++o) rank += (s_cnt[o] > cnt) || (s_cnt[o] == cnt && o < e);
+    tiles[kTileHeader + 2 * mt_cap + rank] = e;
+  }
+}
+
+// Stable scatter: one warp walks its CTA's slots in flat order, 32 at a time;
+// slots of the same expert inside a step are ranked by lane (match_any), and
+// a shared running count per expert carries the rank across steps.
+__global__ void __launch_bounds__(32) route_rank_kernel(const int32_t* __restrict__ topk_ids, int N, int E,
+                                                        int slots_per_block,
+                                                        const int32_t* __restrict__ block_base,
+                                                        int32_t* __restrict__ row_of_slot,
+                                                        int32_t* __restrict__ slot_of_row) {
+  extern __shared__ int s_run[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_run[e] = block_base[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int lane = threadIdx.x;
+  const int f0 = blockIdx.x * slots_per_block;
+  const int f1 = min(N, f0 + slots_per_block);
+  for (int base = f0; base < f1; base += 32) {
+    const int f = base + lane;
+    const bool valid = f < f1;
+    const int e = valid ? topk_ids[f] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int leader = __ffs(peers) - 1;
+    if (valid) {
+      const int row = s_run[e] + rank;
+      row_of_slot[f] = row;
+      slot_of_row[row] = f;
+    }
+    __syncwarp();
+    if (valid && lane == leader) s_run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 q, float w) {
+  uint32_t* p = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = pack_bf16x2(w * bf16lo_to_f32(p[i]), w * bf16hi_to_f32(p[i]));
+  return q;
+}
+
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ src,
+                                                          const int32_t* __restrict__ slot_of_row,
+                                                          const int32_t* __restrict__ tiles,
+                                                          const float* __restrict__ scale_w, int H, int k,
+                                                          uint16_t* __restrict__ dst) {
+  const int rows_used = tiles[1];
+  const int vec = H / 8;
+  for (int row = blockIdx.x; row < rows_used; row += gridDim.x) {
+    const int slot = slot_of_row[row];
+    uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
+    if (slot < 0) {
+      for (int i = threadIdx.x; i < vec; i += blockDim.x) d[i] = make_uint4(0, 0, 0, 0);
+    } else {
+      const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(slot / k) * H);
+      if (scale_w == nullptr) {
+        for (int i = threadIdx.x; i < vec; i += blockDim.x) d[i] = __ldg(s + i);
+      } else {
+        const float w = scale_w[slot];
+        for (int i = threadIdx.x; i < vec; i += blockDim.x) d[i] = scale_bf16x8(__ldg(s + i), w);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ src_perm,
+                                                      const int32_t* __restrict__ row_of_slot,
+                                                      const float* __restrict__ topk_w, int T, int k, int H,
+                                                      uint16_t* __restrict__ out) {
+  __shared__ int s_row[E4B_MAX_TOP_K];
+  __shared__ float s_w[E4B_MAX_TOP_K];
+  const int vec = H / 8;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < k) {
+      s_row[threadIdx.x] = row_of_slot[(size_t)t * k + threadIdx.x];
+      s_w[threadIdx.x] = topk_w ? topk_w[(size_t)t * k + threadIdx.x] : 1.0f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < vec; i += blockDim.x) {
+      float acc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+      for (int j = 0; j < k; ++j) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(src_perm + (size_t)s_row[j] * H) + i);
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(&q);
+        const float w = s_w[j];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[2 * c] += w * bf16lo_to_f32(p[c]);
+          acc[2 * c + 1] += w * bf16hi_to_f32(p[c]);
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out + (size_t)t * H)[i] = o;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restrict__ packed,
+                                                          const float* __restrict__ absmax, int64_t nblocks,
+                                                          uint16_t* __restrict__ out) {
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks;
+       b += (int64_t)gridDim.x * blockDim.x) {
+    const uint4* p = reinterpret_cast<const uint4*>(packed + b * 32);
+    const uint4 q0 = __ldg(p), q1 = __ldg(p + 1);
+    const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    uint32_t v[32];
+    nf4_decode_block(codes, __ldg(absmax + b), v);
+    uint4* o = reinterpret_cast<uint4*>(out + b * 64);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) o[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  }
+}
+
+// Waits on an mbarrier that nothing ever arrives on: the bounded wait must
+// give up, record E4B_ERR_DEVICE_TIMEOUT and let the CTA finish.
+__global__ void watchdog_kernel(DeviceError* err, long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ CtaControl ctl;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, &ctl, err, timeout_ns, /*site=*/1);
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- launchers
+
+cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, int H, int k, int32_t* topk_ids,
+                         float* topk_w, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
+                         int32_t* slot_of_row, int32_t* tiles, int64_t mt_cap, uint16_t* x_perm,
+                         int64_t rows_cap, int32_t* scratch, int num_sms, cudaStream_t stream) {
+  const int nblk = (T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock;
+  int32_t* block_counts = scratch;
+  int32_t* block_base = scratch + (size_t)nblk * E;
+  const size_t smem = (size_t)E * sizeof(int);
+  const int epl = (E + 31) / 32;
+  if (epl <= 1)
+    route_topk_kernel<1><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  else if (epl <= 2)
+    route_topk_kernel<2><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  else if (epl <= 4)
+    route_topk_kernel<4><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  else if (epl <= 8)
+    route_topk_kernel<8><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  else if (epl <= 16)
+    route_topk_kernel<16><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  else
+    route_topk_kernel<32><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  route_scan_kernel<<<1, 1024, 0, stream>>>(block_counts, nblk, E, block_base, counts, offsets, slot_of_row,
+                                            tiles, mt_cap);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  route_rank_kernel<<<nblk, 32, smem, stream>>>(topk_ids, T * k, E, kRouteTokensPerBlock * k, block_base,
+                                                row_of_slot, slot_of_row);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  return launch_gather_rows(x, slot_of_row, tiles, nullptr, H, k, rows_cap, x_perm, num_sms, stream);
+}
+
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, const int32_t* tiles,
+                               const float* scale_w, int H, int k, int64_t rows_cap, uint16_t* dst, int num_sms,
+                               cudaStream_t stream) {
+  const int64_t grid = rows_cap < (int64_t)num_sms * 8 ? rows_cap : (int64_t)num_sms * 8;
+  gather_rows_kernel<<<(int)grid, 256, 0, stream>>>(src, slot_of_row, tiles, scale_w, H, k, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot, const float* topk_w, int T, int k,
+                           int H, uint16_t* out, int num_sms, cudaStream_t stream) {
+  const int grid = T < num_sms * 8 ? T : num_sms * 8;
+  combine_kernel<<<grid, 256, 0, stream>>>(src_perm, row_of_slot, topk_w, T, k, H, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n, uint16_t* out, int num_sms,
+                               cudaStream_t stream) {
+  const int64_t nblocks = n / 64;
+  int64_t grid = (nblocks + 255) / 256;
+  if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
+  if (grid < 1) grid = 1;
+  nf4_dequant_kernel<<<(int)grid, 256, 0, stream>>>(packed, absmax, nblocks, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_watchdog(DeviceError* err, long long timeout_ns, cudaStream_t stream) {
+  watchdog_kernel<<<1, 32, 0, stream>>>(err, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace e4b

@@ -1,0 +1,252 @@
+"""Python binding of the C ABI in ``include/e4b.h`` (ctypes; argument marshalling only).
+
+Every function here forwards to the entry point of the same name in
+``libe4b.so``; all computation runs in that library's CUDA kernels.  Tensors
+are torch CUDA tensors (PyTorch supplies device memory and streams).  A
+non-OK status raises :class:`E4BError`.  There is no fallback: if the library
+is missing, :func:`lib` raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libe4b.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "e4b.h")
+
+c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+STATUS = {0: "E4B_OK", 1: "E4B_ERR_INVALID_ARG", 2: "E4B_ERR_UNSUPPORTED",
+          3: "E4B_ERR_WORKSPACE_TOO_SMALL", 4: "E4B_ERR_CUDA", 5: "E4B_ERR_DEVICE_TIMEOUT"}
+E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_UNSUPPORTED = 0, 1, 2
+E4B_ERR_WORKSPACE_TOO_SMALL, E4B_ERR_CUDA, E4B_ERR_DEVICE_TIMEOUT = 3, 4, 5
+ROW_ALIGN = 128
+
+
+class E4BError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().e4b_status_string(status).decode()
+        super().__init__("%s failed: %s" % (where, msg))
+
+
+class MoeDims(ctypes.Structure):
+    _fields_ = [("E", c_i32), ("H", c_i32), ("I", c_i32), ("top_k", c_i32), ("r", c_i32),
+                ("alpha", c_f32), ("blocksize", c_i32), ("act", c_i32)]
+
+
+class Nf4Experts(ctypes.Structure):
+    _fields_ = [("gate_up_nf4", c_vp), ("gate_up_absmax", c_vp), ("down_nf4", c_vp), ("down_absmax", c_vp)]
+
+
+class Lora(ctypes.Structure):
+    _fields_ = [("A_gu", c_vp), ("B_gu", c_vp), ("A_d", c_vp), ("B_d", c_vp)]
+
+
+class Routing(ctypes.Structure):
+    _fields_ = [("topk_ids", c_vp), ("topk_w", c_vp), ("counts", c_vp), ("offsets", c_vp),
+                ("row_of_slot", c_vp), ("slot_of_row", c_vp), ("tiles", c_vp)]
+
+
+class FwdBuffers(ctypes.Structure):
+    _fields_ = [("x_perm", c_vp), ("p_gu", c_vp), ("gu", c_vp), ("act", c_vp), ("p_d", c_vp), ("y_perm", c_vp)]
+
+
+class BwdBuffers(ctypes.Structure):
+    _fields_ = [("dyw", c_vp), ("q_d", c_vp), ("dgu", c_vp), ("q_gu", c_vp), ("dx_perm", c_vp)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [("slots", c_i64), ("rows_cap", c_i64), ("tiles_cap", c_i64), ("workspace_bytes", c_sz)]
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+_SIGNATURES = {
+    "e4b_status_string": (ctypes.c_char_p, [c_i32]),
+    "e4b_version": (ctypes.c_char_p, []),
+    "e4b_nf4_levels": (None, [ctypes.POINTER(c_f32)]),
+    "e4b_get_sizes": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Sizes)]),
+    "e4b_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
+    "e4b_check_device_error": (c_i32, [c_vp, c_vp]),
+    "e4b_route_permute": (c_i32, [ctypes.POINTER(MoeDims), c_i32, c_vp, c_vp, ctypes.POINTER(Routing), c_vp,
+                                  c_vp, c_sz, c_vp]),
+    "e4b_grouped_nf4_lora_fwd": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
+                                         ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora),
+                                         ctypes.POINTER(FwdBuffers), c_vp, c_vp, c_sz, c_vp]),
+    "e4b_grouped_nf4_lora_dgrad": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
+                                           ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora),
+                                           ctypes.POINTER(FwdBuffers), c_vp, ctypes.POINTER(BwdBuffers), c_vp,
+                                           c_vp, c_sz, c_vp]),
+    "e4b_lora_wgrad": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
+                               ctypes.POINTER(FwdBuffers), ctypes.POINTER(BwdBuffers), c_vp, c_vp, c_vp, c_vp,
+                               c_vp, c_sz, c_vp]),
+    "e4b_nf4_dequant": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
+    "e4b_debug_watchdog": (c_i32, [c_vp, c_sz, c_i64, c_vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Loads ``libe4b.so`` (built in-tree by ``grouped_nf4_expert_b200.build``)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libe4b.so is not built; run `python -m grouped_nf4_expert_b200.build`")
+        so = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(so, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = so
+    return _LIB
+
+
+def header_symbols():
+    """Names of the entry points ``include/e4b.h`` declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:const\s+)?[\w\s\*]*?\b(e4b_\w+)\s*\(", text, flags=re.M)))
+
+
+def _check(status: int, where: str):
+    if status != E4B_OK:
+        raise E4BError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+@dataclass(frozen=True)
+class Dims:
+    E: int
+    H: int
+    I: int  # noqa: E741
+    top_k: int
+    r: int
+    alpha: float
+
+    def c(self) -> MoeDims:
+        return MoeDims(self.E, self.H, self.I, self.top_k, self.r, float(self.alpha), 64, 0)
+
+
+def e4b_get_sizes(dims: Dims, T: int) -> Sizes:
+    out = Sizes()
+    d = dims.c()
+    _check(lib().e4b_get_sizes(ctypes.byref(d), T, ctypes.byref(out)), "e4b_get_sizes")
+    return out
+
+
+def e4b_nf4_levels():
+    buf = (c_f32 * 16)()
+    lib().e4b_nf4_levels(buf)
+    return [buf[i] for i in range(16)]
+
+
+def e4b_workspace_init(ws, stream=None):
+    _check(lib().e4b_workspace_init(_ptr(ws), ws.numel(), _stream(stream)), "e4b_workspace_init")
+
+
+def e4b_check_device_error(ws, stream=None) -> int:
+    """Synchronises the stream; returns the status (does not raise)."""
+    return lib().e4b_check_device_error(_ptr(ws), _stream(stream))
+
+
+def e4b_nf4_dequant(packed, absmax, out, stream=None):
+    _check(lib().e4b_nf4_dequant(_ptr(packed), _ptr(absmax), out.numel(), _ptr(out), _stream(stream)),
+           "e4b_nf4_dequant")
+
+
+def e4b_debug_watchdog(ws, timeout_ns: int, stream=None):
+    _check(lib().e4b_debug_watchdog(_ptr(ws), ws.numel(), int(timeout_ns), _stream(stream)), "e4b_debug_watchdog")
+
+
+class Block:
+    """Device buffers of one block problem (``dims``, ``T`` tokens), allocated with torch.
+
+    Holds the routing arrays, the forward activations, the backward
+    intermediates, the workspace and the outputs, laid out as ``include/e4b.h``
+    requires, and calls the four entry points on them.
+    """
+
+    def __init__(self, dims: Dims, T: int, device="cuda"):
+        import torch
+        self.dims, self.T, self.device = dims, T, torch.device(device)
+        sz = e4b_get_sizes(dims, T)
+        self.sizes = sz
+        E, H, I, k, r = dims.E, dims.H, dims.I, dims.top_k, dims.r
+        R = sz.rows_cap
+        dev = self.device
+
+        def z(shape, dtype):
+            n = 1
+            for s in shape:
+                n *= s
+            return torch.zeros(max(n, 8), dtype=dtype, device=dev)[:n].view(*shape)
+
+        bf, i32, f32 = torch.bfloat16, torch.int32, torch.float32
+        self.topk_ids, self.topk_w = z((T, k), i32), z((T, k), f32)
+        self.counts, self.offsets = z((E,), i32), z((E + 1,), i32)
+        self.row_of_slot, self.slot_of_row, self.tiles = z((T * k,), i32), z((R,), i32), z((sz.tiles_cap,), i32)
+        self.x_perm, self.p_gu, self.gu = z((R, H), bf), z((R, r), bf), z((R, 2 * I), bf)
+        self.act, self.p_d, self.y_perm = z((R, I), bf), z((R, r), bf), z((R, H), bf)
+        self.dyw, self.q_d, self.dgu = z((R, H), bf), z((R, r), bf), z((R, 2 * I), bf)
+        self.q_gu, self.dx_perm = z((R, r), bf), z((R, H), bf)
+        self.y, self.dx = z((T, H), bf), z((T, H), bf)
+        self.dA_gu, self.dB_gu = z((E, r, H), bf), z((E, 2 * I, r), bf)
+        self.dA_d, self.dB_d = z((E, r, I), bf), z((E, H, r), bf)
+        self.ws = z((int(sz.workspace_bytes),), torch.uint8)
+        e4b_workspace_init(self.ws)
+        self._dims_c = dims.c()
+        self._routing = Routing(*(t.data_ptr() for t in (self.topk_ids, self.topk_w, self.counts, self.offsets,
+                                                           self.row_of_slot, self.slot_of_row, self.tiles)))
+        self._fwd = FwdBuffers(*(t.data_ptr() for t in (self.x_perm, self.p_gu, self.gu, self.act, self.p_d,
+                                                         self.y_perm)))
+        self._bwd = BwdBuffers(*(t.data_ptr() for t in (self.dyw, self.q_d, self.dgu, self.q_gu, self.dx_perm)))
+
+    # -- the four hot-path calls -------------------------------------------------
+    def e4b_route_permute(self, logits, x, stream=None):
+        _check(lib().e4b_route_permute(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
+                                       ctypes.byref(self._routing), _ptr(self.x_perm), _ptr(self.ws),
+                                       self.ws.numel(), _stream(stream)), "e4b_route_permute")
+
+    def e4b_grouped_nf4_lora_fwd(self, base: Nf4Experts, lora: Lora, stream=None):
+        _check(lib().e4b_grouped_nf4_lora_fwd(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
+                                              ctypes.byref(base), ctypes.byref(lora), ctypes.byref(self._fwd),
+                                              _ptr(self.y), _ptr(self.ws), self.ws.numel(), _stream(stream)),
+               "e4b_grouped_nf4_lora_fwd")
+
+    def e4b_grouped_nf4_lora_dgrad(self, base: Nf4Experts, lora: Lora, dY, stream=None):
+        _check(lib().e4b_grouped_nf4_lora_dgrad(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
+                                                ctypes.byref(base), ctypes.byref(lora), ctypes.byref(self._fwd),
+                                                _ptr(dY), ctypes.byref(self._bwd), _ptr(self.dx), _ptr(self.ws),
+                                                self.ws.numel(), _stream(stream)), "e4b_grouped_nf4_lora_dgrad")
+
+    def e4b_lora_wgrad(self, stream=None):
+        _check(lib().e4b_lora_wgrad(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
+                                    ctypes.byref(self._fwd), ctypes.byref(self._bwd), _ptr(self.dA_gu),
+                                    _ptr(self.dB_gu), _ptr(self.dA_d), _ptr(self.dB_d), _ptr(self.ws),
+                                    self.ws.numel(), _stream(stream)), "e4b_lora_wgrad")
+
+    def check_device_error(self, stream=None) -> int:
+        return e4b_check_device_error(self.ws, stream)
+
+
+def nf4_experts(gate_up_nf4, gate_up_absmax, down_nf4, down_absmax) -> Nf4Experts:
+    return Nf4Experts(gate_up_nf4.data_ptr(), gate_up_absmax.data_ptr(), down_nf4.data_ptr(),
+                      down_absmax.data_ptr())
+
+
+def lora_factors(A_gu, B_gu, A_d, B_d) -> Lora:
+    return Lora(A_gu.data_ptr(), B_gu.data_ptr(), A_d.data_ptr(), B_d.data_ptr())

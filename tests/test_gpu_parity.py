@@ -1,0 +1,295 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Indices and NF4 dequantisation must match bit for bit; bf16 values must
+satisfy max|gpu - oracle| / max|oracle| <= 1e-2 (fp32 accumulation on the
+GPU, float64 in the oracle); where the oracle is exactly zero the GPU must be
+exactly zero.  Small cases compare every element; the full-size workloads
+compare sampled tokens and experts the oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from grouped_nf4_expert_b200 import build, e4b, inputs
+from grouped_nf4_expert_b200 import device as dv
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+SMALL = {
+    "tiny": inputs.CONFIGS["tiny"],
+    "tiny_b0": inputs.CONFIGS["tiny_b0"],
+    # several tiles per dimension, ragged groups, K loops of several stages
+    "medium": inputs.Config("medium", E=8, H=256, I=384, top_k=2, T=300, r=16, alpha=32.0,
+                            routing="normal", seed=31),
+    # Zipf skew: experts spanning several 128-row tiles next to nearly empty ones; r = 64
+    "medium_zipf_r64": inputs.Config("medium_zipf_r64", E=32, H=512, I=256, top_k=4, T=700, r=64,
+                                     alpha=128.0, routing="zipf", seed=32),
+    # r = 24 (padded to 32), H and I not multiples of 128 (half-empty output tiles)
+    "medium_r24": inputs.Config("medium_r24", E=6, H=192, I=320, top_k=3, T=257, r=24, alpha=48.0,
+                                routing="normal", seed=33),
+}
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built():
+    build.build()
+    e4b.lib()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def rel_err(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    m = np.abs(ref).max() if ref.size else 0.0
+    if m == 0.0:
+        return 0.0 if np.all(gpu == 0) else np.inf
+    return float(np.abs(gpu - ref).max() / m)
+
+
+def f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def oracle_experts(prob):
+    f = lambda b: inputs.bits_to_f32(b).astype(np.float64)  # noqa: E731
+    return oracle.Experts(prob.gate_up_nf4, prob.gate_up_absmax, prob.down_nf4, prob.down_absmax,
+                          f(prob.A_gu), f(prob.B_gu), f(prob.A_d), f(prob.B_d))
+
+
+def run(cfg, fwd=True, dgrad=True, wgrad=True, prob=None):
+    prob = prob if prob is not None else inputs.make_problem(cfg)
+    d = dv.upload(prob)
+    blk = e4b.Block(dv.dims_of(cfg), cfg.T)
+    blk.e4b_route_permute(d.logits, d.x)
+    if fwd:
+        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora())
+    if dgrad:
+        blk.e4b_grouped_nf4_lora_dgrad(d.base(), d.lora(), d.dY)
+    if wgrad:
+        blk.e4b_lora_wgrad()
+    assert blk.check_device_error() == e4b.E4B_OK
+    return prob, d, blk
+
+
+def check_routing(prob, blk):
+    cfg = prob.cfg
+    ids, w = oracle.route_topk(prob.logits, cfg.top_k)
+    g = oracle.group_by_expert(ids, cfg.E)
+    assert np.array_equal(blk.topk_ids.cpu().numpy(), ids)
+    np.testing.assert_allclose(blk.topk_w.cpu().numpy(), w, rtol=4e-6, atol=1e-7)
+    assert np.array_equal(blk.counts.cpu().numpy(), g["counts"])
+    offsets = blk.offsets.cpu().numpy().astype(np.int64)
+    padded = (g["counts"] + 127) // 128 * 128
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), padded)
+    flat = ids.reshape(-1)
+    ros = blk.row_of_slot.cpu().numpy().astype(np.int64)
+    assert np.array_equal(ros - offsets[flat], g["rank"])
+    used = int(offsets[-1])
+    sor = blk.slot_of_row.cpu().numpy()[:used]
+    assert np.array_equal(sor[ros], np.arange(flat.size))
+    pad = np.ones(used, dtype=bool)
+    pad[ros] = False
+    assert np.all(sor[pad] == -1)
+    xp = bits(blk.x_perm)[:used]
+    assert np.array_equal(xp[ros], prob.x[np.arange(flat.size) // cfg.top_k])
+    assert np.all(xp[pad] == 0)
+    tiles = blk.tiles.cpu().numpy()
+    assert tiles[0] == padded.sum() // 128 and tiles[1] == used
+    return ros
+
+
+# --------------------------------------------------------------------- decode
+
+def test_nf4_dequant_bit_exact():
+    rng = np.random.default_rng(0)
+    n = 64 * 8192
+    packed = rng.integers(0, 256, n // 2, dtype=np.uint8)
+    packed[:256] = np.arange(256, dtype=np.uint8)
+    absmax = rng.uniform(0.0, 0.2, n // 64).astype(np.float32)
+    absmax[:12] = np.array([0.0, 1.0, 1e-30, 3e38, 0.5, 2.0 ** -126, 1e-45, 7.5, -0.3, 2.0 ** -149, 1e20, 0.02],
+                           dtype=np.float32)
+    want, _ = oracle.dequantize_nf4(packed.reshape(1, -1), absmax.reshape(1, -1))
+    dp = torch.from_numpy(packed).cuda()
+    da = torch.from_numpy(absmax).cuda()
+    out = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    e4b.e4b_nf4_dequant(dp, da, out)
+    torch.cuda.synchronize()
+    got = bits(out)
+    assert np.array_equal(got, want[0]), np.flatnonzero(got != want[0])[:10]
+
+
+# --------------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_routing_bit_exact_small(name):
+    prob, _, blk = run(SMALL[name], fwd=False, dgrad=False, wgrad=False)
+    check_routing(prob, blk)
+
+
+@pytest.mark.parametrize("name", ["finegrained", "decode", "train"])
+def test_routing_bit_exact_workloads(name):
+    prob, _, blk = run(inputs.CONFIGS[name], fwd=False, dgrad=False, wgrad=False)
+    check_routing(prob, blk)
+
+
+def test_routing_ties_and_deterministic():
+    cfg = inputs.Config("ties", E=16, H=64, I=64, top_k=4, T=500, r=8, alpha=16.0, routing="normal", seed=41)
+    prob = inputs.make_problem(cfg)
+    prob.logits[:] = np.round(prob.logits * 2) / 2  # many exact ties
+    prob.logits[7, :] = 0.0
+    prob.logits[8, 3] = np.nan
+    _, _, a = run(cfg, fwd=False, dgrad=False, wgrad=False, prob=prob)
+    check_routing(prob, a)
+    _, _, b = run(cfg, fwd=False, dgrad=False, wgrad=False, prob=prob)
+    for t in ("topk_ids", "topk_w", "row_of_slot", "slot_of_row", "offsets", "tiles"):
+        assert torch.equal(getattr(a, t), getattr(b, t)), t
+
+
+# --------------------------------------------------------------------- full block, small sizes
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_block_parity_small(name):
+    cfg = SMALL[name]
+    prob, _, blk = run(cfg)
+    ros = check_routing(prob, blk)
+    ex = oracle_experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    s = cfg.alpha / cfg.r
+    fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha)
+    bo = oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha)
+    slots = np.array(sorted(fo["gu"].keys()))
+    rows = ros[slots]
+    errs = {}
+    errs["y"] = rel_err(f64(blk.y), fo["y"])
+    for key, buf, scale in [("gu", blk.gu, 1.0), ("act", blk.act, 1.0), ("p_gu", blk.p_gu, s),
+                            ("p_d", blk.p_d, s), ("yd", blk.y_perm, 1.0)]:
+        errs[key] = rel_err(f64(buf)[rows], np.stack([fo[key][f] for f in slots]) * scale)
+    errs["dx"] = rel_err(f64(blk.dx), bo["dx"])
+    w = bo["w"].reshape(-1)
+    errs["dyw"] = rel_err(f64(blk.dyw)[rows], w[slots, None] * dY[slots // cfg.top_k])
+    for key, buf, scale in [("dgu", blk.dgu, 1.0), ("q_gu", blk.q_gu, s), ("q_d", blk.q_d, s),
+                            ("dx_slot", blk.dx_perm, 1.0)]:
+        errs[key] = rel_err(f64(buf)[rows], np.stack([bo[key][f] for f in slots]) * scale)
+    for key, buf in [("dA_gu", blk.dA_gu), ("dB_gu", blk.dB_gu), ("dA_d", blk.dA_d), ("dB_d", blk.dB_d)]:
+        errs[key] = rel_err(f64(buf), bo[key])
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, (bad, errs)
+
+
+def test_b_zero_delta_is_exactly_zero_on_gpu():
+    cfg = inputs.CONFIGS["tiny_b0"]
+    prob = inputs.make_problem(cfg)
+    _, _, a = run(cfg, dgrad=False, wgrad=False, prob=prob)
+    base_only = inputs.make_problem(cfg)
+    base_only.A_gu[:] = 0
+    base_only.A_d[:] = 0
+    _, _, b = run(cfg, dgrad=False, wgrad=False, prob=base_only)
+    assert np.array_equal(bits(a.y), bits(b.y))
+    assert np.array_equal(bits(a.gu), bits(b.gu))
+
+
+def test_empty_expert_gets_exact_zero_gradients():
+    cfg = SMALL["medium"]
+    prob = inputs.make_problem(cfg)
+    prob.logits[:, 5] = -1e30
+    _, _, blk = run(cfg, prob=prob)
+    assert blk.counts[5].item() == 0
+    for t in (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d):
+        assert torch.count_nonzero(t[5]).item() == 0
+        assert torch.count_nonzero(t[0]).item() > 0
+
+
+def test_frozen_base_bytes_unchanged_and_outputs_deterministic():
+    cfg = SMALL["medium_zipf_r64"]
+    prob = inputs.make_problem(cfg)
+    d = dv.upload(prob)
+    before = [t.clone() for t in (d.gate_up_nf4, d.gate_up_absmax, d.down_nf4, d.down_absmax)]
+    outs = []
+    for _ in range(2):
+        blk = e4b.Block(dv.dims_of(cfg), cfg.T)
+        blk.e4b_route_permute(d.logits, d.x)
+        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora())
+        blk.e4b_grouped_nf4_lora_dgrad(d.base(), d.lora(), d.dY)
+        blk.e4b_lora_wgrad()
+        assert blk.check_device_error() == e4b.E4B_OK
+        outs.append([t.clone() for t in (blk.y, blk.dx, blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d)])
+    for t0, t1 in zip(before, (d.gate_up_nf4, d.gate_up_absmax, d.down_nf4, d.down_absmax)):
+        assert torch.equal(t0, t1)
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_watchdog_times_out_cleanly_and_context_survives():
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    e4b.e4b_workspace_init(ws)
+    e4b.e4b_debug_watchdog(ws, 2_000_000)  # 2 ms
+    assert e4b.e4b_check_device_error(ws) == e4b.E4B_ERR_DEVICE_TIMEOUT
+    e4b.e4b_workspace_init(ws)
+    assert e4b.e4b_check_device_error(ws) == e4b.E4B_OK
+    prob, _, blk = run(inputs.CONFIGS["tiny"], dgrad=False, wgrad=False)
+    assert torch.isfinite(blk.y.float()).all()
+
+
+# --------------------------------------------------------------------- full-size workloads, sampled
+
+def _sample_tokens(T, n, seed):
+    return np.sort(np.random.default_rng(seed).choice(T, size=n, replace=False))
+
+
+@pytest.mark.parametrize("name,ntok", [("finegrained", 24), ("train", 16)])
+def test_workload_fwd_dgrad_sampled_tokens(name, ntok):
+    cfg = inputs.CONFIGS[name]
+    prob, _, blk = run(cfg, wgrad=False)
+    ex = oracle_experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    toks = _sample_tokens(cfg.T, ntok, 100)
+    fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=toks)
+    bo = oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=toks, grad_experts=[])
+    assert rel_err(f64(blk.y)[toks], fo["y"][toks]) <= TOL
+    assert rel_err(f64(blk.dx)[toks], bo["dx"][toks]) <= TOL
+
+
+def test_train_workload_wgrad_sampled_experts():
+    cfg = inputs.CONFIGS["train"]
+    prob, _, blk = run(cfg)
+    counts = blk.counts.cpu().numpy()
+    order = np.argsort(-counts, kind="stable")
+    nz = order[counts[order] > 0]
+    experts = sorted({int(nz[0]), int(nz[len(nz) // 2]), int(nz[-1])})
+    ex = oracle_experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    bo = oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=[], grad_experts=experts)
+    for key, buf in [("dA_gu", blk.dA_gu), ("dB_gu", blk.dB_gu), ("dA_d", blk.dA_d), ("dB_d", blk.dB_d)]:
+        for e in experts:
+            assert rel_err(f64(buf[e]), bo[key][e]) <= TOL, (key, e)
+
+
+def test_decode_workload_full():
+    cfg = inputs.CONFIGS["decode"]
+    prob, _, blk = run(cfg, dgrad=False, wgrad=False)
+    ex = oracle_experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha)
+    assert rel_err(f64(blk.y), fo["y"]) <= TOL
+
+
+def test_mixtral_workload_forward_sampled_tokens():
+    cfg = inputs.CONFIGS["mixtral"]
+    prob, _, blk = run(cfg, dgrad=False, wgrad=False)
+    toks = _sample_tokens(cfg.T, 6, 101)
+    ex = oracle_experts(prob)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=toks)
+    assert rel_err(f64(blk.y)[toks], fo["y"][toks]) <= TOL

@@ -1,0 +1,130 @@
+"""The C-ABI library builds, loads and exports what include/e4b.h declares (CPU only).
+
+No compute entry point is called with valid arguments here: every call below
+fails host-side validation before any CUDA call, which is what is tested.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+
+from conftest import read_golden_floats
+from grouped_nf4_expert_b200 import build as e4b_build
+from grouped_nf4_expert_b200 import e4b
+
+
+@pytest.fixture(scope="module")
+def so():
+    e4b_build.build()
+    return e4b.lib()
+
+
+def test_exports_every_declared_symbol(so):
+    names = e4b.header_symbols()
+    assert len(names) >= 12
+    for required in ("e4b_route_permute", "e4b_grouped_nf4_lora_fwd", "e4b_grouped_nf4_lora_dgrad",
+                     "e4b_lora_wgrad", "e4b_nf4_dequant", "e4b_get_sizes"):
+        assert required in names
+    for n in names:
+        assert hasattr(so, n), n
+
+
+def test_levels_are_the_published_nf4_table(so):
+    lv = np.array(e4b.e4b_nf4_levels(), dtype=np.float32)
+    pub = np.array(read_golden_floats("nf4_levels_qlora.txt"), dtype=np.float32)
+    assert np.array_equal(lv.view(np.uint32), pub.view(np.uint32))
+
+
+def test_status_strings(so):
+    for code, name in e4b.STATUS.items():
+        assert so.e4b_status_string(code).decode().startswith(name)
+    assert b"e4b" in so.e4b_version()
+
+
+def test_sizes_for_the_workloads(so):
+    d = e4b.Dims(E=128, H=2048, I=768, top_k=8, r=64, alpha=128.0)
+    s = e4b.e4b_get_sizes(d, 8192)
+    assert s.slots == 65536
+    assert s.rows_cap % 128 == 0 and s.rows_cap >= 65536 + 128 * 127
+    assert s.workspace_bytes >= 256
+    s0 = e4b.e4b_get_sizes(d, 0)
+    assert s0.slots == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("H", 96, e4b.E4B_ERR_UNSUPPORTED), ("I", 0, e4b.E4B_ERR_UNSUPPORTED), ("top_k", 0, e4b.E4B_ERR_UNSUPPORTED),
+    ("top_k", 5, e4b.E4B_ERR_UNSUPPORTED), ("r", 12, e4b.E4B_ERR_UNSUPPORTED), ("r", 72, e4b.E4B_ERR_UNSUPPORTED),
+    ("E", 0, e4b.E4B_ERR_UNSUPPORTED), ("E", 2048, e4b.E4B_ERR_UNSUPPORTED),
+    ("blocksize", 32, e4b.E4B_ERR_UNSUPPORTED), ("act", 1, e4b.E4B_ERR_UNSUPPORTED),
+    ("alpha", float("nan"), e4b.E4B_ERR_INVALID_ARG),
+])
+def test_bad_dims_are_refused(so, field, value, status):
+    d = e4b.MoeDims(4, 64, 128, 2, 8, 16.0, 64, 0)
+    setattr(d, field, value)
+    out = e4b.Sizes()
+    assert so.e4b_get_sizes(ctypes.byref(d), 32, ctypes.byref(out)) == status
+
+
+def test_negative_tokens_refused(so):
+    d = e4b.MoeDims(4, 64, 128, 2, 8, 16.0, 64, 0)
+    out = e4b.Sizes()
+    assert so.e4b_get_sizes(ctypes.byref(d), -1, ctypes.byref(out)) == e4b.E4B_ERR_INVALID_ARG
+
+
+def _fake(n=64):
+    # Host memory standing in for device pointers: validation reads only the
+    # addresses, never the memory, and fails before any CUDA call.
+    buf = (ctypes.c_uint8 * (n * 16 + 16))()
+    base = (ctypes.addressof(buf) + 15) & ~15
+    return buf, [base + 16 * i for i in range(n)]
+
+
+def test_null_and_misaligned_pointers_refused(so):
+    keep, p = _fake()
+    d = e4b.MoeDims(4, 64, 128, 2, 8, 16.0, 64, 0)
+    T = 32
+    sz = e4b.Sizes()
+    assert so.e4b_get_sizes(ctypes.byref(d), T, ctypes.byref(sz)) == 0
+    routing = e4b.Routing(*p[0:7])
+    ws, wsb = p[10], sz.workspace_bytes
+    # valid-looking call shape but a null logits pointer
+    assert so.e4b_route_permute(ctypes.byref(d), T, None, p[8], ctypes.byref(routing), p[9], ws, wsb,
+                                None) == e4b.E4B_ERR_INVALID_ARG
+    # misaligned x
+    assert so.e4b_route_permute(ctypes.byref(d), T, p[7], p[8] + 2, ctypes.byref(routing), p[9], ws, wsb,
+                                None) == e4b.E4B_ERR_INVALID_ARG
+    # workspace too small
+    assert so.e4b_route_permute(ctypes.byref(d), T, p[7], p[8], ctypes.byref(routing), p[9], ws, 16,
+                                None) == e4b.E4B_ERR_WORKSPACE_TOO_SMALL
+    # routing struct with a null member
+    bad = e4b.Routing(*p[0:6], None)
+    assert so.e4b_route_permute(ctypes.byref(d), T, p[7], p[8], ctypes.byref(bad), p[9], ws, wsb,
+                                None) == e4b.E4B_ERR_INVALID_ARG
+    base = e4b.Nf4Experts(p[11], p[12], None, p[14])
+    lora = e4b.Lora(*p[15:19])
+    fwd = e4b.FwdBuffers(*p[19:25])
+    assert so.e4b_grouped_nf4_lora_fwd(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(base),
+                                       ctypes.byref(lora), ctypes.byref(fwd), p[25], ws, wsb,
+                                       None) == e4b.E4B_ERR_INVALID_ARG
+    bwd = e4b.BwdBuffers(*p[26:30], p[30] + 8)
+    base_ok = e4b.Nf4Experts(*p[11:15])
+    assert so.e4b_grouped_nf4_lora_dgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(base_ok),
+                                         ctypes.byref(lora), ctypes.byref(fwd), p[31], ctypes.byref(bwd), p[32],
+                                         ws, wsb, None) == e4b.E4B_ERR_INVALID_ARG
+    bwd_ok = e4b.BwdBuffers(*p[26:31])
+    assert so.e4b_lora_wgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(fwd), ctypes.byref(bwd_ok),
+                             p[33], None, p[35], p[36], ws, wsb, None) == e4b.E4B_ERR_INVALID_ARG
+    # unsupported dims are refused before pointers are looked at
+    d.r = 12
+    assert so.e4b_lora_wgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(fwd), ctypes.byref(bwd_ok),
+                             p[33], p[34], p[35], p[36], ws, wsb, None) == e4b.E4B_ERR_UNSUPPORTED
+
+
+def test_dequant_and_watchdog_argument_checks(so):
+    keep, p = _fake()
+    assert so.e4b_nf4_dequant(p[0], p[1], 100, p[2], None) == e4b.E4B_ERR_INVALID_ARG  # not a multiple of 64
+    assert so.e4b_nf4_dequant(p[0] + 1, p[1], 64, p[2], None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_nf4_dequant(p[0], p[1], 0, p[2], None) == e4b.E4B_OK  # nothing to do
+    assert so.e4b_debug_watchdog(p[0], 256, 0, None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_debug_watchdog(p[0], 8, 1000, None) == e4b.E4B_ERR_INVALID_ARG
