@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""Throughput of one QLoRA training step of the grouped NF4 expert block.
+
+A step is one pass of the whole hot path over one batch: routing and
+permutation, the grouped NF4+LoRA forward (gate_up with the SiLU-gated
+epilogue, down, combine), the input gradient (down dgrad with the SwiGLU
+backward, gate_up dgrad, un-permute) and the LoRA weight gradients -- the
+four C-ABI calls of libe4b.so.  Default workload: E=128, H=2048, I=768,
+top-8, T=8192 tokens per GPU, LoRA r=64, alpha=128, Zipf(1.1) routing.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+bounded token samples of the same workload instead.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-block fwd+bwd tokens/s and TFLOP/s at 1 B200; % of tensor/HBM roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["e4b", "reference"], default="e4b")
+    ap.add_argument("--workload", default="train")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=24,
+                    help="tokens of the oracle's cpu_baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=1, help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def step_flops(cfg):
+    """Algorithmic FLOPs of one step: routed slots only, 2 FLOP per MAC."""
+    N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
+    base = 12.0 * N * H * I                  # fwd gate_up + down, dgrad down + gate_up
+    lora = 3 * 2.0 * N * r * (2 * H + 3 * I)  # projections and K=r products, fwd + dgrad + wgrad
+    return base + lora
+
+
+def nf4_gemm_flops(cfg):
+    """Algorithmic FLOPs of the four grouped NF4 GEMM launches of one step."""
+    N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
+    return {
+        "nf4_gemm_fwd_gate_up": 2.0 * N * H * 2 * I + 2.0 * N * r * 2 * I,
+        "nf4_gemm_fwd_down": 2.0 * N * I * H + 2.0 * N * r * H,
+        "nf4_gemm_dgrad_down": 2.0 * N * H * I + 2.0 * N * r * I,
+        "nf4_gemm_dgrad_gate_up": 2.0 * N * 2 * I * H + 2.0 * N * r * H,
+    }
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons of one GPU through NVML."""
+
+    def __init__(self, torch_device, period_s=0.01):
+        self.samples, self.period, self.ok = [], period_s, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device).uuid).replace("GPU-", "")
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid:
+                    self.h = h
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = self.h is not None
+        except Exception as exc:  # clocks are reported as unavailable, never guessed
+            self.err = repr(exc)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                watts = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((mhz, reasons, watts))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        mask = 0
+        for s in self.samples:
+            mask |= s[1]
+        reasons = [name for bit, name in NVML_REASONS.items() if mask & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "power_w_max": max(s[2] for s in self.samples)}
+
+
+# --------------------------------------------------------------------------- oracle legs
+
+def oracle_sample_step(prob, tokens):
+    """The CPU oracle as it stands on a token sample: forward + backward (dx and the
+    sample's LoRA-gradient contributions), dequantising the base in both passes."""
+    import numpy as np
+
+    import oracle
+    from grouped_nf4_expert_b200 import inputs
+    cfg = prob.cfg
+    f = lambda b: inputs.bits_to_f32(b).astype(np.float64)  # noqa: E731
+    ex = oracle.Experts(prob.gate_up_nf4, prob.gate_up_absmax, prob.down_nf4, prob.down_absmax,
+                        f(prob.A_gu), f(prob.B_gu), f(prob.A_d), f(prob.B_d))
+    x, dY = f(prob.x), f(prob.dY)
+    oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=tokens)
+    oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=tokens, grad_experts=[])
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(prob, n_tokens):
+    import numpy as np
+    toks = np.sort(np.random.default_rng(7).choice(prob.cfg.T, size=n_tokens, replace=False))
+    t0 = time.perf_counter()
+    oracle_sample_step(prob, toks)
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": "%d random tokens of the %s workload, forward + backward (input gradient and "
+                      "their LoRA-gradient terms), float64 numpy, %.1f s" % (n_tokens, prob.cfg.name, dt)}
+
+
+def run_reference(args):
+    from grouped_nf4_expert_b200 import inputs
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = inputs.CONFIGS[args.workload]
+    prob = inputs.make_problem(cfg)
+    import numpy as np
+    rng = np.random.default_rng(11)
+    times = []
+    for i in range(args.warmup + args.steps):
+        toks = np.sort(rng.choice(cfg.T, size=args.ref_tokens, replace=False))
+        t0 = time.perf_counter()
+        oracle_sample_step(prob, toks)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.ref_tokens * args.steps / total
+    cores = blas_threads()
+    sample = "%d random tokens per step of the %s workload, forward + backward, float64 numpy" % (
+        args.ref_tokens, cfg.name)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, args.gpus, "host memory"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, world, l2_note):
+    return {"workload": "%s: %s" % (cfg.name, cfg.note), "E": cfg.E, "H": cfg.H, "I": cfg.I,
+            "top_k": cfg.top_k, "tokens_per_gpu": cfg.T, "global_batch": cfg.T * world, "r": cfg.r,
+            "alpha": cfg.alpha, "routing": cfg.routing, "nf4_blocksize": 64, "parallelism": "dp%d" % world,
+            "l2": l2_note}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from grouped_nf4_expert_b200 import build, e4b, inputs
+    from grouped_nf4_expert_b200 import device as dv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    e4b.lib()
+
+    cfg = inputs.CONFIGS[args.workload]
+    prob = inputs.make_problem(cfg, data_rank=rank)
+    d = dv.upload(prob, dev)
+    blk = e4b.Block(dv.dims_of(cfg), cfg.T, dev)
+    base, lora = d.base(), d.lora()
+    grads = (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d)
+
+    def step():
+        blk.e4b_route_permute(d.logits, d.x)
+        blk.e4b_grouped_nf4_lora_fwd(base, lora)
+        blk.e4b_grouped_nf4_lora_dgrad(base, lora, d.dY)
+        blk.e4b_lora_wgrad()
+        if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
+            for g in grads:
+                dist.all_reduce(g)
+
+    def sync_all():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # 2x the 126 MB L2
+    for _ in range(max(args.warmup, 3)):
+        step()
+    st = blk.check_device_error()
+    if st != e4b.E4B_OK:
+        raise RuntimeError("device error after warm-up: %s" % e4b.STATUS.get(st, st))
+
+    def timed(K, body):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        sync_all()
+        for i in range(K):
+            flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
+            evs[i][0].record()
+            body()
+            evs[i][1].record()
+        sync_all()
+        ms = sum(a.elapsed_time(b) for a, b in evs)
+        if world > 1:
+            t = torch.tensor([ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    # ---- main timed region
+    launches0 = e4b.e4b_launch_count()
+    with ClockSampler(dev) as clocks:
+        total_ms = timed(args.steps, step)
+    launches = e4b.e4b_launch_count() - launches0
+    st = blk.check_device_error()
+    if st != e4b.E4B_OK:
+        raise RuntimeError("device error in the timed region: %s" % e4b.STATUS.get(st, st))
+    ms_per_step = total_ms / args.steps
+    value = cfg.T * world * args.steps / (total_ms / 1e3)
+    flops = step_flops(cfg)
+
+    # ---- per-kernel device times over a second timed region (library profiler, events on the launch stream)
+    e4b.e4b_profiler_enable(True)
+    prof_ms = timed(args.steps, step)
+    e4b.e4b_profiler_enable(False)
+    kern = e4b.e4b_profiler_read()
+    peaks, peak_src = load_peaks()
+    gflops = nf4_gemm_flops(cfg)
+    nf4_ms = sum(kern.get(n, (0, 0.0))[1] for n in gflops)
+    nf4_launches = sum(kern.get(n, (0, 0.0))[0] for n in gflops)
+    nf4_flop = sum(gflops.values()) * args.steps
+    achieved = nf4_flop / (nf4_ms / 1e3) / 1e12 if nf4_ms > 0 else None
+    kern_total = sum(v[1] for v in kern.values())
+    roofline = {"kernel": "nf4_gemm (fwd gate_up, fwd down, dgrad down, dgrad gate_up)", "bound": "tensor",
+                "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
+                "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long step)" % peak_src,
+                "traffic": None, "launches": nf4_launches,
+                "avg_launch_ms": nf4_ms / max(nf4_launches, 1),
+                "algorithmic_flop_per_step": sum(gflops.values())}
+    per_kernel = {n: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
+                      "share": v[1] / kern_total if kern_total else None} for n, v in kern.items()}
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
+    hx, hl, hdy = pin(d.x), pin(d.logits), pin(d.dY)
+    hx.copy_(d.x)
+    hl.copy_(d.logits)
+    hdy.copy_(d.dY)
+    outs = [blk.y, blk.dx, blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d]
+    houts = [pin(t) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hl, hdy))
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+
+    def e2e_step():
+        d.x.copy_(hx, non_blocking=True)
+        d.logits.copy_(hl, non_blocking=True)
+        d.dY.copy_(hdy, non_blocking=True)
+        step()
+        for h, t in zip(houts, outs):
+            h.copy_(t, non_blocking=True)
+
+    e2e_ms = timed(args.steps, e2e_step)
+    e2e = {"value": cfg.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(cfg, world, "flushed between timed steps by a 256 MiB write"),
+        "tflops": flops * world / (ms_per_step / 1e3) / 1e12,
+        "step_flop_per_gpu": flops,
+        "roofline": roofline,
+        "kernels": per_kernel,
+        "profiled_ms_per_step": prof_ms / args.steps,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(prob, args.cpu_sample_tokens)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -4,7 +4,11 @@
 // synchronises.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <atomic>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 #include <string.h>
 
 #include "e4b_device.cuh"
@@ -142,6 +146,47 @@ cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int r
                               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// ---- launch counting and optional per-kernel event timing
+namespace {
+struct ProfRecord {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof_records;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
+std::atomic<int64_t> g_launches{0};
+}  // namespace
+
+LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : name_(name), stream_(stream), slot_(-1) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (!g_prof_on) return;
+  std::pair<cudaEvent_t, cudaEvent_t> ev;
+  if (!g_prof_pool.empty()) {
+    ev = g_prof_pool.back();
+    g_prof_pool.pop_back();
+  } else if (cudaEventCreate(&ev.first) != cudaSuccess || cudaEventCreate(&ev.second) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return;
+  }
+  if (cudaEventRecord(ev.first, stream_) != cudaSuccess) {
+    (void)cudaGetLastError();
+    g_prof_pool.push_back(ev);
+    return;
+  }
+  slot_ = (int)g_prof_records.size();
+  g_prof_records.push_back({name_, ev.first, ev.second});
+}
+
+LaunchScope::~LaunchScope() {
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (slot_ < (int)g_prof_records.size() && cudaEventRecord(g_prof_records[slot_].stop, stream_) != cudaSuccess)
+    (void)cudaGetLastError();
 }
 
 }  // namespace e4b
@@ -465,6 +510,51 @@ e4b_status e4b_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n
   E4B_CUDA(launch_nf4_dequant(packed, absmax, n, out, sms, (cudaStream_t)stream));
   return E4B_OK;
 }
+
+e4b_status e4b_profiler_enable(int32_t on) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  g_prof_on = on != 0;
+  return E4B_OK;
+}
+
+e4b_status e4b_profiler_read(e4b_kernel_time* out, int32_t capacity, int32_t* count) {
+  if (count == nullptr || capacity < 0 || (capacity > 0 && out == nullptr)) return E4B_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  std::map<std::string, std::pair<int64_t, double>> acc;
+  std::vector<std::string> order;
+  e4b_status st = E4B_OK;
+  for (const ProfRecord& r : g_prof_records) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      (void)cudaGetLastError();
+      st = E4B_ERR_CUDA;
+    }
+    auto it = acc.find(r.name);
+    if (it == acc.end()) {
+      order.push_back(r.name);
+      acc[r.name] = {1, (double)ms};
+    } else {
+      it->second.first += 1;
+      it->second.second += ms;
+    }
+    g_prof_pool.push_back({r.start, r.stop});
+  }
+  g_prof_records.clear();
+  int n = 0;
+  for (const std::string& name : order) {
+    if (n < capacity) {
+      memset(out[n].name, 0, sizeof(out[n].name));
+      strncpy(out[n].name, name.c_str(), sizeof(out[n].name) - 1);
+      out[n].launches = acc[name].first;
+      out[n].total_ms = acc[name].second;
+    }
+    ++n;
+  }
+  *count = n;
+  return st;
+}
+
+int64_t e4b_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 e4b_status e4b_debug_watchdog(void* ws, size_t ws_bytes, int64_t timeout_ns, e4b_stream_t stream) {
   if (!aligned16(ws) || ws_bytes < sizeof(DeviceError) || timeout_ns <= 0 || timeout_ns > 10000000000LL)

@@ -23,6 +23,19 @@ inline int64_t rows_cap(int64_t N, int E) { return ((N + (int64_t)E * 127) + 127
 
 struct DeviceError;
 
+// Brackets one kernel launch: counts it and, while the profiler is on,
+// records CUDA events around it on `stream`.
+class LaunchScope {
+ public:
+  LaunchScope(const char* name, cudaStream_t stream);
+  ~LaunchScope();
+
+ private:
+  const char* name_;
+  cudaStream_t stream_;
+  int slot_;
+};
+
 // ---- routing (route.cu)
 cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, int H, int k,
                          int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,

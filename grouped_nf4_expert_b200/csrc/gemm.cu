@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
     }
   }
 
+  __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the CTA barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -553,6 +554,7 @@ __global__ void __launch_bounds__(lproj::kThreads)
       tph ^= 1;
     }
   }
+  __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the CTA barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -769,6 +771,7 @@ __global__ void __launch_bounds__(wg::kThreads)
       tph ^= 1;
     }
   }
+  __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the CTA barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -858,6 +861,9 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
   const int64_t units_max = h.mt_cap * p.n_nt;
   const int grid = (int)(units_max < num_sms ? units_max : num_sms);
   const int smem = nf4g::SMEM_BYTES;
+  static const char* kNames[4] = {"nf4_gemm_fwd_gate_up", "nf4_gemm_fwd_down", "nf4_gemm_dgrad_down",
+                                  "nf4_gemm_dgrad_gate_up"};
+  LaunchScope scope(kNames[h.mode & 3], stream);
   switch (h.mode) {
     case kFwdGateUp:
       if ((err = set_smem(nf4_gemm_kernel<kFwdGateUp>, smem)) != cudaSuccess) return err;
@@ -901,6 +907,7 @@ cudaError_t launch_lora_proj(const LoraProjHost& h, int num_sms, cudaStream_t st
   const int64_t cap = (int64_t)num_sms * 2;
   const int grid = (int)(h.mt_cap < cap ? h.mt_cap : cap);
   const int smem = lproj::SMEM_BYTES;
+  LaunchScope scope("lora_proj", stream);
   if (h.w_mn_major) {
     if ((err = set_smem(lora_proj_kernel<true>, smem)) != cudaSuccess) return err;
     lora_proj_kernel<true><<<grid, lproj::kThreads, smem, stream>>>(mact, mw, p);
@@ -944,6 +951,7 @@ cudaError_t launch_wgrad(const WgradHost& h, int num_sms, cudaStream_t stream) {
   const int grid = (int)(units < cap ? units : cap);
   const int smem = wg::SMEM_BYTES;
   if ((err = set_smem(wgrad_kernel, smem)) != cudaSuccess) return err;
+  LaunchScope scope("lora_wgrad", stream);
   wgrad_kernel<<<grid, wg::kThreads, smem, stream>>>(ma[0], ma[1], ma[2], ma[3], ml[0], ml[1], ml[2], ml[3], p);
   return cudaGetLastError();
 }

@@ -301,6 +301,8 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
   int32_t* block_base = scratch + (size_t)nblk * E;
   const size_t smem = (size_t)E * sizeof(int);
   const int epl = (E + 31) / 32;
+  {
+  LaunchScope scope("route_topk", stream);
   if (epl <= 1)
     route_topk_kernel<1><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else if (epl <= 2)
@@ -313,13 +315,20 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
     route_topk_kernel<16><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else
     route_topk_kernel<32><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+  }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  route_scan_kernel<<<1, 1024, 0, stream>>>(block_counts, nblk, E, block_base, counts, offsets, slot_of_row,
-                                            tiles, mt_cap);
+  {
+    LaunchScope scope("route_scan", stream);
+    route_scan_kernel<<<1, 1024, 0, stream>>>(block_counts, nblk, E, block_base, counts, offsets, slot_of_row,
+                                              tiles, mt_cap);
+  }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  route_rank_kernel<<<nblk, 32, smem, stream>>>(topk_ids, T * k, E, kRouteTokensPerBlock * k, block_base,
-                                                row_of_slot, slot_of_row);
+  {
+    LaunchScope scope("route_rank", stream);
+    route_rank_kernel<<<nblk, 32, smem, stream>>>(topk_ids, T * k, E, kRouteTokensPerBlock * k, block_base,
+                                                  row_of_slot, slot_of_row);
+  }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return launch_gather_rows(x, slot_of_row, tiles, nullptr, H, k, rows_cap, x_perm, num_sms, stream);
 }
@@ -328,6 +337,7 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, 
                                const float* scale_w, int H, int k, int64_t rows_cap, uint16_t* dst, int num_sms,
                                cudaStream_t stream) {
   const int64_t grid = rows_cap < (int64_t)num_sms * 8 ? rows_cap : (int64_t)num_sms * 8;
+  LaunchScope scope(scale_w ? "gather_dyw" : "gather_x", stream);
   gather_rows_kernel<<<(int)grid, 256, 0, stream>>>(src, slot_of_row, tiles, scale_w, H, k, dst);
   return cudaGetLastError();
 }
@@ -335,6 +345,7 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, 
 cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot, const float* topk_w, int T, int k,
                            int H, uint16_t* out, int num_sms, cudaStream_t stream) {
   const int grid = T < num_sms * 8 ? T : num_sms * 8;
+  LaunchScope scope(topk_w ? "combine_y" : "combine_dx", stream);
   combine_kernel<<<grid, 256, 0, stream>>>(src_perm, row_of_slot, topk_w, T, k, H, out);
   return cudaGetLastError();
 }
@@ -345,11 +356,13 @@ cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64
   int64_t grid = (nblocks + 255) / 256;
   if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
   if (grid < 1) grid = 1;
+  LaunchScope scope("nf4_dequant", stream);
   nf4_dequant_kernel<<<(int)grid, 256, 0, stream>>>(packed, absmax, nblocks, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_watchdog(DeviceError* err, long long timeout_ns, cudaStream_t stream) {
+  LaunchScope scope("watchdog", stream);
   watchdog_kernel<<<1, 32, 0, stream>>>(err, timeout_ns);
   return cudaGetLastError();
 }

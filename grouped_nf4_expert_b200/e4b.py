@@ -65,6 +65,10 @@ class Sizes(ctypes.Structure):
     _fields_ = [("slots", c_i64), ("rows_cap", c_i64), ("tiles_cap", c_i64), ("workspace_bytes", c_sz)]
 
 
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", c_i64), ("total_ms", ctypes.c_double)]
+
+
 _LIB: Optional[ctypes.CDLL] = None
 
 _SIGNATURES = {
@@ -88,6 +92,9 @@ _SIGNATURES = {
                                c_vp, c_sz, c_vp]),
     "e4b_nf4_dequant": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "e4b_debug_watchdog": (c_i32, [c_vp, c_sz, c_i64, c_vp]),
+    "e4b_profiler_enable": (c_i32, [c_i32]),
+    "e4b_profiler_read": (c_i32, [ctypes.POINTER(KernelTime), c_i32, ctypes.POINTER(c_i32)]),
+    "e4b_launch_count": (c_i64, []),
 }
 
 
@@ -170,6 +177,23 @@ def e4b_nf4_dequant(packed, absmax, out, stream=None):
 
 def e4b_debug_watchdog(ws, timeout_ns: int, stream=None):
     _check(lib().e4b_debug_watchdog(_ptr(ws), ws.numel(), int(timeout_ns), _stream(stream)), "e4b_debug_watchdog")
+
+
+def e4b_profiler_enable(on: bool):
+    _check(lib().e4b_profiler_enable(1 if on else 0), "e4b_profiler_enable")
+
+
+def e4b_profiler_read():
+    """Per-kernel {name: (launches, total_ms)} recorded since the last read (waits for the events)."""
+    cap = 64
+    buf = (KernelTime * cap)()
+    n = c_i32(0)
+    _check(lib().e4b_profiler_read(buf, cap, ctypes.byref(n)), "e4b_profiler_read")
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n.value, cap))}
+
+
+def e4b_launch_count() -> int:
+    return int(lib().e4b_launch_count())
 
 
 class Block:

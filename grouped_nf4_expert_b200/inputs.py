@@ -113,15 +113,15 @@ def _nf4_stack(rng, E, rows, K, sigma):
     return codes, absmax
 
 
-def router_logits(cfg: Config, T: int = None) -> np.ndarray:
+def router_logits(cfg: Config, T: int = None, data_rank: int = 0) -> np.ndarray:
     T = cfg.T if T is None else T
-    rng = _rng(cfg.seed, 2)
+    rng = _rng(cfg.seed, 2 + 1000 * data_rank)
     if cfg.routing == "normal":
         return rng.standard_normal((T, cfg.E), dtype=np.float32)
     if cfg.routing == "zipf":
         p = np.arange(1, cfg.E + 1, dtype=np.float64) ** (-cfg.zipf_s)
         p /= p.sum()
-        perm = rng.permutation(cfg.E)
+        perm = _rng(cfg.seed, 10).permutation(cfg.E)  # the expert popularity order is a model property
         logp = np.log(p[perm])
         u = rng.random((T, cfg.E))
         gumbel = -np.log(-np.log(u))
@@ -146,12 +146,16 @@ class Problem:
     extra: dict = field(default_factory=dict)
 
 
-def make_problem(cfg: Config, T: int = None) -> Problem:
-    """All inputs of one workload (``T`` overrides the token count)."""
+def make_problem(cfg: Config, T: int = None, data_rank: int = 0) -> Problem:
+    """All inputs of one workload (``T`` overrides the token count).
+
+    ``data_rank`` selects an independent batch (tokens, logits, upstream
+    gradient) over the same weights, as data-parallel ranks see it.
+    """
     T = cfg.T if T is None else T
     E, H, I, r = cfg.E, cfg.H, cfg.I, cfg.r
-    x = _normal_bf16(_rng(cfg.seed, 1), (T, H), 1.0)
-    logits = router_logits(cfg, T)
+    x = _normal_bf16(_rng(cfg.seed, 1 + 1000 * data_rank), (T, H), 1.0)
+    logits = router_logits(cfg, T, data_rank)
     gu_codes, gu_absmax = _nf4_stack(_rng(cfg.seed, 3), E, 2 * I, H, cfg.sigma_w)
     d_codes, d_absmax = _nf4_stack(_rng(cfg.seed, 4), E, H, I, cfg.sigma_w)
     A_gu = _normal_bf16(_rng(cfg.seed, 5), (E, r, H), 1.0 / np.sqrt(H))
@@ -162,7 +166,7 @@ def make_problem(cfg: Config, T: int = None) -> Problem:
     else:
         B_gu = _normal_bf16(_rng(cfg.seed, 7), (E, 2 * I, r), 0.01)
         B_d = _normal_bf16(_rng(cfg.seed, 8), (E, H, r), 0.01)
-    dY = _normal_bf16(_rng(cfg.seed, 9), (T, H), 1.0)
+    dY = _normal_bf16(_rng(cfg.seed, 9 + 1000 * data_rank), (T, H), 1.0)
     return Problem(cfg, x, logits, gu_codes, gu_absmax, d_codes, d_absmax,
                    A_gu, B_gu, A_d, B_d, dY)
 

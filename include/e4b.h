@@ -217,6 +217,24 @@ e4b_status e4b_nf4_dequant(const uint8_t *packed, const float *absmax, int64_t n
  * wait runs out and records E4B_ERR_DEVICE_TIMEOUT in `ws`.  No GPU fault. */
 e4b_status e4b_debug_watchdog(void *ws, size_t ws_bytes, int64_t timeout_ns, e4b_stream_t stream);
 
+/* ---- Measurement -------------------------------------------------------
+ * Optional per-kernel timing.  While enabled, every kernel the library
+ * launches is bracketed by two CUDA events recorded on that launch's stream;
+ * e4b_profiler_read waits for the recorded events, returns per-kernel launch
+ * counts and summed device times, and clears the record.  Off by default; it
+ * creates CUDA events (host handles), never device buffers. */
+typedef struct {
+  char name[48];      /* kernel (and mode) name */
+  int64_t launches;   /* launches recorded */
+  double total_ms;    /* summed event-to-event device time */
+} e4b_kernel_time;
+
+e4b_status e4b_profiler_enable(int32_t on);
+e4b_status e4b_profiler_read(e4b_kernel_time *out, int32_t capacity, int32_t *count);
+
+/* Number of kernels this library has launched in this process so far. */
+int64_t e4b_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
