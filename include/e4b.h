@@ -171,6 +171,26 @@ e4b_status e4b_route_permute(const e4b_moe_dims *dims, int32_t T, const float *l
                              const e4b_bf16 *x, const e4b_routing *routing, e4b_bf16 *x_perm,
                              void *ws, size_t ws_bytes, e4b_stream_t stream);
 
+/* Routing and grouping exactly as e4b_route_permute, for callers that
+ * cannot allocate device memory and so cannot supply a workspace: code
+ * running while a CUDA graph is captured in global mode (cudaMalloc is not
+ * permitted there), engine plugins limited to memory the engine planned up
+ * front, or runtimes with a fixed device-memory budget.  The pages have no
+ * counterpart; this is an addition of this library.
+ * Scratch lives in a fixed 4 MiB array in the library's own device memory
+ * (held on every GPU that loads the library until the process exits); calls
+ * whose 2 * ceil(T / 256) * E int32 scratch entries exceed 1,048,576 are
+ * refused with E4B_ERR_UNSUPPORTED.  Allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library call).  The first call on a device looks
+ * up the array's device address (a one-time set-up per device, made with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array: calls whose work overlaps on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller.  Nothing in the array needs to start at zero. */
+e4b_status e4b_route_permute_noalloc(const e4b_moe_dims *dims, int32_t T, const float *logits,
+                                     const e4b_bf16 *x, const e4b_routing *routing, e4b_bf16 *x_perm,
+                                     e4b_stream_t stream);
+
 /* Forward: p_gu, gu/act (SiLU-gated epilogue), p_d, y_perm, then the
  * router-weighted un-permute y[t] = sum_j w[t,j] * y_perm[row(t,j)] (fp32
  * sum in j order, rounded once to bf16).  fwd->x_perm must hold what
