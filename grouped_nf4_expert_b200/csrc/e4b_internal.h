@@ -15,10 +15,15 @@ constexpr int kRouteTokensPerBlock = 256;
 // Header ints at the front of the tile list: [0] = m-tiles, [1] = rows used.
 constexpr int kTileHeader = 8;
 
-// Tile list layout (int32): header, then (expert, first row) per 128-row
-// m-tile, then the experts ordered by descending token count.
+// Tile list layout (int32): header ([0] 128-row m-tiles, [1] rows used,
+// [2] 256-row m-units), then (expert, first row) per 128-row m-tile, then the
+// experts ordered by descending token count, then (expert, first row, rows)
+// per 256-row m-unit (two consecutive m-tiles of one expert; the last unit of
+// an expert may hold 128 rows).
 inline int64_t mtiles_cap(int64_t N, int E) { return (N + 127) / 128 + E; }
-inline int64_t tiles_cap(int64_t N, int E) { return kTileHeader + 2 * mtiles_cap(N, E) + E; }
+inline int64_t order_offset(int64_t mt_cap) { return kTileHeader + 2 * mt_cap; }
+inline int64_t munits_offset(int64_t mt_cap, int E) { return kTileHeader + 2 * mt_cap + E; }
+inline int64_t tiles_cap(int64_t N, int E) { return munits_offset(mtiles_cap(N, E), E) + 3 * mtiles_cap(N, E); }
 inline int64_t rows_cap(int64_t N, int E) { return ((N + (int64_t)E * 127) + 127) / 128 * 128; }
 
 struct DeviceError;

@@ -57,19 +57,28 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // =============================================================================
 // NF4 grouped GEMM
 // =============================================================================
+// Work unit: up to 256 rows of one expert (a 256-row m-unit) x 128 output
+// columns.  Each decoded 128x64 weight tile feeds two M=128 UMMAs (rows 0-127
+// and 128-255), so the NF4 decode cost per MMA is half that of a 128-row tile.
+// Warp roles: warp 0 = TMA + absmax copies, warp 1 = TMEM owner and UMMA issuer,
+// warps 4-11 = two decode groups taking alternate k-chunks, warps 12-15 =
+// epilogue.  The accumulators are double-buffered in TMEM (2 x 256 columns), so
+// a tile's epilogue overlaps the next tile's main loop.
 namespace nf4g {
-constexpr int BM = 128, BN = 128, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;                        // activation tile, K-major SW128
-constexpr int B_BYTES = BN * BK * 2;                        // dequantised weight tile
-constexpr int RAW_BYTES = BN * BK / 2;                      // NF4 codes as loaded
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;  // 36 KB, 1024-aligned
-constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;             // p or q tile
-constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;             // LoRA weight tile
+constexpr int BM = 256, BN = 128, BK = 64, STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;                 // activation tile, K-major SW128 (two 128-row halves)
+constexpr int B_BYTES = BN * BK * 2;                 // dequantised weight tile
+constexpr int RAW_BYTES = BN * BK / 2;               // NF4 codes as loaded
+constexpr int AMAX_BYTES = BN * 4;                   // one absmax per decode thread
+constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + RAW_BYTES + AMAX_BYTES + 1023) / 1024) * 1024;
+constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;      // p or q rows of the unit
+constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;      // LoRA weight tile
 constexpr int BAR_BYTES = 1024;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LA_BYTES + LB_BYTES + BAR_BYTES + 1024;
-constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-7 decode, warps 8-11 epilogue
-constexpr int kTmemCols = 128;
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+constexpr int kThreads = 512;
+constexpr int kTmemCols = 512;
+constexpr int kFullCount = 1 + 32;  // the producer's expect_tx arrival + 32 absmax cp.async arrivals
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace nf4g
 
 struct Nf4GemmParams {
@@ -83,6 +92,7 @@ struct Nf4GemmParams {
   int K, n_dim, I, r_pad;
   int stored_rows, stored_cols;
   int n_nt;
+  int64_t mu_offset;  // start of the m-unit list in `tiles`
 };
 
 template <int MODE>
@@ -98,28 +108,30 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   uint8_t* la = smem + STAGES * STAGE_BYTES;
   uint8_t* lb = la + LA_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(lb + LB_BYTES);
-  uint64_t* full = bars;                 // TMA: activation tile + NF4 codes landed
-  uint64_t* bfull = bars + STAGES;       // decode: dequantised tile written
-  uint64_t* empty = bars + 2 * STAGES;   // MMA: stage consumed
-  uint64_t* lfull = bars + 3 * STAGES;   // TMA: LoRA operands landed
-  uint64_t* lempty = lfull + 1;          // MMA: LoRA operands consumed
-  uint64_t* accfull = lfull + 2;         // MMA: accumulator complete
-  uint64_t* accempty = lfull + 3;        // epilogue: accumulator drained
-  uint64_t* drain = lfull + 4;           // MMA: all issued UMMAs finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 5);
-  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 6);
+  uint64_t* full = bars;                 // TMA tiles + absmax copies landed
+  uint64_t* bfull = bars + STAGES;       // decoded weight tile written
+  uint64_t* empty = bars + 2 * STAGES;   // stage consumed by the UMMAs
+  uint64_t* lfull = bars + 3 * STAGES;   // LoRA operands landed
+  uint64_t* lempty = lfull + 1;          // LoRA operands consumed
+  uint64_t* accfull = lfull + 2;         // [2] accumulator buffer complete
+  uint64_t* accempty = lfull + 4;        // [2] accumulator buffer drained
+  uint64_t* drain = lfull + 6;           // all issued UMMAs finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 7);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], kFullCount);
       mbar_init(&bfull[s], 4);
       mbar_init(&empty[s], 1);
     }
     mbar_init(lfull, 1);
     mbar_init(lempty, 1);
-    mbar_init(accfull, 1);
-    mbar_init(accempty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
     mbar_init(drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -133,10 +145,12 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int n_units = p.tiles[0] * p.n_nt;
+  const int32_t* units = p.tiles + p.mu_offset;
+  const int n_units = p.tiles[2] * p.n_nt;
   const int kchunks = p.K / BK;
+  const int blocks_per_row = p.stored_cols / 64;
 
-  // Stored rows of the B tile (row-major stacks, K-major modes): two 64-row halves.
+  // Stored rows of the B tile (K-major modes): two 64-row halves.
   auto kmajor_rows = [&](int nt, int& rA, int& rB) {
     if (MODE == kFwdGateUp) {
       rA = nt * 64;
@@ -148,23 +162,26 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer + absmax copies (whole warp)
     if (lane == 0) {
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_raw);
       tma_prefetch_desc(&map_la);
       tma_prefetch_desc(&map_lb);
-      int s = 0;
-      uint32_t ph = 0, tph = 0, issued = 0, last_par = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const int mt = u / p.n_nt, nt = u % p.n_nt;
-        const int e = p.tiles[kTileHeader + 2 * mt], row0 = p.tiles[kTileHeader + 2 * mt + 1];
-        int rA = 0, rB = 0;
-        if (!kMN) kmajor_rows(nt, rA, rB);
-        if (!(ok = mbar_wait(lempty, tph ^ 1, ctl, p.err, p.timeout_ns, 10))) break;
-        mbar_arrive_expect_tx(lfull, 512u * p.r_pad);
+    }
+    uint32_t j = 0, ti = 0, issued = 0, last_par = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+      const int mu = u / p.n_nt, nt = u % p.n_nt;
+      const int e = units[3 * mu], row0 = units[3 * mu + 1], nrows = units[3 * mu + 2];
+      int rA = 0, rB = 0;
+      if (!kMN) kmajor_rows(nt, rA, rB);
+      ok = __all_sync(kFull, mbar_wait(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 10));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(lfull, (uint32_t)(nrows * 2 * p.r_pad + 256 * p.r_pad));
         tma_load_2d(la, &map_la, lfull, 0, row0);
+        if (nrows > 128) tma_load_2d(la + 256 * p.r_pad, &map_la, lfull, 0, row0 + 128);
         if (!kMN) {
           tma_load_3d(lb, &map_lb, lfull, 0, rA, e);
           tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, 0, rB, e);
@@ -172,60 +189,84 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
           tma_load_3d(lb, &map_lb, lfull, nt * 128, 0, e);
           tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, nt * 128 + 64, 0, e);
         }
-        tph ^= 1;
-        for (int kc = 0; kc < kchunks; ++kc) {
-          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 11))) break;
-          uint8_t* st = stages + s * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], A_BYTES + RAW_BYTES);
+      }
+      for (int kc = 0; kc < kchunks; ++kc, ++j) {
+        const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
+        ok = __all_sync(kFull, mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 11));
+        if (!ok) break;
+        uint8_t* st = stages + s * STAGE_BYTES;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * BK * 2 + RAW_BYTES));
           tma_load_2d(st, &map_a, &full[s], kc * BK, row0);
+          if (nrows > 128) tma_load_2d(st + A_BYTES / 2, &map_a, &full[s], kc * BK, row0 + 128);
           if (!kMN) {
             tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, &full[s], kc * (BK / 2), rA, e);
             tma_load_3d(st + A_BYTES + B_BYTES + RAW_BYTES / 2, &map_raw, &full[s], kc * (BK / 2), rB, e);
           } else {
             tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, &full[s], nt * (BN / 2), kc * BK, e);
           }
-          issued |= 1u << s;
-          last_par = (last_par & ~(1u << s)) | (ph << s);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
         }
-      }
-      if (!ok) {
-        // Let copies already issued land before the CTA's shared memory goes away.
-        for (int i = 0; i < STAGES; ++i)
-          if (issued & (1u << i)) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
-                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
-            }
+        // absmax of the block each decode thread t will decode -> amax[t]
+        float* amax = reinterpret_cast<float*>(st + A_BYTES + B_BYTES + RAW_BYTES);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int t = lane + 32 * qq;
+          int srow, sblk;
+          bool valid;
+          if (!kMN) {
+            srow = (t < 64) ? rA + t : rB + (t - 64);
+            sblk = kc;
+            valid = srow < p.stored_rows;
+          } else {
+            srow = kc * BK + (t & 63);
+            sblk = nt * 2 + (t >> 6);
+            valid = sblk < blocks_per_row;
           }
+          if (valid) cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk);
+        }
+        cp_async_arrive_noinc(&full[s]);
+        issued |= 1u << s;
+        last_par = (last_par & ~(1u << s)) | (ph << s);
       }
     }
+    if (!ok && lane == 0) {
+      // Let copies already issued land before the CTA's shared memory goes away.
+      for (int i = 0; i < STAGES; ++i)
+        if (issued & (1u << i)) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
+                 (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+          }
+        }
+    }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------ UMMA issuer
     if (lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(BM, BN, false, kMN);
+      const uint32_t idesc = make_idesc_bf16(128, BN, false, kMN);
       const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
       const uint32_t la_u = smem_u32(la), lb_u = smem_u32(lb);
-      int s = 0;
-      uint32_t ph = 0, tph = 0;
+      uint32_t j = 0, ti = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        if (!(ok = mbar_wait(accempty, tph ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+        const int nrows = units[3 * (u / p.n_nt) + 2];
+        const uint32_t b = ti & 1, use = ti >> 1;
+        const uint32_t d0 = tmem + b * 256, d1 = d0 + 128;
+        if (!(ok = mbar_wait(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
         tc_fence_after();
-        if (!(ok = mbar_wait(lfull, tph, ctl, p.err, p.timeout_ns, 21))) break;
+        if (!(ok = mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 21))) break;
         tc_fence_after();
-        // LoRA step first: acc = (s*p) * B_lora^T over K = r (overwrites the accumulator).
+        // LoRA step first: acc = (s*p) . B_lora^T over K = r (overwrites the accumulators).
         for (int ks = 0; ks < p.r_pad / 16; ++ks) {
-          const uint64_t ad = make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz);
           const uint64_t bd = kMN ? make_sdesc(lb_u + 2048 * ks, 128 * p.r_pad, 1024, kSw128)
                                   : make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz);
-          umma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+          umma_bf16(d0, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
+          if (nrows > 128)
+            umma_bf16(d1, make_sdesc(la_u + 256 * p.r_pad + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc,
+                      ks > 0 ? 1u : 0u);
         }
         umma_commit(lempty);
-        for (int kc = 0; kc < kchunks; ++kc) {
+        for (int kc = 0; kc < kchunks; ++kc, ++j) {
+          const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
           if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 22))) break;
           if (!(ok = mbar_wait(&bfull[s], ph, ctl, p.err, p.timeout_ns, 23))) break;
           tc_fence_after();
@@ -233,59 +274,46 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
           const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = make_sdesc(a0 + 32 * kk, 16, 1024, kSw128);
             const uint64_t bd =
                 kMN ? make_sdesc(b0 + 2048 * kk, 8192, 1024, kSw128) : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
-            umma_bf16(tmem, ad, bd, idesc, 1u);
+            umma_bf16(d0, make_sdesc(a0 + 32 * kk, 16, 1024, kSw128), bd, idesc, 1u);
+            if (nrows > 128) umma_bf16(d1, make_sdesc(a0 + A_BYTES / 2 + 32 * kk, 16, 1024, kSw128), bd, idesc, 1u);
           }
           umma_commit(&empty[s]);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
         }
         if (!ok) break;
-        umma_commit(accfull);
-        tph ^= 1;
+        umma_commit(&accfull[b]);
       }
       umma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
       }
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ NF4 decode
-    const int t = threadIdx.x - 128;
-    const int blocks_per_row = p.stored_cols / 64;
-    int s = 0;
-    uint32_t ph = 0;
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------ NF4 decode, two groups on alternate k-chunks
+    const uint32_t grp = (warp - 4) >> 2;
+    const int t = (threadIdx.x - 128) & 127;
+    uint32_t j = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int mt = u / p.n_nt, nt = u % p.n_nt;
-      const int e = p.tiles[kTileHeader + 2 * mt];
+      const int nt = u % p.n_nt;
       int rA = 0, rB = 0;
       if (!kMN) kmajor_rows(nt, rA, rB);
-      for (int kc = 0; kc < kchunks; ++kc) {
-        int srow, sblk;
-        bool valid;
-        if (!kMN) {
-          srow = (t < 64) ? rA + t : rB + (t - 64);
-          sblk = kc;
-          valid = srow < p.stored_rows;
-        } else {
-          srow = kc * BK + (t & 63);
-          sblk = nt * 2 + (t >> 6);
-          valid = sblk < blocks_per_row;
-        }
-        const float amax =
-            valid ? __ldg(p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk) : 0.0f;
-        ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 30);
-        ok = __all_sync(kFull, ok);
+      for (int kc = 0; kc < kchunks; ++kc, ++j) {
+        if ((j & 1) != grp) continue;
+        const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
+        ok = __all_sync(kFull, mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 30));
         if (!ok) break;
+        bool valid;
+        if (!kMN)
+          valid = ((t < 64) ? rA + t : rB + (t - 64)) < p.stored_rows;
+        else
+          valid = nt * 2 + (t >> 6) < blocks_per_row;
         uint8_t* st = stages + s * STAGE_BYTES;
         const uint8_t* raw = st + A_BYTES + B_BYTES + (kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32);
         uint32_t v[32];
         if (valid) {
+          const float amax = reinterpret_cast<const float*>(st + A_BYTES + B_BYTES + RAW_BYTES)[t];
           const uint4 q0 = *reinterpret_cast<const uint4*>(raw);
           const uint4 q1 = *reinterpret_cast<const uint4*>(raw + 16);
           const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
@@ -301,86 +329,84 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bfull[s]);
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1;
-        }
       }
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ epilogue
-    const int q = threadIdx.x - 256;  // tile row == TMEM lane
-    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint32_t tph = 0;
+  } else if (warp >= 12) {
+    // ------------------------------------------------ epilogue
+    const int qrt = warp & 3;  // TMEM lane quarter of this warp
+    uint32_t ti = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int mt = u / p.n_nt, nt = u % p.n_nt;
-      const size_t row = (size_t)p.tiles[kTileHeader + 2 * mt + 1] + q;
-      ok = mbar_wait(accfull, tph, ctl, p.err, p.timeout_ns, 40);
-      ok = __all_sync(kFull, ok);
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+      const int mu = u / p.n_nt, nt = u % p.n_nt;
+      const int row0 = units[3 * mu + 1], nrows = units[3 * mu + 2];
+      const uint32_t b = ti & 1, use = ti >> 1;
+      ok = __all_sync(kFull, mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 40));
       if (!ok) break;
       tc_fence_after();
-      if (MODE == kFwdGateUp) {
-        const int I2 = 2 * p.I, c0 = nt * 64;
+      for (int h = 0; h * 128 < nrows; ++h) {
+        const size_t row = (size_t)row0 + h * 128 + qrt * 32 + lane;
+        const uint32_t tl = tmem + b * 256 + h * 128 + ((uint32_t)(qrt * 32) << 16);
+        if (MODE == kFwdGateUp) {
+          const int I2 = 2 * p.I, c0 = nt * 64;
 #pragma unroll 1
-        for (int j = 0; j < 64; j += 16) {
-          float g[16], up[16];
-          tmem_ld16(tl + j, g);
-          tmem_ld16(tl + 64 + j, up);
-          uint32_t gw[8], uw[8], aw[8];
+          for (int jj = 0; jj < 64; jj += 16) {
+            float g[16], up[16];
+            tmem_ld16(tl + jj, g);
+            tmem_ld16(tl + 64 + jj, up);
+            uint32_t gw[8], uw[8], aw[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            gw[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
-            uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
-            aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
-          }
-          store_bf16x16(p.out0 + row * I2 + c0 + j, gw);
-          store_bf16x16(p.out0 + row * I2 + p.I + c0 + j, uw);
-          store_bf16x16(p.out1 + row * p.I + c0 + j, aw);
-        }
-      } else if (MODE == kDgradDown) {
-        const int I2 = 2 * p.I, c0 = nt * 128;
-#pragma unroll 1
-        for (int j = 0; j < 128; j += 16) {
-          if (c0 + j >= p.I) break;
-          float da[16], g[16], up[16];
-          tmem_ld16(tl + j, da);
-          load_bf16x16(p.aux + row * I2 + c0 + j, g);
-          load_bf16x16(p.aux + row * I2 + p.I + c0 + j, up);
-          uint32_t dgw[8], duw[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float dg[2], du[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float gg = g[2 * i + h], uu = up[2 * i + h], d = da[2 * i + h];
-              const float sg = 1.0f / (1.0f + __expf(-gg));
-              dg[h] = d * uu * sg * (1.0f + gg * (1.0f - sg));
-              du[h] = d * gg * sg;
+            for (int i = 0; i < 8; ++i) {
+              gw[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+              uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
+              aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
             }
-            dgw[i] = pack_bf16x2(dg[0], dg[1]);
-            duw[i] = pack_bf16x2(du[0], du[1]);
+            store_bf16x16(p.out0 + row * I2 + c0 + jj, gw);
+            store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, uw);
+            store_bf16x16(p.out1 + row * p.I + c0 + jj, aw);
           }
-          store_bf16x16(p.out0 + row * I2 + c0 + j, dgw);
-          store_bf16x16(p.out0 + row * I2 + p.I + c0 + j, duw);
-        }
-      } else {
-        const int c0 = nt * 128;
+        } else if (MODE == kDgradDown) {
+          const int I2 = 2 * p.I, c0 = nt * 128;
 #pragma unroll 1
-        for (int j = 0; j < 128; j += 16) {
-          if (c0 + j >= p.n_dim) break;
-          float v[16];
-          tmem_ld16(tl + j, v);
-          uint32_t w[8];
+          for (int jj = 0; jj < 128; jj += 16) {
+            if (c0 + jj >= p.I) break;
+            float da[16], g[16], up[16];
+            load_bf16x16(p.aux + row * I2 + c0 + jj, g);
+            load_bf16x16(p.aux + row * I2 + p.I + c0 + jj, up);
+            tmem_ld16(tl + jj, da);
+            uint32_t dgw[8], duw[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          store_bf16x16(p.out0 + row * p.n_dim + c0 + j, w);
+            for (int i = 0; i < 8; ++i) {
+              float dg[2], du[2];
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const float gg = g[2 * i + hh], uu = up[2 * i + hh], d = da[2 * i + hh];
+                const float sg = 1.0f / (1.0f + __expf(-gg));
+                dg[hh] = d * uu * sg * (1.0f + gg * (1.0f - sg));
+                du[hh] = d * gg * sg;
+              }
+              dgw[i] = pack_bf16x2(dg[0], dg[1]);
+              duw[i] = pack_bf16x2(du[0], du[1]);
+            }
+            store_bf16x16(p.out0 + row * I2 + c0 + jj, dgw);
+            store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, duw);
+          }
+        } else {
+          const int c0 = nt * 128;
+#pragma unroll 1
+          for (int jj = 0; jj < 128; jj += 16) {
+            if (c0 + jj >= p.n_dim) break;
+            float v[16];
+            tmem_ld16(tl + jj, v);
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            store_bf16x16(p.out0 + row * p.n_dim + c0 + jj, w);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty);
-      tph ^= 1;
+      if (lane == 0) mbar_arrive(&accempty[b]);
     }
   }
 
@@ -858,6 +884,7 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
   p.stored_rows = h.stored_rows;
   p.stored_cols = h.stored_cols;
   p.n_nt = (h.mode == kFwdGateUp) ? h.I / 64 : (h.n_dim + 127) / 128;
+  p.mu_offset = munits_offset(h.mt_cap, h.E);
   const int64_t units_max = h.mt_cap * p.n_nt;
   const int grid = (int)(units_max < num_sms ? units_max : num_sms);
   const int smem = nf4g::SMEM_BYTES;

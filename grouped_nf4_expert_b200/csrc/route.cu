@@ -24,7 +24,7 @@ __device__ __forceinline__ bool route_better(float av, int ae, float bv, int be)
 // experts, then a softmax over the k selected logits.  The CTA also counts
 // the slots it produced per expert (order-independent shared counters).
 template <int EPL>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(1024) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                          int32_t* __restrict__ topk_ids,
                                                          float* __restrict__ topk_w,
                                                          int32_t* __restrict__ block_counts) {
@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   const int padded = (cnt + 127) / 128 * 128;
   const int off = block_exclusive_scan(e < E ? padded : 0, s_warp);
   const int mt_off = block_exclusive_scan(e < E ? padded / 128 : 0, s_warp);
+  const int n_mu = (padded / 128 + 1) / 2;
+  const int mu_off = block_exclusive_scan(e < E ? n_mu : 0, s_warp);
   if (e < E) {
     s_cnt[e] = cnt;
     counts[e] = cnt;
@@ -144,10 +146,17 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
       tiles[kTileHeader + 2 * (mt_off + i)] = e;
       tiles[kTileHeader + 2 * (mt_off + i) + 1] = off + 128 * i;
     }
+    int32_t* mu = tiles + kTileHeader + 2 * mt_cap + E;
+    for (int i = 0; i < n_mu; ++i) {
+      mu[3 * (mu_off + i)] = e;
+      mu[3 * (mu_off + i) + 1] = off + 256 * i;
+      mu[3 * (mu_off + i) + 2] = min(256, padded - 256 * i);
+    }
     if (e == E - 1) {
       offsets[E] = off + padded;
       tiles[0] = mt_off + padded / 128;
       tiles[1] = off + padded;
+      tiles[2] = mu_off + n_mu;
     }
   }
   __syncthreads();
@@ -304,17 +313,17 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
   {
   LaunchScope scope("route_topk", stream);
   if (epl <= 1)
-    route_topk_kernel<1><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    route_topk_kernel<1><<<nblk, 1024, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else if (epl <= 2)
-    route_topk_kernel<2><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    route_topk_kernel<2><<<nblk, 1024, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else if (epl <= 4)
-    route_topk_kernel<4><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    route_topk_kernel<4><<<nblk, 1024, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else if (epl <= 8)
-    route_topk_kernel<8><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    route_topk_kernel<8><<<nblk, 1024, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else if (epl <= 16)
-    route_topk_kernel<16><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    route_topk_kernel<16><<<nblk, 1024, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   else
-    route_topk_kernel<32><<<nblk, 256, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    route_topk_kernel<32><<<nblk, 1024, smem, stream>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
