@@ -78,6 +78,12 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LA_BYTES + LB_BYTES + BAR_BYTE
 constexpr int kThreads = 512;
 constexpr int kTmemCols = 512;
 constexpr int kFullCount = 1 + 32;  // the producer's expect_tx arrival + 32 absmax cp.async arrivals
+// k-chunk j lands on full barrier (j % STAGES, j % 2): a slot has one barrier per
+// decode group, so each barrier is waited on in order by one group only and a
+// parity wait can never run a phase ahead.  Barrier use count = j / kFullPeriod.
+constexpr int kFullPeriod = (STAGES % 2 == 0) ? STAGES : 2 * STAGES;
+__host__ __device__ constexpr uint32_t full_index(uint32_t j) { return (j % STAGES) * 2 + (j & 1); }
+__host__ __device__ constexpr uint32_t full_parity(uint32_t j) { return (j / kFullPeriod) & 1; }
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace nf4g
 
@@ -108,10 +114,10 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   uint8_t* la = smem + STAGES * STAGE_BYTES;
   uint8_t* lb = la + LA_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(lb + LB_BYTES);
-  uint64_t* full = bars;                 // TMA tiles + absmax copies landed
-  uint64_t* bfull = bars + STAGES;       // decoded weight tile written
-  uint64_t* empty = bars + 2 * STAGES;   // stage consumed by the UMMAs
-  uint64_t* lfull = bars + 3 * STAGES;   // LoRA operands landed
+  uint64_t* full = bars;                 // [STAGES][2] TMA tiles + absmax copies landed
+  uint64_t* bfull = bars + 2 * STAGES;   // decoded weight tile written
+  uint64_t* empty = bars + 3 * STAGES;   // stage consumed by the UMMAs
+  uint64_t* lfull = bars + 4 * STAGES;   // LoRA operands landed
   uint64_t* lempty = lfull + 1;          // LoRA operands consumed
   uint64_t* accfull = lfull + 2;         // [2] accumulator buffer complete
   uint64_t* accempty = lfull + 4;        // [2] accumulator buffer drained
@@ -122,7 +128,8 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], kFullCount);
+      mbar_init(&full[2 * s], kFullCount);
+      mbar_init(&full[2 * s + 1], kFullCount);
       mbar_init(&bfull[s], 4);
       mbar_init(&empty[s], 1);
     }
@@ -169,7 +176,7 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
       tma_prefetch_desc(&map_la);
       tma_prefetch_desc(&map_lb);
     }
-    uint32_t j = 0, ti = 0, issued = 0, last_par = 0;
+    uint32_t j = 0, ti = 0, issued = 0, last_par = 0;  // issued/last_par: per full barrier
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
       const int mu = u / p.n_nt, nt = u % p.n_nt;
@@ -195,15 +202,17 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
         ok = __all_sync(kFull, mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 11));
         if (!ok) break;
         uint8_t* st = stages + s * STAGE_BYTES;
+        const uint32_t fi = full_index(j);
+        uint64_t* fb = &full[fi];
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * BK * 2 + RAW_BYTES));
-          tma_load_2d(st, &map_a, &full[s], kc * BK, row0);
-          if (nrows > 128) tma_load_2d(st + A_BYTES / 2, &map_a, &full[s], kc * BK, row0 + 128);
+          mbar_arrive_expect_tx(fb, (uint32_t)(nrows * BK * 2 + RAW_BYTES));
+          tma_load_2d(st, &map_a, fb, kc * BK, row0);
+          if (nrows > 128) tma_load_2d(st + A_BYTES / 2, &map_a, fb, kc * BK, row0 + 128);
           if (!kMN) {
-            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, &full[s], kc * (BK / 2), rA, e);
-            tma_load_3d(st + A_BYTES + B_BYTES + RAW_BYTES / 2, &map_raw, &full[s], kc * (BK / 2), rB, e);
+            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, kc * (BK / 2), rA, e);
+            tma_load_3d(st + A_BYTES + B_BYTES + RAW_BYTES / 2, &map_raw, fb, kc * (BK / 2), rB, e);
           } else {
-            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, &full[s], nt * (BN / 2), kc * BK, e);
+            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, nt * (BN / 2), kc * BK, e);
           }
         }
         // absmax of the block each decode thread t will decode -> amax[t]
@@ -224,14 +233,14 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
           }
           if (valid) cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk);
         }
-        cp_async_arrive_noinc(&full[s]);
-        issued |= 1u << s;
-        last_par = (last_par & ~(1u << s)) | (ph << s);
+        cp_async_arrive_noinc(fb);
+        issued |= 1u << fi;
+        last_par = (last_par & ~(1u << fi)) | (full_parity(j) << fi);
       }
     }
     if (!ok && lane == 0) {
       // Let copies already issued land before the CTA's shared memory goes away.
-      for (int i = 0; i < STAGES; ++i)
+      for (int i = 0; i < 2 * STAGES; ++i)
         if (issued & (1u << i)) {
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
@@ -267,7 +276,7 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
         umma_commit(lempty);
         for (int kc = 0; kc < kchunks; ++kc, ++j) {
           const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
-          if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 22))) break;
+          if (!(ok = mbar_wait(&full[full_index(j)], full_parity(j), ctl, p.err, p.timeout_ns, 22))) break;
           if (!(ok = mbar_wait(&bfull[s], ph, ctl, p.err, p.timeout_ns, 23))) break;
           tc_fence_after();
           const uint32_t a0 = smem_u32(stages + s * STAGE_BYTES);
@@ -301,8 +310,8 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
       if (!kMN) kmajor_rows(nt, rA, rB);
       for (int kc = 0; kc < kchunks; ++kc, ++j) {
         if ((j & 1) != grp) continue;
-        const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
-        ok = __all_sync(kFull, mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 30));
+        const uint32_t s = j % STAGES;
+        ok = __all_sync(kFull, mbar_wait(&full[full_index(j)], full_parity(j), ctl, p.err, p.timeout_ns, 30));
         if (!ok) break;
         bool valid;
         if (!kMN)

@@ -293,3 +293,24 @@ def test_mixtral_workload_forward_sampled_tokens():
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
     fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=toks)
     assert rel_err(f64(blk.y)[toks], fo["y"][toks]) <= TOL
+
+
+def test_repeated_full_size_runs_are_bit_identical():
+    # Any ordering race in the pipelined kernels shows up as run-to-run differences.
+    cfg = inputs.CONFIGS["finegrained"]
+    prob = inputs.make_problem(cfg)
+    d = dv.upload(prob)
+    blk = e4b.Block(dv.dims_of(cfg), cfg.T)
+    ref = None
+    for _ in range(6):
+        blk.e4b_route_permute(d.logits, d.x)
+        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora())
+        blk.e4b_grouped_nf4_lora_dgrad(d.base(), d.lora(), d.dY)
+        blk.e4b_lora_wgrad()
+        assert blk.check_device_error() == e4b.E4B_OK
+        cur = [t.clone() for t in (blk.y, blk.dx, blk.gu, blk.dgu, blk.dA_gu, blk.dB_d)]
+        if ref is None:
+            ref = cur
+        else:
+            for a, b in zip(ref, cur):
+                assert torch.equal(a, b)
