@@ -55,29 +55,41 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }  // namespace
 
 // =============================================================================
-// NF4 grouped GEMM
+// NF4 grouped GEMM on CTA pairs (2-SM UMMA)
 // =============================================================================
-// Work unit: up to 256 rows of one expert (a 256-row m-unit) x 128 output
-// columns.  Each decoded 128x64 weight tile feeds two M=128 UMMAs (rows 0-127
-// and 128-255), so the NF4 decode cost per MMA is half that of a 128-row tile.
-// Warp roles: warp 0 = TMA + absmax copies, warp 1 = TMEM owner and UMMA issuer,
-// warps 4-11 = two decode groups taking alternate k-chunks, warps 12-15 =
-// epilogue.  The accumulators are double-buffered in TMEM (2 x 256 columns), so
-// a tile's epilogue overlaps the next tile's main loop.
+// Work unit: up to 256 rows of one expert (a 256-row m-unit) x 256 output
+// columns, computed by a cluster of two CTAs with cta_group::2 UMMAs
+// (M = 256, N = 256).  CTA rank c holds rows [128c, 128c+128) of the
+// activation tile and decodes weight rows (output columns) [128c, 128c+128)
+// of the tile; its TMEM receives its 128 rows x 256 columns.  Each CTA loads
+// only its own tiles (no multicast loads).
+// Roles per CTA: warp 0 = TMA + absmax copies, warp 1 = TMEM owner (both CTAs)
+// and UMMA issuer (even CTA only), warp 2 = LoRA-operand relay, warps 4-11 =
+// two decode groups on alternate k-chunks, warps 12-15 = epilogue.
+// The UMMA issuer (even CTA) learns of its own CTA's readiness through local
+// barriers (bdone, lfull) and of the odd CTA's through bfull / lready, which
+// the odd CTA signals with st.async stores whose mbarrier complete_tx carries
+// the cluster-scope release (a release-arrive would stall the signalling warp
+// for about a microsecond).  bfull / lready expect 16 / 4 bytes per phase and
+// are re-armed by the issuer as soon as it has observed a phase.  The issuer's
+// commits arrive on both CTAs' empty / lempty / accfull barriers.
 namespace nf4g {
-constexpr int BM = 256, BN = 128, BK = 64, STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;                 // activation tile, K-major SW128 (two 128-row halves)
+constexpr int BM = 128;   // activation rows per CTA (256 per pair)
+constexpr int BN = 128;   // weight rows decoded per CTA (256 output columns per pair)
+constexpr int BK = 64, STAGES = 5;
+constexpr int A_BYTES = BM * BK * 2;                 // activation tile, K-major SW128
 constexpr int B_BYTES = BN * BK * 2;                 // dequantised weight tile
 constexpr int RAW_BYTES = BN * BK / 2;               // NF4 codes as loaded
 constexpr int AMAX_BYTES = BN * 4;                   // one absmax per decode thread
 constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + RAW_BYTES + AMAX_BYTES + 1023) / 1024) * 1024;
-constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;      // p or q rows of the unit
-constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;      // LoRA weight tile
+constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;      // p or q rows of this CTA
+constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;      // LoRA weight rows of this CTA
 constexpr int BAR_BYTES = 1024;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LA_BYTES + LB_BYTES + BAR_BYTES + 1024;
 constexpr int kThreads = 512;
-constexpr int kTmemCols = 512;
+constexpr int kTmemCols = 512;      // 2 accumulator buffers x 256 columns
 constexpr int kFullCount = 1 + 32;  // the producer's expect_tx arrival + 32 absmax cp.async arrivals
+constexpr int kGroupWarps = 4;      // warps per decode group
 // k-chunk j lands on full barrier (j % STAGES, j % 2): a slot has one barrier per
 // decode group, so each barrier is waited on in order by one group only and a
 // parity wait can never run a phase ahead.  Barrier use count = j / kFullPeriod.
@@ -102,7 +114,7 @@ struct Nf4GemmParams {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(nf4g::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     nf4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_raw,
                     const __grid_constant__ CUtensorMap map_la, const __grid_constant__ CUtensorMap map_lb,
                     const Nf4GemmParams p) {
@@ -114,41 +126,49 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   uint8_t* la = smem + STAGES * STAGE_BYTES;
   uint8_t* lb = la + LA_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(lb + LB_BYTES);
-  uint64_t* full = bars;                 // [STAGES][2] TMA tiles + absmax copies landed
-  uint64_t* bfull = bars + 2 * STAGES;   // decoded weight tile written
-  uint64_t* empty = bars + 3 * STAGES;   // stage consumed by the UMMAs
-  uint64_t* lfull = bars + 4 * STAGES;   // LoRA operands landed
-  uint64_t* lempty = lfull + 1;          // LoRA operands consumed
-  uint64_t* accfull = lfull + 2;         // [2] accumulator buffer complete
-  uint64_t* accempty = lfull + 4;        // [2] accumulator buffer drained
-  uint64_t* drain = lfull + 6;           // all issued UMMAs finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 7);
-  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 8);
+  uint64_t* full = bars;                 // [STAGES][2] local TMA tiles + absmax copies landed
+  uint64_t* bfull = bars + 2 * STAGES;   // [STAGES] (even CTA) the odd CTA's decoded tile written
+  uint64_t* empty = bars + 3 * STAGES;   // [STAGES] stage consumed by the UMMAs
+  uint64_t* bdone = bars + 4 * STAGES;   // [STAGES] (even CTA) its own decoded tile written
+  uint64_t* lfull = bars + 5 * STAGES;   // local LoRA operands landed
+  uint64_t* lready = lfull + 1;          // (even CTA) the odd CTA's LoRA operands landed
+  uint64_t* lempty = lfull + 2;          // LoRA operands consumed
+  uint64_t* accfull = lfull + 3;         // [2] accumulator buffer complete
+  uint64_t* accempty = lfull + 5;        // [2] (even CTA) accumulator buffer drained in both CTAs
+  uint64_t* drain = lfull + 7;           // (even CTA) all issued UMMAs finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 8);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 9);
+  uint32_t* sig = reinterpret_cast<uint32_t*>(lfull + 10);  // target word of the st.async signals
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[2 * s], kFullCount);
       mbar_init(&full[2 * s + 1], kFullCount);
-      mbar_init(&bfull[s], 4);
+      mbar_init(&bfull[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&bdone[s], kGroupWarps);
     }
     mbar_init(lfull, 1);
+    mbar_init(lready, 1);
+    for (int s = 0; s < STAGES; ++s) mbar_arrive_expect_tx(&bfull[s], 4 * kGroupWarps);  // arm phase 0
+    mbar_arrive_expect_tx(lready, 4);
     mbar_init(lempty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], 4);
+      mbar_init(&accempty[b], 8);
     }
     mbar_init(drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_2sm(tmem_slot, kTmemCols);
+    tmem_relinquish_2sm();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -156,16 +176,25 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
   const int n_units = p.tiles[2] * p.n_nt;
   const int kchunks = p.K / BK;
   const int blocks_per_row = p.stored_cols / 64;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
-  // Stored rows of the B tile (K-major modes): two 64-row halves.
+  // Stored rows of this CTA's weight tile (K-major modes): two 64-row halves.
   auto kmajor_rows = [&](int nt, int& rA, int& rB) {
-    if (MODE == kFwdGateUp) {
-      rA = nt * 64;
-      rB = p.I + nt * 64;
+    if (MODE == kFwdGateUp) {  // even CTA: gate rows, odd CTA: the matching up rows
+      rA = (rank ? p.I : 0) + nt * 128;
+      rB = rA + 64;
     } else {
-      rA = nt * 128;
-      rB = nt * 128 + 64;
+      rA = nt * 256 + rank * 128;
+      rB = rA + 64;
     }
+  };
+  // Decoded tile row t of this CTA is valid (exists in the stored matrix / output).
+  auto row_valid = [&](int nt, int t) -> bool {
+    if (!kMN) {
+      if (MODE == kFwdGateUp) return nt * 128 + t < p.I;
+      return nt * 256 + rank * 128 + t < p.stored_rows;
+    }
+    return nt * 4 + rank * 2 + (t >> 6) < blocks_per_row;
   };
 
   if (warp == 0) {
@@ -178,23 +207,33 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
     }
     uint32_t j = 0, ti = 0, issued = 0, last_par = 0;  // issued/last_par: per full barrier
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
-      const int mu = u / p.n_nt, nt = u % p.n_nt;
-      const int e = units[3 * mu], row0 = units[3 * mu + 1], nrows = units[3 * mu + 2];
+    // The next unit's (expert, first row) are loaded one unit ahead, off the critical path.
+    int e_next = 0, r_next = 0;
+    if (pair < n_units) {
+      e_next = units[3 * (pair / p.n_nt)];
+      r_next = units[3 * (pair / p.n_nt) + 1];
+    }
+    for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
+      const int nt = u % p.n_nt;
+      const int e = e_next, row0 = r_next + (int)rank * 128;
+      if (u + n_pairs < n_units) {
+        e_next = units[3 * ((u + n_pairs) / p.n_nt)];
+        r_next = units[3 * ((u + n_pairs) / p.n_nt) + 1];
+      }
       int rA = 0, rB = 0;
       if (!kMN) kmajor_rows(nt, rA, rB);
       ok = __all_sync(kFull, mbar_wait(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 10));
       if (!ok) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(lfull, (uint32_t)(nrows * 2 * p.r_pad + 256 * p.r_pad));
+        mbar_arrive_expect_tx(lfull, (uint32_t)(512 * p.r_pad));
         tma_load_2d(la, &map_la, lfull, 0, row0);
-        if (nrows > 128) tma_load_2d(la + 256 * p.r_pad, &map_la, lfull, 0, row0 + 128);
         if (!kMN) {
           tma_load_3d(lb, &map_lb, lfull, 0, rA, e);
           tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, 0, rB, e);
         } else {
-          tma_load_3d(lb, &map_lb, lfull, nt * 128, 0, e);
-          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, nt * 128 + 64, 0, e);
+          const int c0 = nt * 256 + rank * 128;
+          tma_load_3d(lb, &map_lb, lfull, c0, 0, e);
+          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, c0 + 64, 0, e);
         }
       }
       for (int kc = 0; kc < kchunks; ++kc, ++j) {
@@ -205,14 +244,13 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
         const uint32_t fi = full_index(j);
         uint64_t* fb = &full[fi];
         if (lane == 0) {
-          mbar_arrive_expect_tx(fb, (uint32_t)(nrows * BK * 2 + RAW_BYTES));
+          mbar_arrive_expect_tx(fb, (uint32_t)(A_BYTES + RAW_BYTES));
           tma_load_2d(st, &map_a, fb, kc * BK, row0);
-          if (nrows > 128) tma_load_2d(st + A_BYTES / 2, &map_a, fb, kc * BK, row0 + 128);
           if (!kMN) {
             tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, kc * (BK / 2), rA, e);
             tma_load_3d(st + A_BYTES + B_BYTES + RAW_BYTES / 2, &map_raw, fb, kc * (BK / 2), rB, e);
           } else {
-            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, nt * (BN / 2), kc * BK, e);
+            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, (nt * 256 + rank * 128) / 2, kc * BK, e);
           }
         }
         // absmax of the block each decode thread t will decode -> amax[t]
@@ -221,17 +259,15 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
         for (int qq = 0; qq < 4; ++qq) {
           const int t = lane + 32 * qq;
           int srow, sblk;
-          bool valid;
           if (!kMN) {
             srow = (t < 64) ? rA + t : rB + (t - 64);
             sblk = kc;
-            valid = srow < p.stored_rows;
           } else {
             srow = kc * BK + (t & 63);
-            sblk = nt * 2 + (t >> 6);
-            valid = sblk < blocks_per_row;
+            sblk = nt * 4 + rank * 2 + (t >> 6);
           }
-          if (valid) cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk);
+          if (row_valid(nt, t))
+            cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk);
         }
         cp_async_arrive_noinc(fb);
         issued |= 1u << fi;
@@ -249,35 +285,34 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
         }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------ UMMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(128, BN, false, kMN);
+    // ------------------------------------------------ UMMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = make_idesc_bf16(256, 256, false, kMN);
       const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
       const uint32_t la_u = smem_u32(la), lb_u = smem_u32(lb);
       uint32_t j = 0, ti = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
-        const int nrows = units[3 * (u / p.n_nt) + 2];
+      for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
         const uint32_t b = ti & 1, use = ti >> 1;
-        const uint32_t d0 = tmem + b * 256, d1 = d0 + 128;
-        if (!(ok = mbar_wait(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
+        const uint32_t d = tmem + b * 256;
+        if (!(ok = mbar_wait_cluster(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
         tc_fence_after();
         if (!(ok = mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 21))) break;
+        if (!(ok = mbar_wait_cluster(lready, ti & 1, ctl, p.err, p.timeout_ns, 21))) break;
+        mbar_arrive_expect_tx(lready, 4);  // arm the next phase
         tc_fence_after();
-        // LoRA step first: acc = (s*p) . B_lora^T over K = r (overwrites the accumulators).
+        // LoRA step first: acc = (s*p) . B_lora^T over K = r (overwrites the accumulator).
         for (int ks = 0; ks < p.r_pad / 16; ++ks) {
           const uint64_t bd = kMN ? make_sdesc(lb_u + 2048 * ks, 128 * p.r_pad, 1024, kSw128)
                                   : make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz);
-          umma_bf16(d0, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
-          if (nrows > 128)
-            umma_bf16(d1, make_sdesc(la_u + 256 * p.r_pad + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc,
-                      ks > 0 ? 1u : 0u);
+          umma_bf16_2sm(d, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
         }
-        umma_commit(lempty);
+        umma_commit_2sm(lempty, 0x3);
         for (int kc = 0; kc < kchunks; ++kc, ++j) {
           const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
-          if (!(ok = mbar_wait(&full[full_index(j)], full_parity(j), ctl, p.err, p.timeout_ns, 22))) break;
-          if (!(ok = mbar_wait(&bfull[s], ph, ctl, p.err, p.timeout_ns, 23))) break;
+          if (!(ok = mbar_wait(&bdone[s], ph, ctl, p.err, p.timeout_ns, 24))) break;
+          if (!(ok = mbar_wait_cluster(&bfull[s], ph, ctl, p.err, p.timeout_ns, 23))) break;
+          mbar_arrive_expect_tx(&bfull[s], 4 * kGroupWarps);  // arm the next phase
           tc_fence_after();
           const uint32_t a0 = smem_u32(stages + s * STAGE_BYTES);
           const uint32_t b0 = a0 + A_BYTES;
@@ -285,39 +320,43 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bd =
                 kMN ? make_sdesc(b0 + 2048 * kk, 8192, 1024, kSw128) : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
-            umma_bf16(d0, make_sdesc(a0 + 32 * kk, 16, 1024, kSw128), bd, idesc, 1u);
-            if (nrows > 128) umma_bf16(d1, make_sdesc(a0 + A_BYTES / 2 + 32 * kk, 16, 1024, kSw128), bd, idesc, 1u);
+            umma_bf16_2sm(d, make_sdesc(a0 + 32 * kk, 16, 1024, kSw128), bd, idesc, 1u);
           }
-          umma_commit(&empty[s]);
+          umma_commit_2sm(&empty[s], 0x3);
         }
         if (!ok) break;
-        umma_commit(&accfull[b]);
+        umma_commit_2sm(&accfull[b], 0x3);
       }
-      umma_commit(drain);
+      umma_commit_2sm(drain, 0x1);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
       }
+    }
+  } else if (warp == 2 && rank == 1) {
+    // ------------------------------------------------ relay (odd CTA): LoRA operands landed -> even CTA
+    const uint32_t lready_even = mapa_shared(smem_u32(lready), 0);
+    const uint32_t sig_even = mapa_shared(smem_u32(sig), 0);
+    uint32_t ti = 0;
+    for (int u = pair; u < n_units; u += n_pairs, ++ti) {
+      if (!__all_sync(kFull, mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 50))) break;
+      if (lane == 0) st_async_signal(sig_even, lready_even, 1u);
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------ NF4 decode, two groups on alternate k-chunks
     const uint32_t grp = (warp - 4) >> 2;
     const int t = (threadIdx.x - 128) & 127;
+    const uint32_t bfull_even = mapa_shared(smem_u32(bfull), 0);
+    const uint32_t sig_even = mapa_shared(smem_u32(sig), 0);
     uint32_t j = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int u = pair; u < n_units && ok; u += n_pairs) {
       const int nt = u % p.n_nt;
-      int rA = 0, rB = 0;
-      if (!kMN) kmajor_rows(nt, rA, rB);
+      const bool valid = row_valid(nt, t);
       for (int kc = 0; kc < kchunks; ++kc, ++j) {
         if ((j & 1) != grp) continue;
         const uint32_t s = j % STAGES;
         ok = __all_sync(kFull, mbar_wait(&full[full_index(j)], full_parity(j), ctl, p.err, p.timeout_ns, 30));
         if (!ok) break;
-        bool valid;
-        if (!kMN)
-          valid = ((t < 64) ? rA + t : rB + (t - 64)) < p.stored_rows;
-        else
-          valid = nt * 2 + (t >> 6) < blocks_per_row;
         uint8_t* st = stages + s * STAGE_BYTES;
         const uint8_t* raw = st + A_BYTES + B_BYTES + (kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32);
         uint32_t v[32];
@@ -337,93 +376,111 @@ __global__ void __launch_bounds__(nf4g::kThreads, 1)
           st_swizzled_row128(st + A_BYTES + (t >> 6) * 8192, t & 63, v);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bfull[s]);
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(&bdone[s]);
+          else
+            st_async_signal(sig_even, bfull_even + 8 * s, 1u);
+        }
       }
     }
   } else if (warp >= 12) {
     // ------------------------------------------------ epilogue
     const int qrt = warp & 3;  // TMEM lane quarter of this warp
+    const uint32_t accempty_even = mapa_shared(smem_u32(accempty), 0);
     uint32_t ti = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+    for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
       const int mu = u / p.n_nt, nt = u % p.n_nt;
-      const int row0 = units[3 * mu + 1], nrows = units[3 * mu + 2];
+      const int nrows = units[3 * mu + 2];
+      const bool store = (int)rank * 128 < nrows;
+      const size_t row = (size_t)units[3 * mu + 1] + rank * 128 + qrt * 32 + lane;
       const uint32_t b = ti & 1, use = ti >> 1;
       ok = __all_sync(kFull, mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 40));
       if (!ok) break;
       tc_fence_after();
-      for (int h = 0; h * 128 < nrows; ++h) {
-        const size_t row = (size_t)row0 + h * 128 + qrt * 32 + lane;
-        const uint32_t tl = tmem + b * 256 + h * 128 + ((uint32_t)(qrt * 32) << 16);
-        if (MODE == kFwdGateUp) {
-          const int I2 = 2 * p.I, c0 = nt * 64;
+      const uint32_t tl = tmem + b * 256 + ((uint32_t)(qrt * 32) << 16);
+      if (MODE == kFwdGateUp) {
+        // columns [0,128): gate, [128,256): up, of gate/up columns nt*128 ..
+        const int I2 = 2 * p.I, c0 = nt * 128;
 #pragma unroll 1
-          for (int jj = 0; jj < 64; jj += 16) {
-            float g[16], up[16];
-            tmem_ld16(tl + jj, g);
-            tmem_ld16(tl + 64 + jj, up);
-            uint32_t gw[8], uw[8], aw[8];
+        for (int jj = 0; jj < 128; jj += 16) {
+          if (c0 + jj >= p.I) break;
+          float g[16], up[16];
+          tmem_ld16(tl + jj, g);
+          tmem_ld16(tl + 128 + jj, up);
+          if (!store) continue;
+          uint32_t gw[8], uw[8], aw[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              gw[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
-              uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
-              aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
-            }
-            store_bf16x16(p.out0 + row * I2 + c0 + jj, gw);
-            store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, uw);
-            store_bf16x16(p.out1 + row * p.I + c0 + jj, aw);
+          for (int i = 0; i < 8; ++i) {
+            gw[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+            uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
+            aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
           }
-        } else if (MODE == kDgradDown) {
-          const int I2 = 2 * p.I, c0 = nt * 128;
+          store_bf16x16(p.out0 + row * I2 + c0 + jj, gw);
+          store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, uw);
+          store_bf16x16(p.out1 + row * p.I + c0 + jj, aw);
+        }
+      } else if (MODE == kDgradDown) {
+        const int I2 = 2 * p.I, c0 = nt * 256;
 #pragma unroll 1
-          for (int jj = 0; jj < 128; jj += 16) {
-            if (c0 + jj >= p.I) break;
-            float da[16], g[16], up[16];
+        for (int jj = 0; jj < 256; jj += 16) {
+          if (c0 + jj >= p.I) break;
+          float da[16], g[16], up[16];
+          if (store) {
             load_bf16x16(p.aux + row * I2 + c0 + jj, g);
             load_bf16x16(p.aux + row * I2 + p.I + c0 + jj, up);
-            tmem_ld16(tl + jj, da);
-            uint32_t dgw[8], duw[8];
+          }
+          tmem_ld16(tl + jj, da);
+          if (!store) continue;
+          uint32_t dgw[8], duw[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float dg[2], du[2];
+          for (int i = 0; i < 8; ++i) {
+            float dg[2], du[2];
 #pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const float gg = g[2 * i + hh], uu = up[2 * i + hh], d = da[2 * i + hh];
-                const float sg = 1.0f / (1.0f + __expf(-gg));
-                dg[hh] = d * uu * sg * (1.0f + gg * (1.0f - sg));
-                du[hh] = d * gg * sg;
-              }
-              dgw[i] = pack_bf16x2(dg[0], dg[1]);
-              duw[i] = pack_bf16x2(du[0], du[1]);
+            for (int hh = 0; hh < 2; ++hh) {
+              const float gg = g[2 * i + hh], uu = up[2 * i + hh], dd = da[2 * i + hh];
+              const float sg = 1.0f / (1.0f + __expf(-gg));
+              dg[hh] = dd * uu * sg * (1.0f + gg * (1.0f - sg));
+              du[hh] = dd * gg * sg;
             }
-            store_bf16x16(p.out0 + row * I2 + c0 + jj, dgw);
-            store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, duw);
+            dgw[i] = pack_bf16x2(dg[0], dg[1]);
+            duw[i] = pack_bf16x2(du[0], du[1]);
           }
-        } else {
-          const int c0 = nt * 128;
+          store_bf16x16(p.out0 + row * I2 + c0 + jj, dgw);
+          store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, duw);
+        }
+      } else {
+        const int c0 = nt * 256;
 #pragma unroll 1
-          for (int jj = 0; jj < 128; jj += 16) {
-            if (c0 + jj >= p.n_dim) break;
-            float v[16];
-            tmem_ld16(tl + jj, v);
-            uint32_t w[8];
+        for (int jj = 0; jj < 256; jj += 16) {
+          if (c0 + jj >= p.n_dim) break;
+          float v[16];
+          tmem_ld16(tl + jj, v);
+          if (!store) continue;
+          uint32_t w[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-            store_bf16x16(p.out0 + row * p.n_dim + c0 + jj, w);
-          }
+          for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          store_bf16x16(p.out0 + row * p.n_dim + c0 + jj, w);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[b]);
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&accempty[b]);
+        else
+          mbar_arrive_cluster(accempty_even + 8 * b);
+      }
     }
   }
 
-  __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the CTA barrier
-  __syncthreads();
+  __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the cluster barrier
+  tc_fence_before();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_2sm(tmem, kTmemCols);
   }
 }
 
@@ -892,10 +949,11 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
   p.r_pad = h.r_pad;
   p.stored_rows = h.stored_rows;
   p.stored_cols = h.stored_cols;
-  p.n_nt = (h.mode == kFwdGateUp) ? h.I / 64 : (h.n_dim + 127) / 128;
+  p.n_nt = (h.mode == kFwdGateUp) ? (h.I + 127) / 128 : (h.n_dim + 255) / 256;
   p.mu_offset = munits_offset(h.mt_cap, h.E);
   const int64_t units_max = h.mt_cap * p.n_nt;
-  const int grid = (int)(units_max < num_sms ? units_max : num_sms);
+  const int64_t pairs = units_max < num_sms / 2 ? units_max : num_sms / 2;
+  const int grid = 2 * (int)(pairs > 0 ? pairs : 1);
   const int smem = nf4g::SMEM_BYTES;
   static const char* kNames[4] = {"nf4_gemm_fwd_gate_up", "nf4_gemm_fwd_down", "nf4_gemm_dgrad_down",
                                   "nf4_gemm_dgrad_gate_up"};
