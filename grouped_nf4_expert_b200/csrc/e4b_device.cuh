@@ -144,6 +144,13 @@ __device__ __forceinline__ void st_async_signal(uint32_t remote_word, uint32_t r
                : "memory");
 }
 
+// Arrival without release semantics: it orders none of this thread's earlier
+// memory writes (use it when the receiver needs only the arrival, e.g. that
+// this thread's TMEM reads have completed, and not this thread's global stores).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -35,6 +35,20 @@ __device__ __forceinline__ void store_bf16x16(uint16_t* dst, const uint32_t (&w)
   d[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
+// One full 32-byte sector per thread (dst must be 32-byte aligned).
+__device__ __forceinline__ void store_bf16x16_v8(uint16_t* dst, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void store16(uint16_t* dst, const uint32_t (&w)[8], bool v8) {
+  if (v8)
+    store_bf16x16_v8(dst, w);
+  else
+    store_bf16x16(dst, w);
+}
+
 __device__ __forceinline__ void load_bf16x16(const uint16_t* src, float (&v)[16]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
   const uint4 a = __ldg(s), b = __ldg(s + 1);
@@ -46,7 +60,11 @@ __device__ __forceinline__ void load_bf16x16(const uint16_t* src, float (&v)[16]
   }
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu and the logistic sigmoid with the fast exponential and the fast
+// (reciprocal-based) division: a few ulp, far below bf16 output rounding.  For
+// very negative g the denominator overflows to inf and both give 0.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -110,6 +128,7 @@ struct Nf4GemmParams {
   int K, n_dim, I, r_pad;
   int stored_rows, stored_cols;
   int n_nt;
+  int v8;             // output buffers and row pitches are 32-byte aligned: 32-byte stores
   int64_t mu_offset;  // start of the m-unit list in `tiles`
 };
 
@@ -417,9 +436,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
             uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
             aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
           }
-          store_bf16x16(p.out0 + row * I2 + c0 + jj, gw);
-          store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, uw);
-          store_bf16x16(p.out1 + row * p.I + c0 + jj, aw);
+          store16(p.out0 + row * I2 + c0 + jj, gw, p.v8);
+          store16(p.out0 + row * I2 + p.I + c0 + jj, uw, p.v8);
+          store16(p.out1 + row * p.I + c0 + jj, aw, p.v8);
         }
       } else if (MODE == kDgradDown) {
         const int I2 = 2 * p.I, c0 = nt * 256;
@@ -440,15 +459,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               const float gg = g[2 * i + hh], uu = up[2 * i + hh], dd = da[2 * i + hh];
-              const float sg = 1.0f / (1.0f + __expf(-gg));
+              const float sg = sigmoid_f(gg);
               dg[hh] = dd * uu * sg * (1.0f + gg * (1.0f - sg));
               du[hh] = dd * gg * sg;
             }
             dgw[i] = pack_bf16x2(dg[0], dg[1]);
             duw[i] = pack_bf16x2(du[0], du[1]);
           }
-          store_bf16x16(p.out0 + row * I2 + c0 + jj, dgw);
-          store_bf16x16(p.out0 + row * I2 + p.I + c0 + jj, duw);
+          store16(p.out0 + row * I2 + c0 + jj, dgw, p.v8);
+          store16(p.out0 + row * I2 + p.I + c0 + jj, duw, p.v8);
         }
       } else {
         const int c0 = nt * 256;
@@ -461,16 +480,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           uint32_t w[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          store_bf16x16(p.out0 + row * p.n_dim + c0 + jj, w);
+          store16(p.out0 + row * p.n_dim + c0 + jj, w, p.v8);
         }
       }
+      // The issuer needs only this warp's TMEM reads to be complete (tcgen05.ld
+      // waited, then the tcgen05 fence), not its global stores: the odd CTA's
+      // arrival is relaxed, since a release would first wait for the stores.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         if (rank == 0)
           mbar_arrive(&accempty[b]);
         else
-          mbar_arrive_cluster(accempty_even + 8 * b);
+          mbar_arrive_cluster_relaxed(accempty_even + 8 * b);
       }
     }
   }
@@ -950,6 +972,11 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
   p.stored_rows = h.stored_rows;
   p.stored_cols = h.stored_cols;
   p.n_nt = (h.mode == kFwdGateUp) ? (h.I + 127) / 128 : (h.n_dim + 255) / 256;
+  {
+    auto a32 = [](const void* q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
+    // row pitches in bytes: out0 is [rows, n_dim] (2I for the gate_up forward and the down dgrad), out1 [rows, I]
+    p.v8 = a32(h.out0) && a32(h.out1) && (h.n_dim * 2) % 32 == 0 && (h.I * 2) % 32 == 0 ? 1 : 0;
+  }
   p.mu_offset = munits_offset(h.mt_cap, h.E);
   const int64_t units_max = h.mt_cap * p.n_nt;
   const int64_t pairs = units_max < num_sms / 2 ? units_max : num_sms / 2;
