@@ -59,6 +59,25 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def profiled_traffic():
+    """DRAM bytes per step of the nf4_gemm launches from the committed ncu summary, if the kernel
+    source still hashes to what was profiled; else None."""
+    import hashlib
+    import re
+    src = b"".join(open(os.path.join(ROOT, "grouped_nf4_expert_b200", "csrc", f), "rb").read()
+                   for f in ("gemm.cu", "e4b_device.cuh"))
+    sha = hashlib.sha256(src).hexdigest()[:16]
+    try:
+        text = open(os.path.join(ROOT, "profiles", "nf4_gemm_train_ncu.md")).read()
+    except OSError:
+        return None
+    m_t = re.search(r"^traffic_bytes_per_step: (\d+)", text, re.M)
+    m_s = re.search(r"^source_sha256_16: ([0-9a-f]+)", text, re.M)
+    if m_t and m_s and m_s.group(1) == sha:
+        return int(m_t.group(1))
+    return None
+
+
 def step_flops(cfg):
     """Algorithmic FLOPs of one step: routed slots only, 2 FLOP per MAC."""
     N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
@@ -229,7 +248,7 @@ def main():
     import torch
     import torch.distributed as dist
 
-    from grouped_nf4_expert_b200 import build, e4b, inputs
+    from grouped_nf4_expert_b200 import build, e4b, inputs, parallel
     from grouped_nf4_expert_b200 import device as dv
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -258,8 +277,7 @@ def main():
         blk.e4b_grouped_nf4_lora_dgrad(base, lora, d.dY)
         blk.e4b_lora_wgrad()
         if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
-            for g in grads:
-                dist.all_reduce(g)
+            parallel.allreduce_lora_grads(grads)
 
     def sync_all():
         torch.cuda.synchronize(dev)
@@ -317,7 +335,9 @@ def main():
                 "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
                 "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long step)" % peak_src,
-                "traffic": None, "launches": nf4_launches,
+                "traffic": (profiled_traffic() if args.workload == "train" else None),
+                "traffic_unit": "DRAM bytes per step of the four nf4_gemm launches (ncu)",
+                "launches": nf4_launches,
                 "avg_launch_ms": nf4_ms / max(nf4_launches, 1),
                 "algorithmic_flop_per_step": sum(gflops.values())}
     per_kernel = {n: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
