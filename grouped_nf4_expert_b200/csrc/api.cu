@@ -323,7 +323,8 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
   g.out0 = fwd->gu;
   g.out1 = fwd->act;
   g.aux = nullptr;
-  E4B_CUDA(launch_nf4_gemm(g, sms, st));
+  const bool streaming = use_streaming_forward(N, E);  // decode-sized batch: weight-streaming tiles
+  E4B_CUDA(streaming ? launch_nf4_stream(g, sms, st) : launch_nf4_gemm(g, sms, st));
   // p_d = s * act A_d^T
   lp.act_in = fwd->act;
   lp.K = I;
@@ -343,7 +344,7 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
   g.lora_w = lora->B_d;
   g.out0 = fwd->y_perm;
   g.out1 = nullptr;
-  E4B_CUDA(launch_nf4_gemm(g, sms, st));
+  E4B_CUDA(streaming ? launch_nf4_stream(g, sms, st) : launch_nf4_gemm(g, sms, st));
   // y[t] = sum_j w[t,j] y_perm[row(t,j)]
   E4B_CUDA(launch_combine(fwd->y_perm, routing->row_of_slot, routing->topk_w, T, k, H, y, sms, st));
   return E4B_OK;

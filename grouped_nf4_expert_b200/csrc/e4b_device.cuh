@@ -80,6 +80,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase has not completed may be
+// suspended for up to `hint_ns` (it resumes as soon as the phase completes),
+// so that waiting warps leave the issue slots to the working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared control block of a CTA: an abort flag that every bounded wait
 // watches, so that when one role gives up the others stop too.
 struct CtaControl {
@@ -90,12 +107,16 @@ struct CtaControl {
 // Waits for the phase with `parity` of `bar` to complete.  Gives up (returns
 // false) when `timeout_ns` elapses or another thread of the CTA has given up;
 // a thread that gives up records E4B_ERR_DEVICE_TIMEOUT with `site`.
+// Upper bound of one suspended wait; the abort flag and the timeout are
+// checked between them.
+constexpr uint32_t kWaitSleepNs = 20000;
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, CtaControl* ctl,
                                           DeviceError* err, long long timeout_ns, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (ctl->abort) return false;
     if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
       ctl->abort = 1;
@@ -246,6 +267,21 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// True in exactly one active lane of the (converged) warp.  Issuing roles
+// run their loops and waits with the whole warp, so that loop state stays
+// warp-uniform, and put only the tcgen05 issue under this predicate.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "elect.sync _|p, 0xffffffff;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulation.
@@ -457,6 +493,20 @@ __device__ __forceinline__ void st_swizzled_row128(uint8_t* base, int row, const
     uint4 q = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
     *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = q;
   }
+}
+
+// silu and the logistic sigmoid with the fast exponential and the fast
+// (reciprocal-based) division: a few ulp, far below bf16 output rounding.  For
+// very negative g the denominator overflows to inf and both give 0.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+
+// Rounds a pointer into the dynamic shared-memory window up to a 1024-byte
+// boundary (swizzle atoms).  The offset is added to the original pointer, so
+// the compiler still knows the result addresses shared memory and emits
+// shared (not generic) loads and stores through it.
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
 }
 
 }  // namespace e4b

@@ -23,7 +23,13 @@ constexpr int kTileHeader = 8;
 inline int64_t mtiles_cap(int64_t N, int E) { return (N + 127) / 128 + E; }
 inline int64_t order_offset(int64_t mt_cap) { return kTileHeader + 2 * mt_cap; }
 inline int64_t munits_offset(int64_t mt_cap, int E) { return kTileHeader + 2 * mt_cap + E; }
-inline int64_t tiles_cap(int64_t N, int E) { return munits_offset(mtiles_cap(N, E), E) + 3 * mtiles_cap(N, E); }
+// Then (expert, first row, slots) per 32-slot tile of the weight-streaming
+// forward used for decode-sized batches ([3] = their count).
+inline int64_t stiles_offset(int64_t mt_cap, int E) { return munits_offset(mt_cap, E) + 3 * mt_cap; }
+inline int64_t tiles_cap(int64_t N, int E) { return stiles_offset(mtiles_cap(N, E), E) + 12 * mtiles_cap(N, E); }
+// Forward path choice: the weight-streaming kernel when the batch routes few
+// slots per expert (decode-sized), the 2-SM training tiles otherwise.
+inline bool use_streaming_forward(int64_t N, int E) { return N <= 16 * (int64_t)E; }
 inline int64_t rows_cap(int64_t N, int E) { return ((N + (int64_t)E * 127) + 127) / 128 * 128; }
 
 struct DeviceError;
@@ -62,7 +68,7 @@ cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64
 
 cudaError_t launch_watchdog(DeviceError* err, long long timeout_ns, cudaStream_t stream);
 
-// ---- grouped GEMMs (gemm.cu)
+// ---- grouped GEMMs (gemm.cu, stream.cu)
 enum Nf4Mode { kFwdGateUp = 0, kFwdDown = 1, kDgradDown = 2, kDgradGateUp = 3 };
 
 struct Nf4GemmHost {
@@ -85,6 +91,8 @@ struct Nf4GemmHost {
   long long timeout_ns;
 };
 cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stream);
+// Weight-streaming forward (kFwdGateUp / kFwdDown only) for decode-sized batches.
+cudaError_t launch_nf4_stream(const Nf4GemmHost& h, int num_sms, cudaStream_t stream);
 
 struct LoraProjHost {
   const uint16_t* act_in;  // [rows_cap, K]
@@ -117,6 +125,16 @@ struct WgradHost {
   long long timeout_ns;
 };
 cudaError_t launch_wgrad(const WgradHost& h, int num_sms, cudaStream_t stream);
+
+// Tensor maps of the operands (gemm.cu): row-major bf16 [rows, cols], bf16
+// stacks [E, rows, cols], byte stacks [E, rows, bytes].
+CUtensorMapSwizzle swizzle_for_bytes(int row_bytes);
+cudaError_t map_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                        uint32_t box_rows, CUtensorMapSwizzle swz);
+cudaError_t map_bf16_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
+                        uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+cudaError_t map_u8_3d(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t rows, uint64_t E,
+                      uint32_t box_bytes, uint32_t box_rows);
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda).
 cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,

@@ -60,15 +60,6 @@ __device__ __forceinline__ void load_bf16x16(const uint16_t* src, float (&v)[16]
   }
 }
 
-// silu and the logistic sigmoid with the fast exponential and the fast
-// (reciprocal-based) division: a few ulp, far below bf16 output rounding.  For
-// very negative g the denominator overflows to inf and both give 0.
-__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
-__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
 
 }  // namespace
 
@@ -896,8 +887,6 @@ __global__ void __launch_bounds__(wg::kThreads)
 // =============================================================================
 // Host-side launchers
 // =============================================================================
-namespace {
-
 CUtensorMapSwizzle swizzle_for_bytes(int row_bytes) {
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                           : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -931,11 +920,11 @@ cudaError_t map_u8_3d(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t
                            CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+namespace {
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
-
 }  // namespace
 
 cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stream) {

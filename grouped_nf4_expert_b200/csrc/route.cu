@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   const int mt_off = block_exclusive_scan(e < E ? padded / 128 : 0, s_warp);
   const int n_mu = (padded / 128 + 1) / 2;
   const int mu_off = block_exclusive_scan(e < E ? n_mu : 0, s_warp);
+  const int n_st = (cnt + 31) / 32;
+  const int st_off = block_exclusive_scan(e < E ? n_st : 0, s_warp);
   if (e < E) {
     s_cnt[e] = cnt;
     counts[e] = cnt;
@@ -152,11 +154,18 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
       mu[3 * (mu_off + i) + 1] = off + 256 * i;
       mu[3 * (mu_off + i) + 2] = min(256, padded - 256 * i);
     }
+    int32_t* st = tiles + kTileHeader + 2 * mt_cap + E + 3 * mt_cap;
+    for (int i = 0; i < n_st; ++i) {
+      st[3 * (st_off + i)] = e;
+      st[3 * (st_off + i) + 1] = off + 32 * i;
+      st[3 * (st_off + i) + 2] = min(32, cnt - 32 * i);
+    }
     if (e == E - 1) {
       offsets[E] = off + padded;
       tiles[0] = mt_off + padded / 128;
       tiles[1] = off + padded;
       tiles[2] = mu_off + n_mu;
+      tiles[3] = st_off + n_st;
     }
   }
   __syncthreads();

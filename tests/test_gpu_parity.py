@@ -31,6 +31,13 @@ SMALL = {
     # r = 24 (padded to 32), H and I not multiples of 128 (half-empty output tiles)
     "medium_r24": inputs.Config("medium_r24", E=6, H=192, I=320, top_k=3, T=257, r=24, alpha=48.0,
                                 routing="normal", seed=33),
+    # decode-sized batches (T*k <= 16*E) take the weight-streaming forward:
+    # Zipf skew puts several 32-slot tiles on the popular experts; r = 64
+    "stream_zipf_r64": inputs.Config("stream_zipf_r64", E=64, H=256, I=192, top_k=8, T=100, r=64,
+                                     alpha=128.0, routing="zipf", seed=34),
+    # r = 24, H not a multiple of 128 (half-empty down tile), a few slots per expert
+    "stream_r24": inputs.Config("stream_r24", E=16, H=192, I=128, top_k=2, T=64, r=24, alpha=48.0,
+                                routing="normal", seed=35),
 }
 
 
