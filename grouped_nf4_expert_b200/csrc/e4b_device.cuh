@@ -32,6 +32,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Bounded waits measure elapsed time with the SM cycle counter, which is
+// cheap to read (the global timer is not).  A limit of T ns is taken as 2T
+// cycles: at least T ns at any SM clock up to 2 GHz.
+__device__ __forceinline__ long long wait_limit_cycles(long long timeout_ns) { return 2 * timeout_ns; }
+
 __device__ __forceinline__ void record_error(DeviceError* err, int code, int site) {
   if (err != nullptr) {
     if (atomicCAS(&err->code, 0, code) == 0) {
@@ -114,11 +119,30 @@ constexpr uint32_t kWaitSleepNs = 20000;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, CtaControl* ctl,
                                           DeviceError* err, long long timeout_ns, int site) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long c0 = clock64(), limit = wait_limit_cycles(timeout_ns);
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (ctl->abort) return false;
-    if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
+    if (clock64() - c0 > limit) {
+      ctl->abort = 1;
+      record_error(err, E4B_ERR_DEVICE_TIMEOUT, site);
+      return false;
+    }
+  }
+}
+
+// Bounded wait for roles off the critical path (producers far ahead of their
+// consumers, epilogues waiting for a whole tile): sleeps `sleep_ns` between
+// polls so that the decoding warps get the issue slots.
+__device__ __forceinline__ bool mbar_wait_lazy(uint64_t* bar, uint32_t parity, CtaControl* ctl, DeviceError* err,
+                                               long long timeout_ns, int site, uint32_t sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long c0 = clock64(), limit = wait_limit_cycles(timeout_ns);
+  while (true) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (ctl->abort) return false;
+    if (clock64() - c0 > limit) {
       ctl->abort = 1;
       record_error(err, E4B_ERR_DEVICE_TIMEOUT, site);
       return false;
@@ -191,11 +215,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, CtaControl* ctl,
                                                   DeviceError* err, long long timeout_ns, int site) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long c0 = clock64(), limit = wait_limit_cycles(timeout_ns);
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if (ctl->abort) return false;
-    if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
+    if (clock64() - c0 > limit) {
       ctl->abort = 1;
       record_error(err, E4B_ERR_DEVICE_TIMEOUT, site);
       return false;
@@ -241,6 +265,10 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 // arrival is pre-counted in the barrier's expected count (.noinc).
 __device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// 16-byte variant: both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -353,6 +381,35 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Whole warp: each thread writes 32 consecutive 32-bit columns of its own
+// TMEM lane (the warp's 32-lane quadrant), then waits for the writes.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulation.  A is
+// M lanes x K/2 columns, two consecutive K elements per 32-bit column (the
+// lower-index element in the low half).
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // UMMA descriptors
 // ----------------------------------------------------------------------------
@@ -455,16 +512,48 @@ __device__ __forceinline__ Nf4Planes nf4_block_planes(float absmax) {
   return p;
 }
 
+// Powers of two the decoder multiplies by to move bits right.  They are read
+// at run time so that the compiler keeps the multiplications, which run on
+// the FMA pipe, instead of turning them into shifts on the integer ALU pipe
+// that the table lookups below already fill.
+struct Nf4Shift {
+  uint32_t k16;  // 2^16: hi(x * k16) = x >> 16
+  uint32_t k31;  // 2^31: hi(x * k31) = x >> 1
+};
+__device__ __forceinline__ Nf4Shift nf4_shift_consts() {
+  uint32_t dyn;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+  const uint32_t z = dyn >> 31;  // 0: no launch has 2 GiB of shared memory
+  return {65536u >> z, 0x80000000u >> z};
+}
+__device__ __forceinline__ uint32_t mul_hi_u32(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t mad_hi_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // Decodes the 8 codes of one little-endian 32-bit word (bytes b0..b3,
 // element 2m = high nibble of byte m) into 4 bf16x2 words holding elements
 // (0,1), (2,3), (4,5), (6,7) -- lower element in the low half.
-__device__ __forceinline__ void nf4_decode_word(uint32_t w, const Nf4Planes& p, uint32_t* out) {
+//
+// Each byte plane is a 16-entry table split in two 8-byte halves: one byte
+// permute looks up codes 0..7 (selector = the code), one looks up 8..15
+// (selector = code ^ 8), a third picks per byte by bit 3 of the code, and two
+// more interleave the low and high bytes into bf16 pairs.
+__device__ __forceinline__ void nf4_decode_word(uint32_t w, const Nf4Planes& p, Nf4Shift k, uint32_t* out) {
+  const uint32_t wx = w ^ 0x88888888u;                               // codes 8..15 -> 0..7
+  const uint32_t wp = mad_hi_u32(w & 0x88888888u, k.k31, 0x32103210u);  // byte i from lookup 0..7 or 8..15
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     // Selector nibbles i = 0..3 hold the codes of elements 1, 0, 3, 2 of this half.
-    const uint32_t s = (h == 0) ? w : (w >> 16);
-    const uint32_t s_hi = s ^ 0x8888u;                       // codes 8..15 -> 0..7
-    const uint32_t pick = ((s >> 1) & 0x4444u) | 0x3210u;    // byte i from the 0..7 or 8..15 lookup
+    const uint32_t s = (h == 0) ? w : mul_hi_u32(w, k.k16);
+    const uint32_t s_hi = (h == 0) ? wx : mul_hi_u32(wx, k.k16);
+    const uint32_t pick = (h == 0) ? wp : mul_hi_u32(wp, k.k16);
     const uint32_t xl = prmt(p.lo[0], p.lo[1], s);
     const uint32_t yl = prmt(p.lo[2], p.lo[3], s_hi);
     const uint32_t xh = prmt(p.hi[0], p.hi[1], s);
@@ -479,8 +568,13 @@ __device__ __forceinline__ void nf4_decode_word(uint32_t w, const Nf4Planes& p, 
 // Decodes one block: 32 bytes of codes (as 8 words) -> 64 bf16 (32 words).
 __device__ __forceinline__ void nf4_decode_block(const uint32_t (&codes)[8], float absmax, uint32_t (&out)[32]) {
   const Nf4Planes p = nf4_block_planes(absmax);
+  const Nf4Shift k = nf4_shift_consts();
 #pragma unroll
-  for (int i = 0; i < 8; ++i) nf4_decode_word(codes[i], p, &out[4 * i]);
+  for (int i = 0; i < 8; ++i) nf4_decode_word(codes[i], p, k, &out[4 * i]);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // Writes 64 bf16 (one 128-byte row of a 128B-swizzled atom) to shared memory:

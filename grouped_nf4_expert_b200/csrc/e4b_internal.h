@@ -134,7 +134,7 @@ cudaError_t map_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_
 cudaError_t map_bf16_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
                         uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 cudaError_t map_u8_3d(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t rows, uint64_t E,
-                      uint32_t box_bytes, uint32_t box_rows);
+                      uint32_t box_bytes, uint32_t box_rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE);
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda).
 cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,

@@ -912,12 +912,11 @@ cudaError_t map_bf16_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_
 
 // 3-D byte stack [E, rows, bytes].
 cudaError_t map_u8_3d(CUtensorMap* m, const void* base, uint64_t bytes, uint64_t rows, uint64_t E,
-                      uint32_t box_bytes, uint32_t box_rows) {
+                      uint32_t box_bytes, uint32_t box_rows, CUtensorMapSwizzle swz) {
   const uint64_t dims[3] = {bytes, rows, E};
   const uint64_t strides[2] = {bytes, bytes * rows};
   const uint32_t box[3] = {box_bytes, box_rows, 1};
-  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, swz);
 }
 
 namespace {

@@ -4,11 +4,19 @@
 // reading every touched expert's NF4 weights once.  Here the weights are the
 // UMMA M operand (128 weight rows per tile, decoded into shared memory) and
 // up to 32 routed slots of one expert are the N operand, so each weight byte is
-// fetched and decoded once per 32 slots.  Deep rings of NF4 code tiles and of
-// activation-row tiles keep enough memory traffic in flight; a shorter ring
-// holds the decoded tiles the UMMAs consume.  Same exact decode routine, same outputs as the training
-// tiles (gu / act for gate_up, y_perm for down), with the LoRA term as K = r
-// UMMAs into the same accumulator.
+// fetched and decoded once per 32 slots.  Decoded tiles go to tensor memory,
+// which the UMMA reads as its A operand.  A code stage holds 4 k-chunks, so
+// every weight row contributes one whole 128-byte line (and one 16-byte run
+// of block scales) per stage; rings of code stages and of activation-row tiles
+// keep enough memory traffic in flight.
+//
+// Three teams of four decode warps take the code stages round robin, so that
+// while one team waits on its barriers the other two decode; a team writes
+// the decoded rows of its stage's four k-chunks straight into its own A
+// buffer in tensor memory, and one warp issues every stage's UMMAs in order
+// with those tiles as the A operand read from tensor memory.  Outputs match the training tiles (gu /
+// act for gate_up, y_perm for down), with the LoRA term as K = r UMMAs into
+// the same accumulator.
 //
 // Pages: "How do I QLoRA-train the fused experts of a MoE", section "The
 // abstraction that fails" (per-expert delta before the activation) and
@@ -27,36 +35,43 @@ namespace nf4s {
 constexpr int BM = 128;          // weight rows per tile (UMMA M)
 constexpr int BN = 32;           // routed slots per tile (UMMA N)
 constexpr int BK = 64;
-constexpr int RAW_STAGES = 16;   // NF4 codes + absmax (the HBM stream)
-constexpr int AB_STAGES = 4;     // decoded weights
-constexpr int X_STAGES = 12;     // activation rows (prefetched like the codes)
-constexpr int RAW_BYTES = BM * BK / 2;                 // 4096
-constexpr int AMAX_BYTES = BM * 4;                     // 512
-constexpr int RAW_SLOT = RAW_BYTES + AMAX_BYTES;       // 4608 (128-byte multiple)
-constexpr int A_BYTES = BM * BK * 2;                   // 16384, K-major SW128
-constexpr int X_BYTES = BN * BK * 2;                   // 4096, K-major SW128
+constexpr int RAW_CHUNKS = 4;    // k-chunks per code stage: 128 contiguous code bytes per weight row
+constexpr int kTeams = 3;        // decode teams of 4 warps (one per TMEM lane quadrant)
+constexpr int RAW_STAGES = 6;    // NF4 codes + absmax (the HBM stream); slot r always goes to team r % 3
+constexpr int X_STAGES = 4;      // activation rows of a code stage's 4 chunks (prefetched like the codes)
+constexpr int CODE_BYTES = BM * RAW_CHUNKS * BK / 2;   // 16384, 128B-swizzled rows of 128 bytes
+constexpr int AMAX_BYTES = BM * RAW_CHUNKS * 4;        // 2048, 4 block scales per row
+constexpr int RAW_SLOT = CODE_BYTES + AMAX_BYTES;      // 18432 (1024-byte multiple)
+constexpr int X_BYTES = BN * BK * 2;                   // 4096 per chunk, K-major SW128
+constexpr int XS_BYTES = RAW_CHUNKS * X_BYTES;         // 16384 per stage
 
 constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;        // LoRA B rows of the tile (UMMA A of the K=r step)
 constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;        // p rows of the slots (UMMA B of the K=r step)
 constexpr int EPI_BYTES = 64 * BN * 4;                 // up values handed to the gate lanes
 constexpr int RAW_OFF = 0;
-constexpr int AB_OFF = RAW_STAGES * RAW_SLOT;          // 73728, 1024-aligned
-constexpr int X_OFF = AB_OFF + AB_STAGES * A_BYTES;
-constexpr int LA_OFF = X_OFF + X_STAGES * X_BYTES;
+constexpr int X_OFF = RAW_STAGES * RAW_SLOT;           // 147456, 1024-aligned
+constexpr int LA_OFF = X_OFF + X_STAGES * XS_BYTES;
 constexpr int LB_OFF = LA_OFF + LA_BYTES;
 constexpr int EPI_OFF = LB_OFF + LB_BYTES;
 constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
 constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;
-constexpr int kDecodeGroups = 4;  // groups of 4 warps; group g decodes the k-chunks j with j % 4 == g
-constexpr int kEpiWarp0 = 4 + 4 * kDecodeGroups;
+constexpr int kEpiWarp0 = 4 + 4 * kTeams;
 // warp 0 codes, warp 1 UMMA, warp 2 activations + LoRA, 4.. decode, last 4 epilogue
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
-constexpr int kTmemCols = 64;   // 2 accumulator buffers x 32 columns
+// TMEM columns: 2 accumulator buffers x 32 slot columns at 0, then one A
+// buffer per team (4 chunks x 32 columns = 4 x 64 bf16 per lane) from 128.
+constexpr int kAccCols = BN;
+constexpr int kACols = BK / 2;
+constexpr int kAOff = 128;
+constexpr int kTeamCols = RAW_CHUNKS * kACols;         // 128
+constexpr int kTmemCols = 512;
 constexpr int kRawFullCount = 1 + 32;
-static_assert(AB_OFF % 1024 == 0 && X_OFF % 1024 == 0 && LA_OFF % 1024 == 0 && LB_OFF % 1024 == 0,
-              "swizzle atom alignment");
-static_assert(RAW_STAGES % kDecodeGroups == 0 && AB_STAGES % kDecodeGroups == 0,
-              "each ring slot must belong to one decode group");
+static_assert(X_OFF % 1024 == 0 && LA_OFF % 1024 == 0 && LB_OFF % 1024 == 0, "swizzle atom alignment");
+static_assert(kTmemCols == 512, "one CTA per SM owns all of TMEM");
+static_assert(SMEM_BYTES > 232448 / 2, "shared memory keeps one CTA per SM (TMEM is not shared)");
+static_assert(RAW_STAGES % kTeams == 0, "each code slot belongs to one team (no phase aliasing)");
+static_assert(kAOff + kTeams * kTeamCols <= kTmemCols && 2 * kAccCols <= kAOff, "TMEM budget");
+static_assert(RAW_SLOT % 1024 == 0, "code tiles are 128B-swizzled");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace nf4s
 
@@ -83,20 +98,20 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
   uint8_t* smem = align1024(smem_dyn);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* raw_full = bars;                         // [RAW_STAGES] codes + absmax landed
-  uint64_t* raw_empty = raw_full + RAW_STAGES;       // [RAW_STAGES] codes decoded
-  uint64_t* a_full = raw_empty + RAW_STAGES;         // [AB_STAGES] decoded tile written
-  uint64_t* ab_empty = a_full + AB_STAGES;           // [AB_STAGES] decoded tile consumed by the UMMAs
-  uint64_t* x_full = ab_empty + AB_STAGES;           // [X_STAGES] activation rows landed
+  uint64_t* raw_empty = raw_full + RAW_STAGES;       // [RAW_STAGES] codes read into registers (team's 4 warps)
+  uint64_t* a_ready = raw_empty + RAW_STAGES;        // [kTeams] team's decoded stage written (4 warps)
+  uint64_t* a_empty = a_ready + kTeams;              // [kTeams] team's A buffer consumed by the UMMAs
+  uint64_t* x_full = a_empty + kTeams;               // [X_STAGES] activation rows landed
   uint64_t* x_empty = x_full + X_STAGES;             // [X_STAGES] activation rows consumed
-  uint64_t* lfull = x_empty + X_STAGES;              // LoRA operands landed
+  uint64_t* drain = x_empty + X_STAGES;              // every UMMA completed
+  uint64_t* lfull = drain + 1;                       // LoRA operands landed
   uint64_t* lempty = lfull + 1;                      // LoRA operands consumed
-  uint64_t* accfull = lfull + 2;                     // [2]
-  uint64_t* accempty = lfull + 4;                    // [2]
+  uint64_t* accfull = lfull + 2;                     // [2] accumulator final
+  uint64_t* accempty = lfull + 4;                    // [2] epilogue read the accumulators
   uint64_t* epi_full = lfull + 6;                    // up values in EPI
   uint64_t* epi_empty = lfull + 7;                   // up values consumed
-  uint64_t* drain = lfull + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 9);
-  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 10);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 8);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 9);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -104,14 +119,15 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
       mbar_init(&raw_full[s], kRawFullCount);
       mbar_init(&raw_empty[s], 4);
     }
-    for (int s = 0; s < AB_STAGES; ++s) {
-      mbar_init(&a_full[s], 4);
-      mbar_init(&ab_empty[s], 1);
+    for (int m = 0; m < kTeams; ++m) {
+      mbar_init(&a_ready[m], 4);
+      mbar_init(&a_empty[m], 1);
     }
     for (int s = 0; s < X_STAGES; ++s) {
       mbar_init(&x_full[s], 1);
       mbar_init(&x_empty[s], 1);
     }
+    mbar_init(drain, 1);
     mbar_init(lfull, 1);
     mbar_init(lempty, 1);
     for (int b = 0; b < 2; ++b) {
@@ -120,7 +136,6 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
     }
     mbar_init(epi_full, 2);
     mbar_init(epi_empty, 2);
-    mbar_init(drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -137,6 +152,10 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
   const int n_units = p.tiles[3] * p.n_mt;
   const int kchunks = p.K / BK;
   const int blocks_per_row = p.stored_cols / 64;
+  const int nq = (kchunks + RAW_CHUNKS - 1) / RAW_CHUNKS;  // code stages per unit; the last may be partial
+  // Block scales of a full stage are one aligned 16-byte run per row when
+  // rows hold a multiple of 4 blocks.
+  const bool amax16 = (kchunks % RAW_CHUNKS) == 0 && (reinterpret_cast<uintptr_t>(p.absmax) & 15u) == 0;
 
   // Stored weight rows of tile mt: two 64-row halves.
   auto rows_of = [&](int mt, int& rA, int& rB) {
@@ -161,23 +180,31 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
       if (u + (int)gridDim.x < n_units) e_next = stiles[3 * ((u + gridDim.x) / p.n_mt)];
       int rA, rB;
       rows_of(mt, rA, rB);
-      for (int kc = 0; kc < kchunks; ++kc, ++j) {
+      for (int q = 0; q < nq; ++q, ++j) {
         const uint32_t r = j % RAW_STAGES, ph = (j / RAW_STAGES) & 1;
-        ok = __all_sync(kFull, mbar_wait(&raw_empty[r], ph ^ 1, ctl, p.err, p.timeout_ns, 310));
+        ok = __all_sync(kFull, mbar_wait_lazy(&raw_empty[r], ph ^ 1, ctl, p.err, p.timeout_ns, 310, 128));
         if (!ok) break;
         uint8_t* slot = smem + RAW_OFF + r * RAW_SLOT;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[r], RAW_BYTES);
-          tma_load_3d(slot, &map_raw, &raw_full[r], kc * (BK / 2), rA, e);
-          tma_load_3d(slot + RAW_BYTES / 2, &map_raw, &raw_full[r], kc * (BK / 2), rB, e);
+          // Codes past the end of a row (a partial last stage) are zero-filled.
+          mbar_arrive_expect_tx(&raw_full[r], CODE_BYTES);
+          tma_load_3d(slot, &map_raw, &raw_full[r], q * (RAW_CHUNKS * BK / 2), rA, e);
+          tma_load_3d(slot + CODE_BYTES / 2, &map_raw, &raw_full[r], q * (RAW_CHUNKS * BK / 2), rB, e);
         }
-        float* amax = reinterpret_cast<float*>(slot + RAW_BYTES);
+        float* amax = reinterpret_cast<float*>(slot + CODE_BYTES);
+        const int nb = min(RAW_CHUNKS, kchunks - q * RAW_CHUNKS);
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           const int t = lane + 32 * qq;
           const int srow = (t < 64) ? rA + t : rB + (t - 64);
-          if (srow < p.stored_rows)
-            cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + kc);
+          if (srow < p.stored_rows) {
+            const float* src = p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + q * RAW_CHUNKS;
+            if (amax16) {
+              cp_async_16(amax + t * RAW_CHUNKS, src);
+            } else {
+              for (int c = 0; c < nb; ++c) cp_async_4(amax + t * RAW_CHUNKS + c, src + c);
+            }
+          }
         }
         cp_async_arrive_noinc(&raw_full[r]);
         issued |= 1u << r;
@@ -206,17 +233,20 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
         const int e = stiles[3 * st], row0 = stiles[3 * st + 1];
         int rA, rB;
         rows_of(mt, rA, rB);
-        if (!(ok = mbar_wait(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 320))) break;
+        if (!(ok = mbar_wait_lazy(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 320, 128))) break;
         mbar_arrive_expect_tx(lfull, (uint32_t)((BM + BN) * 2 * p.r_pad));
         uint8_t* la = smem + LA_OFF;
         tma_load_3d(la, &map_lw, lfull, 0, rA, e);
         tma_load_3d(la + 128 * p.r_pad, &map_lw, lfull, 0, rB, e);
         tma_load_2d(smem + LB_OFF, &map_lp, lfull, 0, row0);
-        for (int kc = 0; kc < kchunks; ++kc, ++j) {
+        for (int q = 0; q < nq; ++q, ++j) {
           const uint32_t s = j % X_STAGES, ph = (j / X_STAGES) & 1;
-          if (!(ok = mbar_wait(&x_empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 321))) break;
-          mbar_arrive_expect_tx(&x_full[s], X_BYTES);
-          tma_load_2d(smem + X_OFF + s * X_BYTES, &map_x, &x_full[s], kc * BK, row0);
+          if (!(ok = mbar_wait_lazy(&x_empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 321, 128))) break;
+          const int nb = min(RAW_CHUNKS, kchunks - q * RAW_CHUNKS);
+          mbar_arrive_expect_tx(&x_full[s], (uint32_t)(nb * X_BYTES));
+          for (int c = 0; c < nb; ++c)
+            tma_load_2d(smem + X_OFF + s * XS_BYTES + c * X_BYTES, &map_x, &x_full[s], (q * RAW_CHUNKS + c) * BK,
+                        row0);
           issued |= 1u << s;
           last_par = (last_par & ~(1u << s)) | (ph << s);
         }
@@ -236,38 +266,45 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
     const uint32_t idesc = make_idesc_bf16(BM, BN, false, false);
     const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
     const uint32_t la_u = smem_u32(smem + LA_OFF), lb_u = smem_u32(smem + LB_OFF);
-    const uint32_t ab_u = smem_u32(smem + AB_OFF), x_u = smem_u32(smem + X_OFF);
-    uint32_t j = 0, ti = 0;
+    const uint64_t xdesc0 = make_sdesc(smem_u32(smem + X_OFF), 16, 1024, kSw128);
+    uint32_t ti = 0, rq = 0, xs = 0, xph = 0;  // units, code stages, activation ring slot and parity
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
       const uint32_t b = ti & 1, use = ti >> 1;
-      const uint32_t d = tmem + b * BN;
+      const uint32_t d = tmem + b * kAccCols;
       if (!(ok = __all_sync(kFull, mbar_wait(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 330)))) break;
       if (!(ok = __all_sync(kFull, mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 331)))) break;
       tc_fence_after();
       if (elect_one_sync()) {
-        for (int ks = 0; ks < p.r_pad / 16; ++ks)
-          umma_bf16(d, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz),
-                    make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz), idesc, ks > 0 ? 1u : 0u);
+        for (int k = 0; k < p.r_pad / 16; ++k)
+          umma_bf16(d, make_sdesc(la_u + 32 * k, 16, 16 * p.r_pad, lswz),
+                    make_sdesc(lb_u + 32 * k, 16, 16 * p.r_pad, lswz), idesc, k > 0 ? 1u : 0u);
         umma_commit(lempty);
       }
       __syncwarp();
-      for (int kc = 0; kc < kchunks; ++kc, ++j) {
-        const uint32_t s = j % AB_STAGES, ph = (j / AB_STAGES) & 1;
-        const uint32_t xs = j % X_STAGES, xph = (j / X_STAGES) & 1;
-        if (!(ok = __all_sync(kFull, mbar_wait(&a_full[s], ph, ctl, p.err, p.timeout_ns, 332)))) break;
-        if (!(ok = __all_sync(kFull, mbar_wait(&x_full[xs], xph, ctl, p.err, p.timeout_ns, 333)))) break;
+      for (int q = 0; q < nq; ++q, ++rq) {
+        const uint32_t team = rq % kTeams, aph = (rq / kTeams) & 1;
+        ok = __all_sync(kFull, mbar_wait(&a_ready[team], aph, ctl, p.err, p.timeout_ns, 332));
+        if (ok) ok = __all_sync(kFull, mbar_wait(&x_full[xs], xph, ctl, p.err, p.timeout_ns, 333));
+        if (!ok) break;
         tc_fence_after();
-        const uint64_t adesc = make_sdesc(ab_u + s * A_BYTES, 16, 1024, kSw128);
-        const uint64_t xdesc = make_sdesc(x_u + xs * X_BYTES, 16, 1024, kSw128);
         if (elect_one_sync()) {
+          const int nb = min(RAW_CHUNKS, kchunks - q * RAW_CHUNKS);
+          const uint32_t a_col = tmem + kAOff + team * kTeamCols;
+          const uint64_t xdesc = xdesc0 + (uint64_t)((xs * XS_BYTES) >> 4);
+          for (int c = 0; c < nb; ++c)
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K = +2 in the address field
-            umma_bf16(d, adesc + 2 * kk, xdesc + 2 * kk, idesc, 1u);
-          umma_commit(&ab_empty[s]);
+            for (int kk = 0; kk < BK / 16; ++kk)  // K16 step: 8 TMEM columns of A, +32 bytes of x
+              umma_bf16_ta(d, a_col + c * kACols + 8 * kk, xdesc + (uint64_t)(c * (X_BYTES >> 4) + 2 * kk), idesc,
+                           1u);
+          umma_commit(&a_empty[team]);
           umma_commit(&x_empty[xs]);
         }
         __syncwarp();
+        if (++xs == X_STAGES) {
+          xs = 0;
+          xph ^= 1;
+        }
       }
       if (!ok) break;
       if (elect_one_sync()) umma_commit(&accfull[b]);
@@ -279,46 +316,58 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
     while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
     }
   } else if (warp >= 4 && warp < kEpiWarp0) {
-    // ------------------------------------------------ NF4 decode, groups take k-chunks round robin
-    const uint32_t grp = (uint32_t)(warp - 4) >> 2;
-    const int t = (threadIdx.x - 128) & 127;  // weight row of the tile
-    uint32_t j = 0;
+    // ------------------------------------------------ NF4 decode into TMEM, teams take code stages round robin
+    // Team m decodes every code stage rq with rq % 3 == m; thread t owns
+    // weight row t, which is TMEM lane t, and writes the stage's decoded
+    // rows (4 k-chunks x 64 bf16) straight into the team's A buffer there.
+    const uint32_t team = (uint32_t)(warp - 4) >> 2;
+    const int t = (threadIdx.x - 128) & 127;
+    const Nf4Shift ks = nf4_shift_consts();
+    const uint32_t a_base = tmem + kAOff + team * kTeamCols + ((uint32_t)(warp & 3) * 32u << 16);
+    uint32_t rq = 0, tuse = 0;  // code stages seen, stages this team decoded
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const int mt = u % p.n_mt;
       int rA, rB;
       rows_of(mt, rA, rB);
       const bool valid = ((t < 64) ? rA + t : rB + (t - 64)) < p.stored_rows;
-      for (int kc = 0; kc < kchunks; ++kc, ++j) {
-        if (j % kDecodeGroups != grp) continue;
-        const uint32_t r = j % RAW_STAGES, rph = (j / RAW_STAGES) & 1;
-        const uint32_t s = j % AB_STAGES, sph = (j / AB_STAGES) & 1;
+      for (int q = 0; q < nq; ++q, ++rq) {
+        if (rq % kTeams != team) continue;
+        const uint32_t r = rq % RAW_STAGES, rph = (rq / RAW_STAGES) & 1;
+        const uint32_t aph = tuse++ & 1;
+        const int nb = min(RAW_CHUNKS, kchunks - q * RAW_CHUNKS);  // a partial last stage has fewer chunks
         ok = __all_sync(kFull, mbar_wait(&raw_full[r], rph, ctl, p.err, p.timeout_ns, 340));
-        if (ok) ok = __all_sync(kFull, mbar_wait(&ab_empty[s], sph ^ 1, ctl, p.err, p.timeout_ns, 341));
         if (!ok) break;
         const uint8_t* slot = smem + RAW_OFF + r * RAW_SLOT;
-        uint8_t* arow = smem + AB_OFF + s * A_BYTES + (t >> 3) * 1024 + (t & 7) * 128;
-        if (valid) {
-          const uint4 q0 = *reinterpret_cast<const uint4*>(slot + t * 32);
-          const uint4 q1 = *reinterpret_cast<const uint4*>(slot + t * 32 + 16);
-          const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-          const Nf4Planes pl = nf4_block_planes(reinterpret_cast<const float*>(slot + RAW_BYTES)[t]);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {  // 16-byte chunk c of the 128-byte row, 128B-swizzled
-            uint32_t w4[4];
-            nf4_decode_word(codes[c], pl, w4);
-            *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        const uint8_t* crow = slot + t * 128;  // 128B-swizzled: 16-byte piece c sits at c ^ (t % 8)
+        const float* amax = reinterpret_cast<const float*>(slot + CODE_BYTES) + t * RAW_CHUNKS;
+        for (int c = 0; c < nb; ++c) {
+          const uint4 q0 = *reinterpret_cast<const uint4*>(crow + (((2 * c) ^ (t & 7)) << 4));
+          const uint4 q1 = *reinterpret_cast<const uint4*>(crow + (((2 * c + 1) ^ (t & 7)) << 4));
+          const float a = amax[c];
+          if (c == nb - 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&raw_empty[r]);  // the stage's codes are in registers
           }
-        } else {
+          const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          // Rows past the end of the matrix get a zero scale, so every entry
+          // of their table (and every decoded weight) is zero whatever the codes.
+          const Nf4Planes pl = nf4_block_planes(valid ? a : 0.0f);
+          uint32_t v[32];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(arow + (c << 4)) = make_uint4(0u, 0u, 0u, 0u);
+          for (int i = 0; i < 8; ++i) nf4_decode_word(codes[i], pl, ks, &v[4 * i]);
+          if (c == 0) {
+            // The UMMAs of this team's previous stage have finished reading the buffer.
+            ok = __all_sync(kFull, mbar_wait(&a_empty[team], aph ^ 1, ctl, p.err, p.timeout_ns, 341));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          tmem_st32(a_base + c * kACols, v);
         }
-        fence_proxy_async_smem();
+        if (!ok) break;
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&raw_empty[r]);
-          mbar_arrive(&a_full[s]);
-        }
+        if (lane == 0) mbar_arrive(&a_ready[team]);
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -332,13 +381,13 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
       const int st = u / p.n_mt, mt = u % p.n_mt;
       const size_t row0 = (size_t)stiles[3 * st + 1];
       const uint32_t b = ti & 1, use = ti >> 1;
-      ok = __all_sync(kFull, mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 350));
+      ok = __all_sync(kFull, mbar_wait_lazy(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 350, 256));
       if (!ok) break;
       tc_fence_after();
       float v[32];
       {
         float v0[16], v1[16];
-        const uint32_t tl = tmem + b * BN + ((uint32_t)(qrt * 32) << 16);
+        const uint32_t tl = tmem + b * kAccCols + ((uint32_t)(qrt * 32) << 16);
         tmem_ld16(tl, v0);
         tmem_ld16(tl + 16, v1);
 #pragma unroll
@@ -409,7 +458,9 @@ cudaError_t launch_nf4_stream(const Nf4GemmHost& h, int num_sms, cudaStream_t st
   const CUtensorMapSwizzle rswz = swizzle_for_bytes(2 * h.r_pad);
   if ((err = map_bf16_2d(&mx, h.act_in, h.K, h.rows_cap, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
     return err;
-  if ((err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 32, 64)) != cudaSuccess) return err;
+  if ((err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, RAW_CHUNKS * BK / 2, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+    return err;
   if ((err = map_bf16_3d(&mlw, h.lora_w, h.r, h.stored_rows, h.E, h.r_pad, 64, rswz)) != cudaSuccess) return err;
   if ((err = map_bf16_2d(&mlp, h.lora_a_rows, h.r, h.rows_cap, h.r_pad, BN, rswz)) != cudaSuccess) return err;
   Nf4StreamParams p;
