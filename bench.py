@@ -86,6 +86,20 @@ def step_flops(cfg):
     return base + lora
 
 
+def fwd_flops(cfg):
+    """Algorithmic FLOPs of the forward alone (gate_up, down and the forward LoRA terms)."""
+    N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
+    return 6.0 * N * H * I + 2.0 * N * r * (2 * H + 3 * I)
+
+
+def stream_bytes(cfg, touched):
+    """Algorithmic HBM bytes of the two streaming forward launches: the NF4 codes and
+    fp32 block scales of every expert the batch routes to, each read once."""
+    per_weight = 0.5 + 4.0 / 64
+    return {"nf4_stream_fwd_gate_up": touched * 2 * cfg.I * cfg.H * per_weight,
+            "nf4_stream_fwd_down": touched * cfg.H * cfg.I * per_weight}
+
+
 def nf4_gemm_flops(cfg):
     """Algorithmic FLOPs of the four grouped NF4 GEMM launches of one step."""
     N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
@@ -163,7 +177,8 @@ class ClockSampler:
 
 def oracle_sample_step(prob, tokens):
     """The CPU oracle as it stands on a token sample: forward + backward (dx and the
-    sample's LoRA-gradient contributions), dequantising the base in both passes."""
+    sample's LoRA-gradient contributions), dequantising the base in both passes;
+    the forward alone for a forward-only workload."""
     import numpy as np
 
     import oracle
@@ -174,7 +189,8 @@ def oracle_sample_step(prob, tokens):
                         f(prob.A_gu), f(prob.B_gu), f(prob.A_d), f(prob.B_d))
     x, dY = f(prob.x), f(prob.dY)
     oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=tokens)
-    oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=tokens, grad_experts=[])
+    if cfg.passes != ("fwd",):
+        oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=tokens, grad_experts=[])
 
 
 def blas_threads():
@@ -188,13 +204,19 @@ def blas_threads():
 
 def cpu_baseline(prob, n_tokens):
     import numpy as np
+    n_tokens = min(n_tokens, prob.cfg.T)
     toks = np.sort(np.random.default_rng(7).choice(prob.cfg.T, size=n_tokens, replace=False))
     t0 = time.perf_counter()
     oracle_sample_step(prob, toks)
     dt = time.perf_counter() - t0
     return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": "%d random tokens of the %s workload, forward + backward (input gradient and "
-                      "their LoRA-gradient terms), float64 numpy, %.1f s" % (n_tokens, prob.cfg.name, dt)}
+            "sample": "%d random tokens of the %s workload, %s, float64 numpy, %.1f s" % (
+                n_tokens, prob.cfg.name, passes_text(prob.cfg), dt)}
+
+
+def passes_text(cfg):
+    return ("forward only" if cfg.passes == ("fwd",)
+            else "forward + backward (input gradient and their LoRA-gradient terms)")
 
 
 def run_reference(args):
@@ -207,6 +229,7 @@ def run_reference(args):
     import numpy as np
     rng = np.random.default_rng(11)
     times = []
+    args.ref_tokens = min(args.ref_tokens, cfg.T)
     for i in range(args.warmup + args.steps):
         toks = np.sort(rng.choice(cfg.T, size=args.ref_tokens, replace=False))
         t0 = time.perf_counter()
@@ -216,8 +239,8 @@ def run_reference(args):
     total = sum(times)
     value = args.ref_tokens * args.steps / total
     cores = blas_threads()
-    sample = "%d random tokens per step of the %s workload, forward + backward, float64 numpy" % (
-        args.ref_tokens, cfg.name)
+    sample = "%d random tokens per step of the %s workload, %s, float64 numpy" % (
+        args.ref_tokens, cfg.name, passes_text(cfg))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
@@ -234,7 +257,7 @@ def workload_config(cfg, world, l2_note):
     return {"workload": "%s: %s" % (cfg.name, cfg.note), "E": cfg.E, "H": cfg.H, "I": cfg.I,
             "top_k": cfg.top_k, "tokens_per_gpu": cfg.T, "global_batch": cfg.T * world, "r": cfg.r,
             "alpha": cfg.alpha, "routing": cfg.routing, "nf4_blocksize": 64, "parallelism": "dp%d" % world,
-            "l2": l2_note}
+            "passes": list(cfg.passes), "l2": l2_note}
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -271,9 +294,13 @@ def main():
     base, lora = d.base(), d.lora()
     grads = (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d)
 
+    fwd_only = cfg.passes == ("fwd",)  # decode-sized serving batch: the forward alone
+
     def step():
         blk.e4b_route_permute(d.logits, d.x)
         blk.e4b_grouped_nf4_lora_fwd(base, lora)
+        if fwd_only:
+            return
         blk.e4b_grouped_nf4_lora_dgrad(base, lora, d.dY)
         blk.e4b_lora_wgrad()
         if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
@@ -317,7 +344,7 @@ def main():
         raise RuntimeError("device error in the timed region: %s" % e4b.STATUS.get(st, st))
     ms_per_step = total_ms / args.steps
     value = cfg.T * world * args.steps / (total_ms / 1e3)
-    flops = step_flops(cfg)
+    flops = fwd_flops(cfg) if fwd_only else step_flops(cfg)
 
     # ---- per-kernel device times over a second timed region (library profiler, events on the launch stream)
     e4b.e4b_profiler_enable(True)
@@ -340,6 +367,18 @@ def main():
                 "launches": nf4_launches,
                 "avg_launch_ms": nf4_ms / max(nf4_launches, 1),
                 "algorithmic_flop_per_step": sum(gflops.values())}
+    sbytes = stream_bytes(cfg, int((blk.counts > 0).sum().item()))
+    st_ms = sum(kern.get(n, (0, 0.0))[1] for n in sbytes)
+    if st_ms > 0:  # the weight-streaming forward ran: it is HBM-bound by design
+        st_launches = sum(kern.get(n, (0, 0.0))[0] for n in sbytes)
+        st_bytes = sum(sbytes.values()) * args.steps
+        ach = st_bytes / (st_ms / 1e3) / 1e9
+        roofline = {"kernel": "nf4_stream (fwd gate_up, fwd down)", "bound": "hbm", "achieved": ach,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                    "peak_source": "%s hbm_gbs" % peak_src, "traffic": None,
+                    "traffic_unit": "DRAM bytes per launch (ncu), see profiles/",
+                    "launches": st_launches, "avg_launch_ms": st_ms / max(st_launches, 1),
+                    "algorithmic_bytes_per_step": sum(sbytes.values())}
     per_kernel = {n: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
                       "share": v[1] / kern_total if kern_total else None} for n, v in kern.items()}
 
@@ -349,15 +388,17 @@ def main():
     hx.copy_(d.x)
     hl.copy_(d.logits)
     hdy.copy_(d.dY)
-    outs = [blk.y, blk.dx, blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d]
+    outs = [blk.y] if fwd_only else [blk.y, blk.dx, blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d]
     houts = [pin(t) for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in (hx, hl, hdy))
+    ins = (hx, hl) if fwd_only else (hx, hl, hdy)
+    h2d = sum(t.numel() * t.element_size() for t in ins)
     d2h = sum(t.numel() * t.element_size() for t in houts)
 
     def e2e_step():
         d.x.copy_(hx, non_blocking=True)
         d.logits.copy_(hl, non_blocking=True)
-        d.dY.copy_(hdy, non_blocking=True)
+        if not fwd_only:
+            d.dY.copy_(hdy, non_blocking=True)
         step()
         for h, t in zip(houts, outs):
             h.copy_(t, non_blocking=True)

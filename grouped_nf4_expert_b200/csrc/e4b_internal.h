@@ -11,7 +11,7 @@
 namespace e4b {
 
 // Tokens handled by one CTA of the routing kernels.
-constexpr int kRouteTokensPerBlock = 256;
+constexpr int kRouteTokensPerBlock = 64;
 // Header ints at the front of the tile list: [0] = m-tiles, [1] = rows used.
 constexpr int kTileHeader = 8;
 

@@ -20,9 +20,23 @@ __device__ __forceinline__ bool route_better(float av, int ae, float bv, int be)
   return av > bv || (av == bv && ae < be);
 }
 
+// Order-preserving unsigned key of a logit: larger value -> larger key, both
+// zeros -> the same key, NaN -> 0 (below every number, whose keys are >= 1).
+__device__ __forceinline__ uint32_t route_key(float v) {
+  if (isnan(v)) return 0u;
+  const uint32_t b = (v == 0.0f) ? 0u : __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float route_key_value(uint32_t key) {
+  if (key == 0u) return __int_as_float(0x7fc00000);
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 // One warp per token: k rounds of a warp-wide argmax over the unpicked
-// experts, then a softmax over the k selected logits.  The CTA also counts
-// the slots it produced per expert (order-independent shared counters).
+// experts (a max-reduction of the value keys, then a min-reduction of the
+// expert ids holding that key: ties go to the lower id), then a softmax over
+// the k selected logits.  The CTA also counts the slots it produced per
+// expert (order-independent shared counters).
 template <int EPL>
 __global__ void __launch_bounds__(1024) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                          int32_t* __restrict__ topk_ids,
@@ -36,39 +50,31 @@ __global__ void __launch_bounds__(1024) route_topk_kernel(const float* __restric
   const int t1 = min(T, t0 + kRouteTokensPerBlock);
   for (int t = t0 + warp; t < t1; t += nwarps) {
     const float* row = logits + (size_t)t * E;
-    float v[EPL];
-    uint32_t picked = 0;
+    uint32_t key[EPL];  // 0 once picked or past E (a NaN logit also has key 0, but keeps its id)
+    uint32_t live = 0;  // bit i: element i is a real, unpicked expert
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      v[i] = (e < E) ? row[e] : 0.0f;
-      if (e >= E) picked |= 1u << i;
+      key[i] = (e < E) ? route_key(__ldg(row + e)) : 0u;
+      if (e < E) live |= 1u << i;
     }
     float my_v = 0.0f;
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
-      float bv = __int_as_float(0x7fc00000);  // NaN: loses to everything
-      int be = 0x7fffffff;
+      // This lane's best live element: largest key, then lowest id (lowest i).
+      uint32_t bk = 0u, bi = 0xffffffffu;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        if (!(picked & (1u << i)) && route_better(v[i], lane + 32 * i, bv, be)) {
-          bv = v[i];
-          be = lane + 32 * i;
+      for (int i = 0; i < EPL; ++i)
+        if ((live & (1u << i)) && (bi == 0xffffffffu || key[i] > bk)) {
+          bk = key[i];
+          bi = (uint32_t)(lane + 32 * i);
         }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (route_better(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if ((be & 31) == lane) picked |= 1u << (be >> 5);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t e_sel = __reduce_min_sync(0xffffffffu, (bk == kmax) ? bi : 0xffffffffu);
+      if ((int)(e_sel & 31u) == lane) live &= ~(1u << (e_sel >> 5));
       if (lane == j) {
-        my_v = bv;
-        my_e = be;
+        my_v = route_key_value(kmax);
+        my_e = (int)e_sel;
       }
     }
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
@@ -178,7 +184,10 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
 
 // Stable scatter: one warp walks its CTA's slots in flat order, 32 at a time;
 // slots of the same expert inside a step are ranked by lane (match_any), and
-// a shared running count per expert carries the rank across steps.
+// a shared running count per expert carries the rank across steps.  The
+// warp's expert ids are loaded before the walk (kRouteTokensPerBlock * k /
+// 32 per lane).
+constexpr int kRankIdsPerLane = kRouteTokensPerBlock * E4B_MAX_TOP_K / 32;
 __global__ void __launch_bounds__(32) route_rank_kernel(const int32_t* __restrict__ topk_ids, int N, int E,
                                                         int slots_per_block,
                                                         const int32_t* __restrict__ block_base,
@@ -190,10 +199,19 @@ __global__ void __launch_bounds__(32) route_rank_kernel(const int32_t* __restric
   const int lane = threadIdx.x;
   const int f0 = blockIdx.x * slots_per_block;
   const int f1 = min(N, f0 + slots_per_block);
-  for (int base = f0; base < f1; base += 32) {
-    const int f = base + lane;
-    const bool valid = f < f1;
-    const int e = valid ? topk_ids[f] : -1;
+  const int steps = (f1 - f0 + 31) / 32;  // <= kRankIdsPerLane
+  int ids[kRankIdsPerLane];
+#pragma unroll
+  for (int s = 0; s < kRankIdsPerLane; ++s) {
+    const int f = f0 + 32 * s + lane;
+    ids[s] = (s < steps && f < f1) ? __ldg(topk_ids + f) : -1;
+  }
+#pragma unroll
+  for (int s = 0; s < kRankIdsPerLane; ++s) {
+    if (s >= steps) break;
+    const int f = f0 + 32 * s + lane;
+    const int e = ids[s];
+    const bool valid = e >= 0;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     const int leader = __ffs(peers) - 1;
@@ -215,56 +233,119 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 q, float w) {
   return q;
 }
 
+// One warp per permuted row (padding rows are zero-filled).  A row is moved
+// in batches of up to 8 16-byte pieces per lane (4 KB per warp), every load
+// of a batch issued before its stores; the next row's slot index is fetched
+// one row ahead.
+constexpr int kPiecesPerBatch = 8;
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ src,
                                                           const int32_t* __restrict__ slot_of_row,
                                                           const int32_t* __restrict__ tiles,
                                                           const float* __restrict__ scale_w, int H, int k,
                                                           uint16_t* __restrict__ dst) {
   const int rows_used = tiles[1];
-  const int vec = H / 8;
-  for (int row = blockIdx.x; row < rows_used; row += gridDim.x) {
-    const int slot = slot_of_row[row];
+  const int vec = H / 8;  // 16-byte pieces per row
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), nw = gridDim.x * (blockDim.x >> 5);
+  int slot = (gw < rows_used) ? __ldg(slot_of_row + gw) : -1;
+  for (int row = gw; row < rows_used; row += nw) {
+    const int next = (row + nw < rows_used) ? __ldg(slot_of_row + row + nw) : -1;
     uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
     if (slot < 0) {
-      for (int i = threadIdx.x; i < vec; i += blockDim.x) d[i] = make_uint4(0, 0, 0, 0);
+      for (int i = lane; i < vec; i += 32) d[i] = make_uint4(0, 0, 0, 0);
     } else {
       const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(slot / k) * H);
-      if (scale_w == nullptr) {
-        for (int i = threadIdx.x; i < vec; i += blockDim.x) d[i] = __ldg(s + i);
-      } else {
-        const float w = scale_w[slot];
-        for (int i = threadIdx.x; i < vec; i += blockDim.x) d[i] = scale_bf16x8(__ldg(s + i), w);
+      const float w = scale_w ? __ldg(scale_w + slot) : 1.0f;
+      for (int b0 = 0; b0 < vec; b0 += 32 * kPiecesPerBatch) {
+        uint4 q[kPiecesPerBatch];
+#pragma unroll
+        for (int i = 0; i < kPiecesPerBatch; ++i) {
+          const int pc = b0 + 32 * i + lane;
+          if (pc < vec) q[i] = __ldg(s + pc);
+        }
+#pragma unroll
+        for (int i = 0; i < kPiecesPerBatch; ++i) {
+          const int pc = b0 + 32 * i + lane;
+          if (pc < vec) d[pc] = scale_w ? scale_bf16x8(q[i], w) : q[i];
+        }
       }
     }
+    slot = next;
   }
 }
 
+// One warp per token: the k permuted rows are summed in slot order (weighted
+// by the routing weights for y, unweighted for dx) in fp32 per 16-byte piece;
+// the rows of a piece are loaded in groups of 8, all in flight together.
+constexpr int kRowsPerBatch = 8;
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ src_perm,
                                                       const int32_t* __restrict__ row_of_slot,
                                                       const float* __restrict__ topk_w, int T, int k, int H,
                                                       uint16_t* __restrict__ out) {
-  __shared__ int s_row[E4B_MAX_TOP_K];
-  __shared__ float s_w[E4B_MAX_TOP_K];
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), nw = gridDim.x * (blockDim.x >> 5);
   const int vec = H / 8;
-  for (int t = blockIdx.x; t < T; t += gridDim.x) {
-    __syncthreads();
-    if (threadIdx.x < k) {
-      s_row[threadIdx.x] = row_of_slot[(size_t)t * k + threadIdx.x];
-      s_w[threadIdx.x] = topk_w ? topk_w[(size_t)t * k + threadIdx.x] : 1.0f;
+  for (int t = gw; t < T; t += nw) {
+    // lane j < k holds slot j's permuted row and weight
+    const int my_row = (lane < k) ? __ldg(row_of_slot + (size_t)t * k + lane) : 0;
+    const float my_w = (lane < k) ? (topk_w ? __ldg(topk_w + (size_t)t * k + lane) : 1.0f) : 0.0f;
+    if (k <= kRowsPerBatch) {  // common case: the k row pointers and weights stay in registers
+      const uint4* rp[kRowsPerBatch];
+      float rw[kRowsPerBatch];
+#pragma unroll
+      for (int j = 0; j < kRowsPerBatch; ++j) {
+        rp[j] = reinterpret_cast<const uint4*>(src_perm + (size_t)__shfl_sync(0xffffffffu, my_row, j) * H);
+        rw[j] = __shfl_sync(0xffffffffu, my_w, j);
+      }
+      for (int pc = lane; pc < vec; pc += 32) {
+        uint4 q[kRowsPerBatch];
+#pragma unroll
+        for (int j = 0; j < kRowsPerBatch; ++j)
+          if (j < k) q[j] = __ldg(rp[j] + pc);
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kRowsPerBatch; ++j)
+          if (j < k) {
+            const uint32_t* p = reinterpret_cast<const uint32_t*>(&q[j]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              acc[2 * c] += rw[j] * bf16lo_to_f32(p[c]);
+              acc[2 * c + 1] += rw[j] * bf16hi_to_f32(p[c]);
+            }
+          }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4*>(out + (size_t)t * H)[pc] = o;
+      }
+      continue;
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < vec; i += blockDim.x) {
+    for (int pc = lane; pc < vec; pc += 32) {
       float acc[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-      for (int j = 0; j < k; ++j) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(src_perm + (size_t)s_row[j] * H) + i);
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(&q);
-        const float w = s_w[j];
+      for (int j0 = 0; j0 < k; j0 += kRowsPerBatch) {
+        uint4 q[kRowsPerBatch];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          acc[2 * c] += w * bf16lo_to_f32(p[c]);
-          acc[2 * c + 1] += w * bf16hi_to_f32(p[c]);
+        for (int j = 0; j < kRowsPerBatch; ++j) {
+          const int r = __shfl_sync(0xffffffffu, my_row, (j0 + j) & 31);
+          if (j0 + j < k) q[j] = __ldg(reinterpret_cast<const uint4*>(src_perm + (size_t)r * H) + pc);
+        }
+#pragma unroll
+        for (int j = 0; j < kRowsPerBatch; ++j) {
+          const float w = __shfl_sync(0xffffffffu, my_w, (j0 + j) & 31);
+          if (j0 + j < k) {
+            const uint32_t* p = reinterpret_cast<const uint32_t*>(&q[j]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              acc[2 * c] += w * bf16lo_to_f32(p[c]);
+              acc[2 * c + 1] += w * bf16hi_to_f32(p[c]);
+            }
+          }
         }
       }
       uint4 o;
@@ -272,7 +353,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       o.y = pack_bf16x2(acc[2], acc[3]);
       o.z = pack_bf16x2(acc[4], acc[5]);
       o.w = pack_bf16x2(acc[6], acc[7]);
-      reinterpret_cast<uint4*>(out + (size_t)t * H)[i] = o;
+      reinterpret_cast<uint4*>(out + (size_t)t * H)[pc] = o;
     }
   }
 }
@@ -354,7 +435,8 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
 cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, const int32_t* tiles,
                                const float* scale_w, int H, int k, int64_t rows_cap, uint16_t* dst, int num_sms,
                                cudaStream_t stream) {
-  const int64_t grid = rows_cap < (int64_t)num_sms * 8 ? rows_cap : (int64_t)num_sms * 8;
+  const int64_t blocks = (rows_cap + 7) / 8;  // 8 warps of 256 threads, a warp per row
+  const int64_t grid = blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8;
   LaunchScope scope(scale_w ? "gather_dyw" : "gather_x", stream);
   gather_rows_kernel<<<(int)grid, 256, 0, stream>>>(src, slot_of_row, tiles, scale_w, H, k, dst);
   return cudaGetLastError();
@@ -362,7 +444,8 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, 
 
 cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot, const float* topk_w, int T, int k,
                            int H, uint16_t* out, int num_sms, cudaStream_t stream) {
-  const int grid = T < num_sms * 8 ? T : num_sms * 8;
+  const int blocks = (T + 7) / 8;  // 8 warps of 256 threads, a warp per token
+  const int grid = blocks < num_sms * 8 ? blocks : num_sms * 8;
   LaunchScope scope(topk_w ? "combine_y" : "combine_dx", stream);
   combine_kernel<<<grid, 256, 0, stream>>>(src_perm, row_of_slot, topk_w, T, k, H, out);
   return cudaGetLastError();

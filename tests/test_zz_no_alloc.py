@@ -59,7 +59,7 @@ def test_noalloc_routing_matches_workspace_routing_twice_in_a_row():
 def test_noalloc_refuses_problems_beyond_its_fixed_scratch():
     fn = _noalloc_fn()
     dims = e4b.Dims(E=1024, H=64, I=64, top_k=2, r=8, alpha=16.0).c()
-    T = 256 * 600   # 2 * 600 blocks * 1024 experts > 1,048,576 entries
+    T = 256 * 600   # 2 * ceil(T / tokens-per-routing-block) * 1024 experts > 1,048,576 entries
     x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     routing = e4b.Routing(*([x.data_ptr()] * 7))
     st = fn(ctypes.byref(dims), T, x.data_ptr(), x.data_ptr(), ctypes.byref(routing), x.data_ptr(), None)
