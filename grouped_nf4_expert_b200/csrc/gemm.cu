@@ -72,39 +72,52 @@ __device__ __forceinline__ void load_bf16x16(const uint16_t* src, float (&v)[16]
 // activation tile and decodes weight rows (output columns) [128c, 128c+128)
 // of the tile; its TMEM receives its 128 rows x 256 columns.  Each CTA loads
 // only its own tiles (no multicast loads).
-// Roles per CTA: warp 0 = TMA + absmax copies, warp 1 = TMEM owner (both CTAs)
-// and UMMA issuer (even CTA only), warp 2 = LoRA-operand relay, warps 4-11 =
-// two decode groups on alternate k-chunks, warps 12-15 = epilogue.
+// Roles per CTA: warp 0 = NF4 codes + block scales into a ring of their own
+// (one slot per decode group, filled far ahead), warp 1 = TMEM owner (both
+// CTAs) and UMMA issuer (even CTA only), warp 2 = relay (odd CTA), warp 3 =
+// activation tiles and LoRA operands, warps 4-19 = four decode groups taking
+// the k-chunks round robin, warps 20-23 = epilogue.  A stage slot holds one
+// k-chunk's activation tile and decoded weight tile; decoders decode into
+// registers from the code ring and only wait for the slot to be free to store,
+// so a slot's round trip is the activation load plus a store.
 // The UMMA issuer (even CTA) learns of its own CTA's readiness through local
-// barriers (bdone, lfull) and of the odd CTA's through bfull / lready, which
-// the odd CTA signals with st.async stores whose mbarrier complete_tx carries
-// the cluster-scope release (a release-arrive would stall the signalling warp
-// for about a microsecond).  bfull / lready expect 16 / 4 bytes per phase and
-// are re-armed by the issuer as soon as it has observed a phase.  The issuer's
-// commits arrive on both CTAs' empty / lempty / accfull barriers.
+// barriers (bdone, xfull, lfull) and of the odd CTA's through bfull / lready,
+// which the odd CTA's relay signals with st.async stores whose mbarrier
+// complete_tx carries the cluster-scope release (a release-arrive would stall
+// the signalling warp for about a microsecond).  bfull / lready expect 4 bytes
+// per phase and are re-armed by the issuer as soon as it has observed a phase.
+// The issuer's commits arrive on both CTAs' empty / lempty / accfull barriers.
 namespace nf4g {
 constexpr int BM = 128;   // activation rows per CTA (256 per pair)
 constexpr int BN = 128;   // weight rows decoded per CTA (256 output columns per pair)
-constexpr int BK = 64, STAGES = 5;
+constexpr int BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;                 // activation tile, K-major SW128
 constexpr int B_BYTES = BN * BK * 2;                 // dequantised weight tile
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
+constexpr int kGroups = 4;          // decode groups; group g decodes the k-chunks j with j % 4 == g
+constexpr int kGroupWarps = 4;      // warps per decode group (one per 32 weight rows)
+constexpr int RAW_STAGES = 2 * kGroups;  // code slot r always belongs to group r % 4 (no phase aliasing)
 constexpr int RAW_BYTES = BN * BK / 2;               // NF4 codes as loaded
 constexpr int AMAX_BYTES = BN * 4;                   // one absmax per decode thread
-constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + RAW_BYTES + AMAX_BYTES + 1023) / 1024) * 1024;
+constexpr int RAW_SLOT = RAW_BYTES + AMAX_BYTES;     // 4608
+constexpr int RAW_OFF = STAGES * STAGE_BYTES;
+constexpr int LA_OFF = RAW_OFF + RAW_STAGES * RAW_SLOT;
 constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;      // p or q rows of this CTA
 constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;      // LoRA weight rows of this CTA
+constexpr int LB_OFF = LA_OFF + LA_BYTES;
+constexpr int BAR_OFF = LB_OFF + LB_BYTES;
 constexpr int BAR_BYTES = 1024;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LA_BYTES + LB_BYTES + BAR_BYTES + 1024;
-constexpr int kThreads = 512;
+constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;
+constexpr int kEpiWarp0 = 4 + kGroups * kGroupWarps;
+constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTmemCols = 512;      // 2 accumulator buffers x 256 columns
-constexpr int kFullCount = 1 + 32;  // the producer's expect_tx arrival + 32 absmax cp.async arrivals
-constexpr int kGroupWarps = 4;      // warps per decode group
-// k-chunk j lands on full barrier (j % STAGES, j % 2): a slot has one barrier per
-// decode group, so each barrier is waited on in order by one group only and a
-// parity wait can never run a phase ahead.  Barrier use count = j / kFullPeriod.
-constexpr int kFullPeriod = (STAGES % 2 == 0) ? STAGES : 2 * STAGES;
-__host__ __device__ constexpr uint32_t full_index(uint32_t j) { return (j % STAGES) * 2 + (j & 1); }
-__host__ __device__ constexpr uint32_t full_parity(uint32_t j) { return (j / kFullPeriod) & 1; }
+constexpr int kRawFullCount = 1 + 32;  // the producer's expect_tx arrival + 32 absmax cp.async arrivals
+static_assert(LA_OFF % 1024 == 0 && LB_OFF % 1024 == 0, "swizzle atom alignment");
+static_assert(RAW_STAGES % kGroups == 0, "code slots are owned by one decode group each");
+// A decode group waits for stage slot j % STAGES after its previous chunk j - kGroups
+// waited for the commit of chunk j - kGroups - STAGES; the barrier cannot be two
+// phases behind as long as STAGES >= kGroups.
+static_assert(STAGES >= kGroups, "stage-slot waits cannot alias");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace nf4g
 
@@ -133,14 +146,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align1024(smem_dyn);
   uint8_t* stages = smem;
-  uint8_t* la = smem + STAGES * STAGE_BYTES;
-  uint8_t* lb = la + LA_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(lb + LB_BYTES);
-  uint64_t* full = bars;                 // [STAGES][2] local TMA tiles + absmax copies landed
-  uint64_t* bfull = bars + 2 * STAGES;   // [STAGES] (even CTA) the odd CTA's decoded tile written
-  uint64_t* empty = bars + 3 * STAGES;   // [STAGES] stage consumed by the UMMAs
-  uint64_t* bdone = bars + 4 * STAGES;   // [STAGES] (even CTA) its own decoded tile written
-  uint64_t* lfull = bars + 5 * STAGES;   // local LoRA operands landed
+  uint8_t* rawbuf = smem + RAW_OFF;
+  uint8_t* la = smem + LA_OFF;
+  uint8_t* lb = smem + LB_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* raw_full = bars;                   // [RAW_STAGES] codes + block scales landed
+  uint64_t* raw_empty = raw_full + RAW_STAGES; // [RAW_STAGES] codes read into registers (group's 4 warps)
+  uint64_t* xfull = raw_empty + RAW_STAGES;    // [STAGES] activation tile landed
+  uint64_t* bfull = xfull + STAGES;            // [STAGES] (even CTA) the odd CTA's stage complete (relay)
+  uint64_t* empty = bfull + STAGES;            // [STAGES] stage consumed by the UMMAs
+  uint64_t* bdone = empty + STAGES;            // [STAGES] this CTA's decoded tile written (group's 4 warps)
+  uint64_t* lfull = bdone + STAGES;            // local LoRA operands landed
   uint64_t* lready = lfull + 1;          // (even CTA) the odd CTA's LoRA operands landed
   uint64_t* lempty = lfull + 2;          // LoRA operands consumed
   uint64_t* accfull = lfull + 3;         // [2] accumulator buffer complete
@@ -153,16 +169,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   if (threadIdx.x == 0) {
+    for (int r = 0; r < RAW_STAGES; ++r) {
+      mbar_init(&raw_full[r], kRawFullCount);
+      mbar_init(&raw_empty[r], kGroupWarps);
+    }
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[2 * s], kFullCount);
-      mbar_init(&full[2 * s + 1], kFullCount);
+      mbar_init(&xfull[s], 1);
       mbar_init(&bfull[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&bdone[s], kGroupWarps);
     }
     mbar_init(lfull, 1);
     mbar_init(lready, 1);
-    for (int s = 0; s < STAGES; ++s) mbar_arrive_expect_tx(&bfull[s], 4 * kGroupWarps);  // arm phase 0
+    for (int s = 0; s < STAGES; ++s) mbar_arrive_expect_tx(&bfull[s], 4);  // arm phase 0
     mbar_arrive_expect_tx(lready, 4);
     mbar_init(lempty, 1);
     for (int b = 0; b < 2; ++b) {
@@ -208,63 +227,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer + absmax copies (whole warp)
-    if (lane == 0) {
-      tma_prefetch_desc(&map_a);
-      tma_prefetch_desc(&map_raw);
-      tma_prefetch_desc(&map_la);
-      tma_prefetch_desc(&map_lb);
-    }
-    uint32_t j = 0, ti = 0, issued = 0, last_par = 0;  // issued/last_par: per full barrier
+    // ------------------------------------------------ NF4 codes + block scales into the code ring (whole warp)
+    if (lane == 0) tma_prefetch_desc(&map_raw);
+    uint32_t j = 0, issued = 0, last_par = 0;  // issued/last_par: per code slot
     bool ok = true;
-    // The next unit's (expert, first row) are loaded one unit ahead, off the critical path.
-    int e_next = 0, r_next = 0;
-    if (pair < n_units) {
-      e_next = units[3 * (pair / p.n_nt)];
-      r_next = units[3 * (pair / p.n_nt) + 1];
-    }
-    for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
+    int e_next = (pair < n_units) ? units[3 * (pair / p.n_nt)] : 0;
+    for (int u = pair; u < n_units && ok; u += n_pairs) {
       const int nt = u % p.n_nt;
-      const int e = e_next, row0 = r_next + (int)rank * 128;
-      if (u + n_pairs < n_units) {
-        e_next = units[3 * ((u + n_pairs) / p.n_nt)];
-        r_next = units[3 * ((u + n_pairs) / p.n_nt) + 1];
-      }
+      const int e = e_next;
+      if (u + n_pairs < n_units) e_next = units[3 * ((u + n_pairs) / p.n_nt)];
       int rA = 0, rB = 0;
       if (!kMN) kmajor_rows(nt, rA, rB);
-      ok = __all_sync(kFull, mbar_wait(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 10));
-      if (!ok) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(lfull, (uint32_t)(512 * p.r_pad));
-        tma_load_2d(la, &map_la, lfull, 0, row0);
-        if (!kMN) {
-          tma_load_3d(lb, &map_lb, lfull, 0, rA, e);
-          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, 0, rB, e);
-        } else {
-          const int c0 = nt * 256 + rank * 128;
-          tma_load_3d(lb, &map_lb, lfull, c0, 0, e);
-          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, c0 + 64, 0, e);
-        }
-      }
       for (int kc = 0; kc < kchunks; ++kc, ++j) {
-        const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
-        ok = __all_sync(kFull, mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 11));
+        const uint32_t r = j % RAW_STAGES, ph = (j / RAW_STAGES) & 1;
+        ok = __all_sync(kFull, mbar_wait_lazy(&raw_empty[r], ph ^ 1, ctl, p.err, p.timeout_ns, 11, 64));
         if (!ok) break;
-        uint8_t* st = stages + s * STAGE_BYTES;
-        const uint32_t fi = full_index(j);
-        uint64_t* fb = &full[fi];
+        uint8_t* slot = rawbuf + r * RAW_SLOT;
         if (lane == 0) {
-          mbar_arrive_expect_tx(fb, (uint32_t)(A_BYTES + RAW_BYTES));
-          tma_load_2d(st, &map_a, fb, kc * BK, row0);
+          mbar_arrive_expect_tx(&raw_full[r], (uint32_t)RAW_BYTES);
           if (!kMN) {
-            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, kc * (BK / 2), rA, e);
-            tma_load_3d(st + A_BYTES + B_BYTES + RAW_BYTES / 2, &map_raw, fb, kc * (BK / 2), rB, e);
+            tma_load_3d(slot, &map_raw, &raw_full[r], kc * (BK / 2), rA, e);
+            tma_load_3d(slot + RAW_BYTES / 2, &map_raw, &raw_full[r], kc * (BK / 2), rB, e);
           } else {
-            tma_load_3d(st + A_BYTES + B_BYTES, &map_raw, fb, (nt * 256 + rank * 128) / 2, kc * BK, e);
+            tma_load_3d(slot, &map_raw, &raw_full[r], (nt * 256 + rank * 128) / 2, kc * BK, e);
           }
         }
         // absmax of the block each decode thread t will decode -> amax[t]
-        float* amax = reinterpret_cast<float*>(st + A_BYTES + B_BYTES + RAW_BYTES);
+        float* amax = reinterpret_cast<float*>(slot + RAW_BYTES);
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           const int t = lane + 32 * qq;
@@ -279,29 +268,92 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           if (row_valid(nt, t))
             cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk);
         }
-        cp_async_arrive_noinc(fb);
-        issued |= 1u << fi;
-        last_par = (last_par & ~(1u << fi)) | (full_parity(j) << fi);
+        cp_async_arrive_noinc(&raw_full[r]);
+        issued |= 1u << r;
+        last_par = (last_par & ~(1u << r)) | (ph << r);
       }
     }
     if (!ok && lane == 0) {
       // Let copies already issued land before the CTA's shared memory goes away.
-      for (int i = 0; i < 2 * STAGES; ++i)
+      for (int i = 0; i < RAW_STAGES; ++i)
         if (issued & (1u << i)) {
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
+          while (!mbar_try_wait(&raw_full[i], (last_par >> i) & 1u) &&
                  (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
           }
         }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------ UMMA issuer (even CTA)
-    if (lane == 0 && rank == 0) {
+  } else if (warp == 3) {
+    // ------------------------------------------------ activation tiles + LoRA operands (one lane)
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_la);
+      tma_prefetch_desc(&map_lb);
+      uint32_t ti = 0, s = 0, ph = 0, issued = 0, last_par = 0;  // issued/last_par: per stage slot
+      bool ok = true;
+      for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
+        const int nt = u % p.n_nt;
+        const int e = units[3 * (u / p.n_nt)], row0 = units[3 * (u / p.n_nt) + 1] + (int)rank * 128;
+        int rA = 0, rB = 0;
+        if (!kMN) kmajor_rows(nt, rA, rB);
+        if (!(ok = mbar_wait_lazy(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 10, 64))) break;
+        mbar_arrive_expect_tx(lfull, (uint32_t)(512 * p.r_pad));
+        tma_load_2d(la, &map_la, lfull, 0, row0);
+        if (!kMN) {
+          tma_load_3d(lb, &map_lb, lfull, 0, rA, e);
+          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, 0, rB, e);
+        } else {
+          const int c0 = nt * 256 + rank * 128;
+          tma_load_3d(lb, &map_lb, lfull, c0, 0, e);
+          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, c0 + 64, 0, e);
+        }
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 12))) break;
+          mbar_arrive_expect_tx(&xfull[s], (uint32_t)A_BYTES);
+          tma_load_2d(stages + s * STAGE_BYTES, &map_a, &xfull[s], kc * BK, row0);
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < STAGES; ++i)
+          if (issued & (1u << i)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&xfull[i], (last_par >> i) & 1u) &&
+                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1 && rank == 0) {
+    // ------------------------------------------------ UMMA issuer (even CTA, one elected lane)
+    // A 256x256x16 pair UMMA keeps the tensor pipe busy for about as long as
+    // the issuing thread is blocked handing in the next one, so any gap between
+    // the last UMMA of a k-chunk and the first of the next leaves the pipe
+    // idle.  The readiness of the next k-chunk is therefore tested (without
+    // blocking) while the current chunk's UMMAs are being handed in; only if it
+    // is not ready yet does the thread fall back to a bounded wait.
+    if (elect_one_sync()) {
       const uint32_t idesc = make_idesc_bf16(256, 256, false, kMN);
       const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
       const uint32_t la_u = smem_u32(la), lb_u = smem_u32(lb);
-      uint32_t j = 0, ti = 0;
+      const uint32_t st_u = smem_u32(stages);
+      const uint32_t bstep = kMN ? 128u : 2u;  // K16 step of B in the descriptor address field
+      uint32_t ti = 0, s = 0, ph = 0;          // unit counter; k-chunk stage slot and parity
       bool ok = true;
+      // Both CTAs' halves of the k-chunk in slot s (activation tile and decoded
+      // weight tile) are in place; arms bfull[s] for its next use.
+      auto wait_chunk = [&](uint32_t ss, uint32_t pp) -> bool {
+        if (!mbar_wait(&bdone[ss], pp, ctl, p.err, p.timeout_ns, 24)) return false;
+        if (!mbar_wait(&xfull[ss], pp, ctl, p.err, p.timeout_ns, 25)) return false;
+        if (!mbar_wait_cluster(&bfull[ss], pp, ctl, p.err, p.timeout_ns, 23)) return false;
+        mbar_arrive_expect_tx(&bfull[ss], 4);
+        return true;
+      };
       for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
         const uint32_t b = ti & 1, use = ti >> 1;
         const uint32_t d = tmem + b * 256;
@@ -318,21 +370,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           umma_bf16_2sm(d, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
         }
         umma_commit_2sm(lempty, 0x3);
-        for (int kc = 0; kc < kchunks; ++kc, ++j) {
-          const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
-          if (!(ok = mbar_wait(&bdone[s], ph, ctl, p.err, p.timeout_ns, 24))) break;
-          if (!(ok = mbar_wait_cluster(&bfull[s], ph, ctl, p.err, p.timeout_ns, 23))) break;
-          mbar_arrive_expect_tx(&bfull[s], 4 * kGroupWarps);  // arm the next phase
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(stages + s * STAGE_BYTES);
-          const uint32_t b0 = a0 + A_BYTES;
+        if (!(ok = wait_chunk(s, ph))) break;
+        tc_fence_after();
+        for (int kc = 0; kc < kchunks; ++kc) {
+          const uint32_t a0 = st_u + s * STAGE_BYTES;
+          const uint64_t adesc = make_sdesc(a0, 16, 1024, kSw128);
+          const uint64_t bdesc = kMN ? make_sdesc(a0 + A_BYTES, 8192, 1024, kSw128)
+                                     : make_sdesc(a0 + A_BYTES, 16, 1024, kSw128);
+          const uint32_t s1 = (s + 1 == STAGES) ? 0 : s + 1, ph1 = (s + 1 == STAGES) ? ph ^ 1 : ph;
+          const bool more = kc + 1 < kchunks;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bd =
-                kMN ? make_sdesc(b0 + 2048 * kk, 8192, 1024, kSw128) : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
-            umma_bf16_2sm(d, make_sdesc(a0 + 32 * kk, 16, 1024, kSw128), bd, idesc, 1u);
-          }
+          for (int kk = 0; kk < BK / 16 - 1; ++kk)  // K16 step: +32 bytes of A; +32 (K-major) / +2048 bytes of B
+            umma_bf16_2sm(d, adesc + 2 * kk, bdesc + bstep * kk, idesc, 1u);
+          // Peek at the next k-chunk while the UMMAs above execute.
+          const bool next_ready = more && mbar_test_wait(&bdone[s1], ph1) && mbar_test_wait(&xfull[s1], ph1) &&
+                                  mbar_test_wait_cluster(&bfull[s1], ph1);
+          umma_bf16_2sm(d, adesc + 2 * (BK / 16 - 1), bdesc + bstep * (BK / 16 - 1), idesc, 1u);
           umma_commit_2sm(&empty[s], 0x3);
+          s = s1;
+          ph = ph1;
+          if (more) {
+            if (next_ready)
+              mbar_arrive_expect_tx(&bfull[s], 4);
+            else if (!(ok = wait_chunk(s, ph)))
+              break;
+            tc_fence_after();
+          }
         }
         if (!ok) break;
         umma_commit_2sm(&accfull[b], 0x3);
@@ -342,59 +405,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
       }
     }
+    __syncwarp();
   } else if (warp == 2 && rank == 1) {
-    // ------------------------------------------------ relay (odd CTA): LoRA operands landed -> even CTA
+    // ------------------------------------------------ relay (odd CTA): its LoRA operands and each k-chunk's
+    // activation + decoded tiles are in place -> even CTA (one 4-byte st.async per event)
     const uint32_t lready_even = mapa_shared(smem_u32(lready), 0);
-    const uint32_t sig_even = mapa_shared(smem_u32(sig), 0);
-    uint32_t ti = 0;
-    for (int u = pair; u < n_units; u += n_pairs, ++ti) {
-      if (!__all_sync(kFull, mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 50))) break;
-      if (lane == 0) st_async_signal(sig_even, lready_even, 1u);
-    }
-  } else if (warp >= 4 && warp < 12) {
-    // ------------------------------------------------ NF4 decode, two groups on alternate k-chunks
-    const uint32_t grp = (warp - 4) >> 2;
-    const int t = (threadIdx.x - 128) & 127;
     const uint32_t bfull_even = mapa_shared(smem_u32(bfull), 0);
     const uint32_t sig_even = mapa_shared(smem_u32(sig), 0);
-    uint32_t j = 0;
+    uint32_t ti = 0, s = 0, ph = 0;
     bool ok = true;
-    for (int u = pair; u < n_units && ok; u += n_pairs) {
-      const int nt = u % p.n_nt;
-      const bool valid = row_valid(nt, t);
-      for (int kc = 0; kc < kchunks; ++kc, ++j) {
-        if ((j & 1) != grp) continue;
-        const uint32_t s = j % STAGES;
-        ok = __all_sync(kFull, mbar_wait(&full[full_index(j)], full_parity(j), ctl, p.err, p.timeout_ns, 30));
+    for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
+      if (!(ok = __all_sync(kFull, mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 50)))) break;
+      if (lane == 0) st_async_signal(sig_even, lready_even, 1u);
+      for (int kc = 0; kc < kchunks; ++kc) {
+        ok = __all_sync(kFull, mbar_wait(&bdone[s], ph, ctl, p.err, p.timeout_ns, 51));
+        if (ok) ok = __all_sync(kFull, mbar_wait(&xfull[s], ph, ctl, p.err, p.timeout_ns, 52));
         if (!ok) break;
-        uint8_t* st = stages + s * STAGE_BYTES;
-        const uint8_t* raw = st + A_BYTES + B_BYTES + (kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32);
-        uint32_t v[32];
-        if (valid) {
-          const float amax = reinterpret_cast<const float*>(st + A_BYTES + B_BYTES + RAW_BYTES)[t];
-          const uint4 q0 = *reinterpret_cast<const uint4*>(raw);
-          const uint4 q1 = *reinterpret_cast<const uint4*>(raw + 16);
-          const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-          nf4_decode_block(codes, amax, v);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
-        }
-        if (!kMN)
-          st_swizzled_row128(st + A_BYTES, t, v);
-        else
-          st_swizzled_row128(st + A_BYTES + (t >> 6) * 8192, t & 63, v);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (rank == 0)
-            mbar_arrive(&bdone[s]);
-          else
-            st_async_signal(sig_even, bfull_even + 8 * s, 1u);
+        if (lane == 0) st_async_signal(sig_even, bfull_even + 8 * s, 1u);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
         }
       }
     }
-  } else if (warp >= 12) {
+  } else if (warp >= 4 && warp < kEpiWarp0) {
+    // ------------------------------------------------ NF4 decode, groups take the k-chunks round robin
+    // Group g decodes chunk j (j % 4 == g) from code slot j % RAW_STAGES into
+    // registers, then waits for stage slot j % STAGES to be free and stores the tile.
+    const uint32_t grp = (warp - 4) >> 2;
+    const int t = (threadIdx.x - 128) & 127;
+    const Nf4Shift ks = nf4_shift_consts();
+    const int raw_off = kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32;
+    // Row `drow` of the decoded 128B-swizzled tile: 16-byte chunk c at c ^ (drow % 8).
+    const int drow = kMN ? (t & 63) : t;
+    const uint32_t drow_off = (kMN ? (t >> 6) * 8192 : 0) + (drow >> 3) * 1024 + (drow & 7) * 128;
+    const uint32_t b_u = smem_u32(stages) + A_BYTES;
+    uint32_t j = 0;  // chunk counter at the unit's start
+    bool ok = true;
+    for (int u = pair; u < n_units && ok; u += n_pairs, j += kchunks) {
+      const int nt = u % p.n_nt;
+      const bool valid = row_valid(nt, t);
+      for (int kc = (int)((grp + kGroups - j % kGroups) % kGroups); kc < kchunks; kc += kGroups) {
+        const uint32_t jj = j + kc;
+        const uint32_t r = jj % RAW_STAGES, rph = (jj / RAW_STAGES) & 1;
+        ok = __all_sync(kFull, mbar_wait(&raw_full[r], rph, ctl, p.err, p.timeout_ns, 30));
+        if (!ok) break;
+        const uint8_t* slot = rawbuf + r * RAW_SLOT;
+        const float amax = reinterpret_cast<const float*>(slot + RAW_BYTES)[t];
+        const uint4 q0 = *reinterpret_cast<const uint4*>(slot + raw_off);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(slot + raw_off + 16);
+        const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        // Rows past the end of the matrix decode with a zero scale: all zeros.
+        const Nf4Planes pl = nf4_block_planes(valid ? amax : 0.0f);
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) nf4_decode_word(codes[c], pl, ks, &v[4 * c]);
+        const uint32_t s = jj % STAGES, sph = (jj / STAGES) & 1;
+        ok = __all_sync(kFull, mbar_wait(&empty[s], sph ^ 1, ctl, p.err, p.timeout_ns, 31));
+        if (!ok) break;
+        const uint32_t dbase = b_u + s * STAGE_BYTES + drow_off;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(dbase + ((c ^ (drow & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        // One proxy fence orders both this thread's reads of the code slot
+        // before the next TMA write into it (generic reads, then an async-proxy
+        // write: released through raw_empty) and its tile stores before the
+        // UMMA reads them.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bdone[s]);
+          mbar_arrive(&raw_empty[r]);
+        }
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ epilogue
     const int qrt = warp & 3;  // TMEM lane quarter of this warp
     const uint32_t accempty_even = mapa_shared(smem_u32(accempty), 0);

@@ -346,8 +346,11 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
           const uint4 q1 = *reinterpret_cast<const uint4*>(crow + (((2 * c + 1) ^ (t & 7)) << 4));
           const float a = amax[c];
           if (c == nb - 1) {
+            // The stage's codes are in registers.  A proxy fence orders these
+            // generic reads before the next TMA write into the slot.
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&raw_empty[r]);  // the stage's codes are in registers
+            if (lane == 0) mbar_arrive(&raw_empty[r]);
           }
           const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
           // Rows past the end of the matrix get a zero scale, so every entry
