@@ -49,17 +49,6 @@ __device__ __forceinline__ void store16(uint16_t* dst, const uint32_t (&w)[8], b
     store_bf16x16(dst, w);
 }
 
-__device__ __forceinline__ void load_bf16x16(const uint16_t* src, float (&v)[16]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-  const uint4 a = __ldg(s), b = __ldg(s + 1);
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = bf16lo_to_f32(w[i]);
-    v[2 * i + 1] = bf16hi_to_f32(w[i]);
-  }
-}
-
 
 }  // namespace
 
@@ -517,33 +506,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           store16(p.out1 + row * p.I + c0 + jj, aw, p.v8);
         }
       } else if (MODE == kDgradDown) {
+        // SwiGLU backward in 8-column steps; the forward gate/up values of the
+        // next step are loaded while this step's are used (loads from 128
+        // different rows per warp: their latency must overlap the work).
         const int I2 = 2 * p.I, c0 = nt * 256;
+        const int ncol = min(256, p.I - c0);  // a multiple of 64
+        const uint16_t* grow = p.aux + row * I2 + c0;
+        uint4 gq = make_uint4(0, 0, 0, 0), uq = make_uint4(0, 0, 0, 0);
+        if (store) {
+          gq = __ldg(reinterpret_cast<const uint4*>(grow));
+          uq = __ldg(reinterpret_cast<const uint4*>(grow + p.I));
+        }
 #pragma unroll 1
-        for (int jj = 0; jj < 256; jj += 16) {
-          if (c0 + jj >= p.I) break;
-          float da[16], g[16], up[16];
+        for (int jj = 0; jj < ncol; jj += 8) {
+          uint4 gn = make_uint4(0, 0, 0, 0), un = make_uint4(0, 0, 0, 0);
+          if (store && jj + 8 < ncol) {
+            gn = __ldg(reinterpret_cast<const uint4*>(grow + jj + 8));
+            un = __ldg(reinterpret_cast<const uint4*>(grow + p.I + jj + 8));
+          }
+          float da[8];
+          tmem_ld8(tl + jj, da);
           if (store) {
-            load_bf16x16(p.aux + row * I2 + c0 + jj, g);
-            load_bf16x16(p.aux + row * I2 + p.I + c0 + jj, up);
-          }
-          tmem_ld16(tl + jj, da);
-          if (!store) continue;
-          uint32_t dgw[8], duw[8];
+            const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w}, uw[4] = {uq.x, uq.y, uq.z, uq.w};
+            uint32_t dgw[4], duw[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float dg[2], du[2];
+            for (int i = 0; i < 4; ++i) {
+              float dg[2], du[2];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const float gg = g[2 * i + hh], uu = up[2 * i + hh], dd = da[2 * i + hh];
-              const float sg = sigmoid_f(gg);
-              dg[hh] = dd * uu * sg * (1.0f + gg * (1.0f - sg));
-              du[hh] = dd * gg * sg;
+              for (int hh = 0; hh < 2; ++hh) {
+                const float gg = hh ? bf16hi_to_f32(gw[i]) : bf16lo_to_f32(gw[i]);
+                const float uu = hh ? bf16hi_to_f32(uw[i]) : bf16lo_to_f32(uw[i]);
+                const float dd = da[2 * i + hh];
+                const float sg = sigmoid_f(gg);
+                dg[hh] = dd * uu * sg * (1.0f + gg * (1.0f - sg));
+                du[hh] = dd * gg * sg;
+              }
+              dgw[i] = pack_bf16x2(dg[0], dg[1]);
+              duw[i] = pack_bf16x2(du[0], du[1]);
             }
-            dgw[i] = pack_bf16x2(dg[0], dg[1]);
-            duw[i] = pack_bf16x2(du[0], du[1]);
+            *reinterpret_cast<uint4*>(p.out0 + row * I2 + c0 + jj) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+            *reinterpret_cast<uint4*>(p.out0 + row * I2 + p.I + c0 + jj) =
+                make_uint4(duw[0], duw[1], duw[2], duw[3]);
           }
-          store16(p.out0 + row * I2 + c0 + jj, dgw, p.v8);
-          store16(p.out0 + row * I2 + p.I + c0 + jj, duw, p.v8);
+          gq = gn;
+          uq = un;
         }
       } else {
         const int c0 = nt * 256;
