@@ -506,31 +506,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           store16(p.out1 + row * p.I + c0 + jj, aw, p.v8);
         }
       } else if (MODE == kDgradDown) {
-        // SwiGLU backward in 8-column steps; the forward gate/up values of the
-        // next step are loaded while this step's are used (loads from 128
-        // different rows per warp: their latency must overlap the work).
+        // SwiGLU backward; the forward gate/up values of the next step are
+        // loaded while this step's are used.
         const int I2 = 2 * p.I, c0 = nt * 256;
         const int ncol = min(256, p.I - c0);  // a multiple of 64
         const uint16_t* grow = p.aux + row * I2 + c0;
-        uint4 gq = make_uint4(0, 0, 0, 0), uq = make_uint4(0, 0, 0, 0);
         if (store) {
-          gq = __ldg(reinterpret_cast<const uint4*>(grow));
-          uq = __ldg(reinterpret_cast<const uint4*>(grow + p.I));
+          // The unit's gate/up values of this row (2 x ncol bf16, from HBM: the
+          // buffer is larger than L2) are pulled into L2 up front, so the step
+          // loads below wait for L2, not for DRAM.
+          for (int off = 0; off < ncol; off += 64) {
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(grow + off));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(grow + p.I + off));
+          }
+        }
+        // 16-column steps: every load and store covers whole 32-byte sectors.
+        uint4 gq[2], uq[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          gq[h] = store ? __ldg(reinterpret_cast<const uint4*>(grow) + h) : make_uint4(0, 0, 0, 0);
+          uq[h] = store ? __ldg(reinterpret_cast<const uint4*>(grow + p.I) + h) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll 1
-        for (int jj = 0; jj < ncol; jj += 8) {
-          uint4 gn = make_uint4(0, 0, 0, 0), un = make_uint4(0, 0, 0, 0);
-          if (store && jj + 8 < ncol) {
-            gn = __ldg(reinterpret_cast<const uint4*>(grow + jj + 8));
-            un = __ldg(reinterpret_cast<const uint4*>(grow + p.I + jj + 8));
-          }
-          float da[8];
-          tmem_ld8(tl + jj, da);
-          if (store) {
-            const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w}, uw[4] = {uq.x, uq.y, uq.z, uq.w};
-            uint32_t dgw[4], duw[4];
+        for (int jj = 0; jj < ncol; jj += 16) {
+          uint4 gn[2], un[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+          for (int h = 0; h < 2; ++h) {
+            const bool more = store && jj + 16 < ncol;
+            gn[h] = more ? __ldg(reinterpret_cast<const uint4*>(grow + jj + 16) + h) : make_uint4(0, 0, 0, 0);
+            un[h] = more ? __ldg(reinterpret_cast<const uint4*>(grow + p.I + jj + 16) + h) : make_uint4(0, 0, 0, 0);
+          }
+          float da[16];
+          tmem_ld16(tl + jj, da);
+          if (store) {
+            const uint32_t gw[8] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w};
+            const uint32_t uw[8] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w};
+            uint32_t dgw[8], duw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
               float dg[2], du[2];
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
@@ -544,12 +557,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
               dgw[i] = pack_bf16x2(dg[0], dg[1]);
               duw[i] = pack_bf16x2(du[0], du[1]);
             }
-            *reinterpret_cast<uint4*>(p.out0 + row * I2 + c0 + jj) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-            *reinterpret_cast<uint4*>(p.out0 + row * I2 + p.I + c0 + jj) =
-                make_uint4(duw[0], duw[1], duw[2], duw[3]);
+            store16(p.out0 + row * I2 + c0 + jj, dgw, p.v8);
+            store16(p.out0 + row * I2 + p.I + c0 + jj, duw, p.v8);
           }
-          gq = gn;
-          uq = un;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            gq[h] = gn[h];
+            uq[h] = un[h];
+          }
         }
       } else {
         const int c0 = nt * 256;
