@@ -29,26 +29,19 @@ namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
 
-__device__ __forceinline__ void store_bf16x16(uint16_t* dst, const uint32_t (&w)[8]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+// 16 bf16 (32 bytes) from registers to global memory: one full-sector store
+// when the destination is 32-byte aligned, else two 16-byte stores.
+__device__ __forceinline__ void store_row16(uint16_t* dst, const uint32_t (&w)[8], bool v8) {
+  if (v8) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
 }
-
-// One full 32-byte sector per thread (dst must be 32-byte aligned).
-__device__ __forceinline__ void store_bf16x16_v8(uint16_t* dst, const uint32_t (&w)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
-               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-               : "memory");
-}
-
-__device__ __forceinline__ void store16(uint16_t* dst, const uint32_t (&w)[8], bool v8) {
-  if (v8)
-    store_bf16x16_v8(dst, w);
-  else
-    store_bf16x16(dst, w);
-}
-
 
 }  // namespace
 
@@ -94,7 +87,12 @@ constexpr int LA_OFF = RAW_OFF + RAW_STAGES * RAW_SLOT;
 constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;      // p or q rows of this CTA
 constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;      // LoRA weight rows of this CTA
 constexpr int LB_OFF = LA_OFF + LA_BYTES;
-constexpr int BAR_OFF = LB_OFF + LB_BYTES;
+// Epilogue staging: per epilogue warp, two steps x up to three 32-row x 16-column output tiles.
+constexpr int kEpiTileBytes = 32 * 16 * 2;
+constexpr int kEpiStepBytes = 3 * kEpiTileBytes;
+constexpr int kEpiWarpBytes = 2 * kEpiStepBytes;
+constexpr int EPI_OFF = LB_OFF + LB_BYTES;
+constexpr int BAR_OFF = EPI_OFF + 4 * kEpiWarpBytes;
 constexpr int BAR_BYTES = 1024;
 constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;
 constexpr int kEpiWarp0 = 4 + kGroups * kGroupWarps;
@@ -121,7 +119,7 @@ struct Nf4GemmParams {
   int K, n_dim, I, r_pad;
   int stored_rows, stored_cols;
   int n_nt;
-  int v8;             // output buffers and row pitches are 32-byte aligned: 32-byte stores
+  int v8;             // (down dgrad) dgu and its row pitch are 32-byte aligned: 32-byte stores
   int64_t mu_offset;  // start of the m-unit list in `tiles`
 };
 
@@ -129,6 +127,7 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     nf4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_raw,
                     const __grid_constant__ CUtensorMap map_la, const __grid_constant__ CUtensorMap map_lb,
+                    const __grid_constant__ CUtensorMap map_o0, const __grid_constant__ CUtensorMap map_o1,
                     const Nf4GemmParams p) {
   using namespace nf4g;
   constexpr bool kMN = (MODE == kDgradDown || MODE == kDgradGateUp);  // B operand N-contiguous
@@ -470,15 +469,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ epilogue
+    // Output tiles of a 16-column step (32 rows x 16 columns, 1 KB each) are
+    // staged in this warp's shared memory and written by TMA bulk stores:
+    // per-row global stores (32 rows per warp instruction) congest the L1
+    // path that the UMMAs read their operands through (measured: the k-chunks
+    // running beside an epilogue took twice as long).  The down dgrad keeps
+    // direct stores (see there).
     const int qrt = warp & 3;  // TMEM lane quarter of this warp
     const uint32_t accempty_even = mapa_shared(smem_u32(accempty), 0);
-    uint32_t ti = 0;
+    const uint32_t ebuf = smem_u32(smem + EPI_OFF + qrt * kEpiWarpBytes);
+    if (lane == 0) {
+      tma_prefetch_desc(&map_o0);
+      tma_prefetch_desc(&map_o1);
+    }
+    uint32_t ti = 0, step = 0;
     bool ok = true;
+    // Staging buffer of this step, free once the stores of the step two back have read it.
+    auto step_buffer = [&]() -> uint32_t {
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      return ebuf + (step & 1) * kEpiStepBytes;
+    };
+    auto stage = [&](uint32_t buf, int tile, const uint32_t (&w)[8]) {
+      const uint32_t a = buf + tile * kEpiTileBytes + lane * 32;
+      st_shared_v4(a, w[0], w[1], w[2], w[3]);
+      st_shared_v4(a + 16, w[4], w[5], w[6], w[7]);
+    };
+    auto publish = [&]() {  // the staged tiles are visible to the TMA (async proxy)
+      fence_proxy_async_smem();
+      __syncwarp();
+    };
     for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
       const int mu = u / p.n_nt, nt = u % p.n_nt;
       const int nrows = units[3 * mu + 2];
       const bool store = (int)rank * 128 < nrows;
-      const size_t row = (size_t)units[3 * mu + 1] + rank * 128 + qrt * 32 + lane;
+      const int wrow0 = units[3 * mu + 1] + (int)rank * 128 + qrt * 32;  // this warp's first row
+      const size_t row = (size_t)wrow0 + lane;
       const uint32_t b = ti & 1, use = ti >> 1;
       ok = __all_sync(kFull, mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 40));
       if (!ok) break;
@@ -486,7 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       const uint32_t tl = tmem + b * 256 + ((uint32_t)(qrt * 32) << 16);
       if (MODE == kFwdGateUp) {
         // columns [0,128): gate, [128,256): up, of gate/up columns nt*128 ..
-        const int I2 = 2 * p.I, c0 = nt * 128;
+        const int c0 = nt * 128;
 #pragma unroll 1
         for (int jj = 0; jj < 128; jj += 16) {
           if (c0 + jj >= p.I) break;
@@ -501,9 +527,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
             uw[i] = pack_bf16x2(up[2 * i], up[2 * i + 1]);
             aw[i] = pack_bf16x2(silu_f(g[2 * i]) * up[2 * i], silu_f(g[2 * i + 1]) * up[2 * i + 1]);
           }
-          store16(p.out0 + row * I2 + c0 + jj, gw, p.v8);
-          store16(p.out0 + row * I2 + p.I + c0 + jj, uw, p.v8);
-          store16(p.out1 + row * p.I + c0 + jj, aw, p.v8);
+          const uint32_t buf = step_buffer();
+          stage(buf, 0, gw);
+          stage(buf, 1, uw);
+          stage(buf, 2, aw);
+          publish();
+          if (lane == 0) {
+            tma_store_2d(&map_o0, buf, c0 + jj, wrow0);
+            tma_store_2d(&map_o0, buf + kEpiTileBytes, p.I + c0 + jj, wrow0);
+            tma_store_2d(&map_o1, buf + 2 * kEpiTileBytes, c0 + jj, wrow0);
+            bulk_commit();
+          }
+          ++step;
         }
       } else if (MODE == kDgradDown) {
         // SwiGLU backward; the forward gate/up values of the next step are
@@ -557,8 +592,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
               dgw[i] = pack_bf16x2(dg[0], dg[1]);
               duw[i] = pack_bf16x2(du[0], du[1]);
             }
-            store16(p.out0 + row * I2 + c0 + jj, dgw, p.v8);
-            store16(p.out0 + row * I2 + p.I + c0 + jj, duw, p.v8);
+            // Direct full-sector stores here: this epilogue is as long as the
+            // unit's UMMAs, and the staging hand-off would lengthen it.
+            store_row16(p.out0 + row * I2 + c0 + jj, dgw, p.v8);
+            store_row16(p.out0 + row * I2 + p.I + c0 + jj, duw, p.v8);
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -577,7 +614,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           uint32_t w[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          store16(p.out0 + row * p.n_dim + c0 + jj, w, p.v8);
+          const uint32_t buf = step_buffer();
+          stage(buf, 0, w);
+          publish();
+          if (lane == 0) {
+            tma_store_2d(&map_o0, buf, c0 + jj, wrow0);
+            bulk_commit();
+          }
+          ++step;
         }
       }
       // The issuer needs only this warp's TMEM reads to be complete (tcgen05.ld
@@ -592,6 +636,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           mbar_arrive_cluster_relaxed(accempty_even + 8 * b);
       }
     }
+    // Every bulk store of this warp has written global memory (and stopped
+    // reading its staging buffer) before the CTA goes away.
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
   }
 
   __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the cluster barrier
@@ -1034,10 +1082,20 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stream) {
   const bool mn = (h.mode == kDgradDown || h.mode == kDgradGateUp);
-  CUtensorMap ma, mraw, mla, mlb;
+  CUtensorMap ma, mraw, mla, mlb, mo0, mo1;
   cudaError_t err;
   if ((err = map_bf16_2d(&ma, h.act_in, h.K, h.rows_cap, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
     return err;
+  // Epilogue outputs, written as 32-row x 16-column tiles: out0 [rows, n_dim] (gate_up forward: [rows, 2I]
+  // with n_dim = 2I; down dgrad: dgu [rows, 2I] with n_dim = I), out1 [rows, I] (gate_up forward: act).
+  const int64_t out0_cols = (h.mode == kDgradDown) ? 2 * (int64_t)h.I : h.n_dim;
+  if ((err = map_bf16_2d(&mo0, h.out0, out0_cols, h.rows_cap, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
+    return err;
+  if (h.out1 != nullptr)
+    err = map_bf16_2d(&mo1, h.out1, h.I, h.rows_cap, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    mo1 = mo0;
+  if (err != cudaSuccess) return err;
   if (!mn)
     err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 32, 64);
   else
@@ -1066,11 +1124,7 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
   p.stored_rows = h.stored_rows;
   p.stored_cols = h.stored_cols;
   p.n_nt = (h.mode == kFwdGateUp) ? (h.I + 127) / 128 : (h.n_dim + 255) / 256;
-  {
-    auto a32 = [](const void* q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
-    // row pitches in bytes: out0 is [rows, n_dim] (2I for the gate_up forward and the down dgrad), out1 [rows, I]
-    p.v8 = a32(h.out0) && a32(h.out1) && (h.n_dim * 2) % 32 == 0 && (h.I * 2) % 32 == 0 ? 1 : 0;
-  }
+  p.v8 = ((reinterpret_cast<uintptr_t>(h.out0) & 31u) == 0 && (h.I * 4) % 32 == 0) ? 1 : 0;
   p.mu_offset = munits_offset(h.mt_cap, h.E);
   const int64_t units_max = h.mt_cap * p.n_nt;
   const int64_t pairs = units_max < num_sms / 2 ? units_max : num_sms / 2;
@@ -1082,19 +1136,19 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
   switch (h.mode) {
     case kFwdGateUp:
       if ((err = set_smem(nf4_gemm_kernel<kFwdGateUp>, smem)) != cudaSuccess) return err;
-      nf4_gemm_kernel<kFwdGateUp><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      nf4_gemm_kernel<kFwdGateUp><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, mo0, mo1, p);
       break;
     case kFwdDown:
       if ((err = set_smem(nf4_gemm_kernel<kFwdDown>, smem)) != cudaSuccess) return err;
-      nf4_gemm_kernel<kFwdDown><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      nf4_gemm_kernel<kFwdDown><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, mo0, mo1, p);
       break;
     case kDgradDown:
       if ((err = set_smem(nf4_gemm_kernel<kDgradDown>, smem)) != cudaSuccess) return err;
-      nf4_gemm_kernel<kDgradDown><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      nf4_gemm_kernel<kDgradDown><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, mo0, mo1, p);
       break;
     default:
       if ((err = set_smem(nf4_gemm_kernel<kDgradGateUp>, smem)) != cudaSuccess) return err;
-      nf4_gemm_kernel<kDgradGateUp><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, p);
+      nf4_gemm_kernel<kDgradGateUp><<<grid, nf4g::kThreads, smem, stream>>>(ma, mraw, mla, mlb, mo0, mo1, p);
       break;
   }
   return cudaGetLastError();
