@@ -45,5 +45,6 @@ from .moe import (  # noqa: F401
     group_by_expert,
     moe_forward,
     moe_backward,
+    router_backward,
     expert_weights,
 )

@@ -281,3 +281,38 @@ def moe_backward(x, logits, dY, experts: Experts, k: int, alpha: float,
     out.update(grads)
     out.update(per_slot)
     return out
+
+
+def router_backward(x, logits, dY, experts: Experts, k: int, alpha: float,
+                    tokens: Optional[Iterable[int]] = None):
+    """Gradient of the loss with respect to the router logits, for a trained router.
+
+    The router is frozen by default; with it trained ("How do I QLoRA-train
+    the fused experts of a MoE", section "The abstraction that fails, and what
+    replaces it": ``TRAIN_ROUTER=1``), the logits receive a gradient through
+    the routing weights only -- the top-k selection is piecewise constant.
+    With ``yd[t, j]`` the output of the j-th selected expert for token t
+    (before weighting) and upstream ``dY``:
+
+    * ``dw[t, j] = <dY[t], yd[t, j]>`` (since ``y[t] = sum_j w[t, j] yd[t, j]``);
+    * softmax over the k selected logits:
+      ``dlogits[t, ids[t, j]] = w[t, j] * (dw[t, j] - sum_i w[t, i] dw[t, i])``;
+    * every unselected expert's logit gets exactly 0.
+
+    Returns ``d_logits`` [T, E] float64 (rows of unselected tokens zero) and
+    ``dw`` [T, k].
+    """
+    fwd = moe_forward(x, logits, experts, k, alpha, tokens=tokens)
+    ids, w = fwd["ids"], fwd["w"]
+    dY = np.asarray(dY, dtype=np.float64)
+    T = dY.shape[0]
+    E = np.asarray(logits).shape[1]
+    rows = range(T) if tokens is None else sorted(set(int(t) for t in tokens))
+    d_logits = np.zeros((T, E), dtype=np.float64)
+    dw = np.zeros((T, k), dtype=np.float64)
+    for t in rows:
+        for j in range(k):
+            dw[t, j] = float(np.dot(dY[t], fwd["yd"][t * k + j]))
+        d_logits[t, ids[t]] = w[t] * (dw[t] - float(np.dot(w[t], dw[t])))
+    return {"d_logits": d_logits, "dw": dw, "ids": ids, "w": w}
+

@@ -232,3 +232,58 @@ def test_backward_subsets_match_full(tiny):
     np.testing.assert_allclose(sub["dx"][[1, 2]], full["dx"][[1, 2]], rtol=1e-12, atol=1e-15)
     for key in ("dA_gu", "dB_gu", "dA_d", "dB_d"):
         np.testing.assert_allclose(sub[key][2], full[key][2], rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------- router backward
+
+def test_router_backward_finite_differences(tiny):
+    # d/d(logits) of L = sum_t <dY_t, y_t> against central differences of the
+    # forward: the selected logits move the softmax weights; an unselected
+    # logit moved by less than its distance to the k-th selected one changes nothing.
+    prob, ex, x = tiny
+    cfg = prob.cfg
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    rb = oracle.router_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha)
+    lg = np.asarray(prob.logits, dtype=np.float32)
+    srt = np.sort(lg, axis=1)[:, ::-1]
+    gap = srt[:, cfg.top_k - 1] - srt[:, cfg.top_k]
+    eps = np.float32(2.0 ** -10)
+    checked = 0
+    for t in np.flatnonzero(gap > 64 * eps)[:6]:
+        for e in range(cfg.E):
+            lp, lm = lg.copy(), lg.copy()
+            lp[t, e] = lg[t, e] + eps
+            lm[t, e] = lg[t, e] - eps
+            h = float(lp[t, e]) - float(lm[t, e])  # the representable float32 step
+            fd = (_loss(x, lp, dY, ex, cfg.top_k, cfg.alpha) - _loss(x, lm, dY, ex, cfg.top_k, cfg.alpha)) / h
+            an = rb["d_logits"][t, e]
+            assert abs(fd - an) <= 1e-4 * max(1.0, np.abs(rb["d_logits"][t]).max()), (t, e, fd, an)
+            checked += 1
+    assert checked >= 4 * cfg.E
+    assert np.abs(rb["d_logits"]).max() > 1e-3
+
+
+def test_router_backward_invariants(tiny):
+    prob, ex, x = tiny
+    cfg = prob.cfg
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    rb = oracle.router_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha)
+    dl, ids = rb["d_logits"], rb["ids"]
+    # softmax shift invariance: the selected entries of a row sum to zero
+    assert np.allclose(dl.sum(axis=1), 0.0, atol=1e-12 * max(1.0, np.abs(dl).max()))
+    # unselected experts get exact zeros
+    mask = np.zeros_like(dl, dtype=bool)
+    np.put_along_axis(mask, ids.astype(np.int64), True, axis=1)
+    assert np.all(dl[~mask] == 0.0)
+    # dw is the plain dot product of dY with each selected expert's output
+    fwd = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha)
+    t, j = 3, 1
+    assert rb["dw"][t, j] == float(np.dot(dY[t], fwd["yd"][t * cfg.top_k + j]))
+    # one expert per token: the routing weight is constant 1, no gradient
+    rb1 = oracle.router_backward(x, prob.logits, dY, ex, 1, cfg.alpha)
+    assert np.all(rb1["d_logits"] == 0.0)
+    # token subsets agree with the full computation
+    sub = oracle.router_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=[0, 7, 19])
+    assert np.allclose(sub["d_logits"][[0, 7, 19]], dl[[0, 7, 19]], rtol=1e-12, atol=0)  # BLAS blocking only
+    assert np.all(sub["d_logits"][1] == 0.0)
+

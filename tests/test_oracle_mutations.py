@@ -27,6 +27,8 @@ MUTATIONS = [
      "codes[..., 0::2] = lo\n    codes[..., 1::2] = hi"),                         # nibble order
     ("nf4.py", "product = (table[codes] * scale)", "product = (table[codes[..., ::-1]] * scale)"),
     ("moe.py", 'order = np.argsort(-logits, axis=1, kind="stable")', 'order = np.argsort(logits, axis=1, kind="stable")[:, ::-1]'),
+    ("moe.py", "w[t] * (dw[t] - float(np.dot(w[t], dw[t])))", "w[t] * dw[t]"),     # router: no softmax mean
+    ("moe.py", "w[t] * (dw[t] - float(np.dot(w[t], dw[t])))", "(dw[t] - float(np.dot(w[t], dw[t])))"),
 ]
 
 
