@@ -512,6 +512,17 @@ e4b_status e4b_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n
   return E4B_OK;
 }
 
+e4b_status e4b_nf4_quantize(const e4b_bf16* w, int64_t n, uint8_t* packed, float* absmax, e4b_stream_t stream) {
+  if (n < 0 || n % 64) return E4B_ERR_INVALID_ARG;
+  if (n == 0) return E4B_OK;
+  if (!aligned16(w) || !aligned16(packed) || absmax == nullptr || (reinterpret_cast<uintptr_t>(absmax) & 3u))
+    return E4B_ERR_INVALID_ARG;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  E4B_CUDA(launch_nf4_quantize(reinterpret_cast<const uint16_t*>(w), n, packed, absmax, sms, (cudaStream_t)stream));
+  return E4B_OK;
+}
+
 e4b_status e4b_profiler_enable(int32_t on) {
   std::lock_guard<std::mutex> lock(g_prof_mu);
   g_prof_on = on != 0;

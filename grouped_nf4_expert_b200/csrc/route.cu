@@ -374,6 +374,46 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restr
   }
 }
 
+// NF4 quantisation, one warp per block of 64 weights (lane l holds elements
+// 2l and 2l+1): absmax = max |w| over the block; each code is the level
+// nearest to w / absmax (IEEE float32 division and distances, an exact tie to
+// the lower code); a block whose absmax is not positive gets the code of the
+// level 0 (7).
+__device__ __forceinline__ uint32_t nf4_nearest_code(float x) {
+  uint32_t best = 0;
+  float bd = fabsf(__fsub_rn(x, nf4_level(0)));
+#pragma unroll
+  for (int c = 1; c < 16; ++c) {
+    const float d = fabsf(__fsub_rn(x, nf4_level(c)));
+    if (d < bd) {
+      bd = d;
+      best = (uint32_t)c;
+    }
+  }
+  return best;
+}
+
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const uint32_t* __restrict__ w_pairs, int64_t nblocks,
+                                                           uint8_t* __restrict__ packed, float* __restrict__ absmax) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t b = gw; b < nblocks; b += nw) {
+    const uint32_t pr = __ldg(w_pairs + b * 32 + lane);
+    const float w0 = bf16lo_to_f32(pr), w1 = bf16hi_to_f32(pr);
+    // |w| >= 0: its bit patterns order like unsigned integers (a NaN ranks above every number).
+    const uint32_t m = max(__float_as_uint(fabsf(w0)), __float_as_uint(fabsf(w1)));
+    const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, m));
+    uint32_t c0 = 7, c1 = 7;
+    if (amax > 0.0f) {
+      c0 = nf4_nearest_code(__fdiv_rn(w0, amax));
+      c1 = nf4_nearest_code(__fdiv_rn(w1, amax));
+    }
+    packed[b * 32 + lane] = (uint8_t)((c0 << 4) | c1);
+    if (lane == 0) absmax[b] = amax;
+  }
+}
+
 // Waits on an mbarrier that nothing ever arrives on: the bounded wait must
 // give up, record E4B_ERR_DEVICE_TIMEOUT and let the CTA finish.
 __global__ void watchdog_kernel(DeviceError* err, long long timeout_ns) {
@@ -459,6 +499,17 @@ cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64
   if (grid < 1) grid = 1;
   LaunchScope scope("nf4_dequant", stream);
   nf4_dequant_kernel<<<(int)grid, 256, 0, stream>>>(packed, absmax, nblocks, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t n, uint8_t* packed, float* absmax, int num_sms,
+                                cudaStream_t stream) {
+  const int64_t nblocks = n / 64;
+  int64_t grid = (nblocks + 7) / 8;  // 8 warps of 256 threads, a warp per block
+  if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
+  if (grid < 1) grid = 1;
+  LaunchScope scope("nf4_quantize", stream);
+  nf4_quantize_kernel<<<(int)grid, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(w), nblocks, packed, absmax);
   return cudaGetLastError();
 }
 

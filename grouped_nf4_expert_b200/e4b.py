@@ -91,6 +91,7 @@ _SIGNATURES = {
                                ctypes.POINTER(FwdBuffers), ctypes.POINTER(BwdBuffers), c_vp, c_vp, c_vp, c_vp,
                                c_vp, c_sz, c_vp]),
     "e4b_nf4_dequant": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
+    "e4b_nf4_quantize": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_vp]),
     "e4b_debug_watchdog": (c_i32, [c_vp, c_sz, c_i64, c_vp]),
     "e4b_profiler_enable": (c_i32, [c_i32]),
     "e4b_profiler_read": (c_i32, [ctypes.POINTER(KernelTime), c_i32, ctypes.POINTER(c_i32)]),
@@ -173,6 +174,12 @@ def e4b_check_device_error(ws, stream=None) -> int:
 def e4b_nf4_dequant(packed, absmax, out, stream=None):
     _check(lib().e4b_nf4_dequant(_ptr(packed), _ptr(absmax), out.numel(), _ptr(out), _stream(stream)),
            "e4b_nf4_dequant")
+
+
+def e4b_nf4_quantize(w, packed, absmax, stream=None):
+    """bf16 weights (n elements, n % 64 == 0) -> packed NF4 codes [n/2] u8 and absmax [n/64] f32."""
+    _check(lib().e4b_nf4_quantize(_ptr(w), w.numel(), _ptr(packed), _ptr(absmax), _stream(stream)),
+           "e4b_nf4_quantize")
 
 
 def e4b_debug_watchdog(ws, timeout_ns: int, stream=None):

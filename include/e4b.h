@@ -232,6 +232,25 @@ e4b_status e4b_lora_wgrad(const e4b_moe_dims *dims, int32_t T, const e4b_routing
 e4b_status e4b_nf4_dequant(const uint8_t *packed, const float *absmax, int64_t n, e4b_bf16 *out,
                            e4b_stream_t stream);
 
+/* Quantises n bf16 weights (n a multiple of 64; blocks of 64 consecutive
+ * elements, i.e. along the rows of a row-major [..., K] stack with K % 64 ==
+ * 0) to NF4: packed uint8 [n/2] (element 2m in the high nibble of byte m),
+ * absmax float32 [n/64].  Per block absmax = max |w|; each code is the level
+ * nearest to w / absmax, computed as an IEEE float32 division and float32
+ * distances |w/absmax - level| with an exact tie going to the lower code; a
+ * block whose absmax is 0 gets code 7 (the level 0) throughout.  This is the
+ * step that turns a bf16 fused expert stack into the frozen NF4 base the
+ * grouped GEMMs read (and that e4b_nf4_dequant inverts up to rounding).
+ * w and packed 16-byte aligned, absmax 4-byte aligned; device pointers owned
+ * by the caller; invalid sizes or alignment -> E4B_ERR_INVALID_ARG with no
+ * launch.  Non-finite weights give what the same float32 rules give (a NaN
+ * makes the block's absmax NaN and its codes 7).
+ * Pages: "How do I QLoRA-train the fused experts of a MoE", section "The
+ * abstraction that fails, and what replaces it" (the packed NF4 base chosen
+ * with quant_type= on the loader) and section "Smallest correct example"
+ * (the loader quantising the fused stacks to 4 bit). */
+e4b_status e4b_nf4_quantize(const e4b_bf16 *w, int64_t n, uint8_t *packed, float *absmax, e4b_stream_t stream);
+
 /* Watchdog self-test: launches one CTA that waits on an mbarrier nothing
  * arrives on, with a limit of `timeout_ns` nanoseconds, so that the bounded
  * wait runs out and records E4B_ERR_DEVICE_TIMEOUT in `ws`.  No GPU fault. */

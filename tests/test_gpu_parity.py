@@ -134,6 +134,61 @@ def test_nf4_dequant_bit_exact():
     assert np.array_equal(got, want[0]), np.flatnonzero(got != want[0])[:10]
 
 
+def _quantize_gpu(w_bits):
+    w = torch.from_numpy(w_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    packed = torch.empty(w.numel() // 2, dtype=torch.uint8, device="cuda")
+    absmax = torch.empty(w.numel() // 64, dtype=torch.float32, device="cuda")
+    e4b.e4b_nf4_quantize(w, packed, absmax)
+    torch.cuda.synchronize()
+    return packed.cpu().numpy(), absmax.cpu().numpy()
+
+
+def test_nf4_quantize_bit_exact_special_blocks():
+    # codes are integers decided in float32 on both sides: they must agree bit for bit
+    rng = np.random.default_rng(3)
+    lv = oracle.nf4_table().astype(np.float32)
+    blocks = [np.zeros(64, np.float32),                                   # zero block -> code 7, absmax 0
+              np.r_[np.zeros(63), 0.25].astype(np.float32),              # a single nonzero
+              rng.standard_normal(64).astype(np.float32) * 1e-38,        # subnormal scale
+              rng.standard_normal(64).astype(np.float32) * 1e37,         # huge scale
+              -np.abs(rng.standard_normal(64)).astype(np.float32),      # all negative
+              np.r_[1.0, -1.0, np.zeros(62)].astype(np.float32)]         # the two extreme levels
+    # exact midpoints between adjacent levels (scaled by a power of two: w / absmax stays exact)
+    mids = (lv[:-1] + lv[1:]) / np.float32(2.0)
+    blk = np.zeros(64, np.float32)
+    blk[0] = 1.0
+    blk[1:16] = mids
+    blocks.append(blk * np.float32(0.5))
+    for scale in (0.02, 1.0, 3.0):
+        blocks += [(rng.standard_normal(64) * scale).astype(np.float32) for _ in range(200)]
+    w = np.stack(blocks).reshape(-1)
+    w_bits = oracle.bf16_round_bits(w)                # the bf16 weights both sides see
+    w32 = inputs.bits_to_f32(w_bits)
+    want_p, want_a = oracle.quantize_nf4(w32.reshape(1, -1))
+    got_p, got_a = _quantize_gpu(w_bits)
+    assert np.array_equal(got_p, want_p[0]), np.flatnonzero(got_p != want_p[0])[:10]
+    assert np.array_equal(got_a.view(np.uint32), want_a[0].view(np.uint32))
+
+
+def test_nf4_quantize_full_size_stack_sampled_blocks():
+    # a gate_up-sized stack of the fine-grained workload (128 x 1536 x 2048 bf16, 805 MB), checked on sampled blocks
+    E, R, K = 128, 1536, 2048
+    g = torch.Generator(device="cuda").manual_seed(5)
+    w = (torch.randn(E * R * K, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    packed = torch.empty(w.numel() // 2, dtype=torch.uint8, device="cuda")
+    absmax = torch.empty(w.numel() // 64, dtype=torch.float32, device="cuda")
+    e4b.e4b_nf4_quantize(w, packed, absmax)
+    torch.cuda.synchronize()
+    nblk = w.numel() // 64
+    idx = torch.from_numpy(np.sort(np.random.default_rng(6).choice(nblk, 20000, replace=False))).cuda()
+    wb = w.view(-1, 64)[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+    want_p, want_a = oracle.quantize_nf4(inputs.bits_to_f32(wb))
+    got_p = packed.view(-1, 32)[idx].cpu().numpy()
+    got_a = absmax[idx].cpu().numpy()
+    assert np.array_equal(got_p, want_p)
+    assert np.array_equal(got_a.view(np.uint32), want_a.reshape(-1).view(np.uint32))
+
+
 # --------------------------------------------------------------------- routing
 
 @pytest.mark.parametrize("name", list(SMALL))

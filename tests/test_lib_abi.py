@@ -126,5 +126,10 @@ def test_dequant_and_watchdog_argument_checks(so):
     assert so.e4b_nf4_dequant(p[0], p[1], 100, p[2], None) == e4b.E4B_ERR_INVALID_ARG  # not a multiple of 64
     assert so.e4b_nf4_dequant(p[0] + 1, p[1], 64, p[2], None) == e4b.E4B_ERR_INVALID_ARG
     assert so.e4b_nf4_dequant(p[0], p[1], 0, p[2], None) == e4b.E4B_OK  # nothing to do
+    assert so.e4b_nf4_quantize(p[0], 100, p[1], p[2], None) == e4b.E4B_ERR_INVALID_ARG  # not a multiple of 64
+    assert so.e4b_nf4_quantize(p[0] + 2, 64, p[1], p[2], None) == e4b.E4B_ERR_INVALID_ARG  # unaligned weights
+    assert so.e4b_nf4_quantize(p[0], 64, p[1] + 1, p[2], None) == e4b.E4B_ERR_INVALID_ARG  # unaligned codes
+    assert so.e4b_nf4_quantize(p[0], 64, p[1], p[2] + 2, None) == e4b.E4B_ERR_INVALID_ARG  # unaligned absmax
+    assert so.e4b_nf4_quantize(p[0], 0, p[1], p[2], None) == e4b.E4B_OK  # nothing to do
     assert so.e4b_debug_watchdog(p[0], 256, 0, None) == e4b.E4B_ERR_INVALID_ARG
     assert so.e4b_debug_watchdog(p[0], 8, 1000, None) == e4b.E4B_ERR_INVALID_ARG
