@@ -46,5 +46,6 @@ from .moe import (  # noqa: F401
     moe_forward,
     moe_backward,
     router_backward,
+    topk_softmax_backward,
     expert_weights,
 )

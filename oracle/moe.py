@@ -32,7 +32,10 @@ Pins (tests/test_oracle_moe.py): B = 0 gives exactly the base-only block;
 a per-token, per-expert brute-force loop; dense-delta equivalence with
 ``W + s B A`` materialised; E = 1, k = 1 against torch's SiLU, matmul and
 autograd; central finite differences of every gradient; routing against
-torch.topk/softmax and a stable library sort.
+torch.topk/softmax and a stable library sort.  Router backward (for a trained
+router): central finite differences of the block's loss in the logits, torch
+autograd through topk + softmax, and the softmax invariants (selected entries
+of a row sum to 0, unselected entries exactly 0, k = 1 gives 0).
 """
 
 from __future__ import annotations
@@ -283,6 +286,29 @@ def moe_backward(x, logits, dY, experts: Experts, k: int, alpha: float,
     return out
 
 
+def topk_softmax_backward(logits, k: int, dY, yd, tokens: Optional[Iterable[int]] = None):
+    """Router-logit gradient from the per-slot expert outputs ``yd``.
+
+    ``yd`` is indexed by flat slot ``t * k + j`` (an array [T*k, H] or a
+    mapping); ``ids`` and ``w`` are the top-k routing of ``logits``.  The
+    steps are the two of :func:`router_backward`: ``dw[t, j] = <dY[t],
+    yd[t*k + j]>``, then the softmax-over-top-k backward.  Only the rows in
+    ``tokens`` (every row when None) are computed; the others stay zero.
+    """
+    ids, w = route_topk(logits, k)
+    dY = np.asarray(dY, dtype=np.float64)
+    T = dY.shape[0]
+    E = np.asarray(logits).shape[1]
+    rows = range(T) if tokens is None else sorted(set(int(t) for t in tokens))
+    d_logits = np.zeros((T, E), dtype=np.float64)
+    dw = np.zeros((T, k), dtype=np.float64)
+    for t in rows:
+        for j in range(k):
+            dw[t, j] = float(np.dot(dY[t], np.asarray(yd[t * k + j], dtype=np.float64)))
+        d_logits[t, ids[t]] = w[t] * (dw[t] - float(np.dot(w[t], dw[t])))
+    return {"d_logits": d_logits, "dw": dw, "ids": ids, "w": w}
+
+
 def router_backward(x, logits, dY, experts: Experts, k: int, alpha: float,
                     tokens: Optional[Iterable[int]] = None):
     """Gradient of the loss with respect to the router logits, for a trained router.
@@ -303,16 +329,4 @@ def router_backward(x, logits, dY, experts: Experts, k: int, alpha: float,
     ``dw`` [T, k].
     """
     fwd = moe_forward(x, logits, experts, k, alpha, tokens=tokens)
-    ids, w = fwd["ids"], fwd["w"]
-    dY = np.asarray(dY, dtype=np.float64)
-    T = dY.shape[0]
-    E = np.asarray(logits).shape[1]
-    rows = range(T) if tokens is None else sorted(set(int(t) for t in tokens))
-    d_logits = np.zeros((T, E), dtype=np.float64)
-    dw = np.zeros((T, k), dtype=np.float64)
-    for t in rows:
-        for j in range(k):
-            dw[t, j] = float(np.dot(dY[t], fwd["yd"][t * k + j]))
-        d_logits[t, ids[t]] = w[t] * (dw[t] - float(np.dot(w[t], dw[t])))
-    return {"d_logits": d_logits, "dw": dw, "ids": ids, "w": w}
-
+    return topk_softmax_backward(logits, k, dY, fwd["yd"], tokens=tokens)

@@ -287,3 +287,22 @@ def test_router_backward_invariants(tiny):
     assert np.allclose(sub["d_logits"][[0, 7, 19]], dl[[0, 7, 19]], rtol=1e-12, atol=0)  # BLAS blocking only
     assert np.all(sub["d_logits"][1] == 0.0)
 
+
+
+def test_topk_softmax_backward_against_torch_autograd():
+    # The same gradient from torch's own topk + softmax + autograd (float64),
+    # for arbitrary per-slot outputs yd: L = sum_t sum_j w_tj <dY_t, yd_tj>.
+    rng = np.random.default_rng(11)
+    T, E, k, H = 24, 12, 4, 40
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    dY = rng.standard_normal((T, H))
+    yd = rng.standard_normal((T * k, H))
+    got = oracle.topk_softmax_backward(logits, k, dY, yd)
+    lt = torch.tensor(logits, dtype=torch.float64, requires_grad=True)
+    vals, idx = torch.topk(lt, k, dim=1)
+    w = torch.softmax(vals, dim=1)
+    dw = (torch.tensor(dY)[:, None, :] * torch.tensor(yd).view(T, k, H)).sum(-1)
+    (w * dw).sum().backward()
+    assert np.array_equal(got["ids"], idx.numpy())
+    assert np.allclose(got["d_logits"], lt.grad.numpy(), rtol=1e-12, atol=1e-13)
+    assert np.allclose(got["dw"], dw.detach().numpy(), rtol=1e-12, atol=1e-13)
