@@ -100,6 +100,20 @@ def stream_bytes(cfg, touched):
             "nf4_stream_fwd_down": touched * cfg.H * cfg.I * per_weight}
 
 
+def router_bwd_bytes(cfg):
+    """Algorithmic HBM bytes of one router-backward launch: per token its k expert-output rows and
+    its upstream-gradient row (bf16), its ids, weights and rows (int32/fp32), and its [E] fp32
+    logit-gradient row written."""
+    T, k, H, E = cfg.T, cfg.top_k, cfg.H, cfg.E
+    return T * (k + 1) * H * 2 + T * k * 12 + T * E * 4
+
+
+def quantize_bytes(n):
+    """Algorithmic HBM bytes of quantising n bf16 weights: read once, NF4 codes and fp32 block
+    scales written once."""
+    return n * 2 + n // 2 + (n // 64) * 4
+
+
 def nf4_gemm_flops(cfg):
     """Algorithmic FLOPs of the four grouped NF4 GEMM launches of one step."""
     N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
@@ -407,6 +421,30 @@ def main():
     e2e = {"value": cfg.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
+    # ---- the rows next to the path, each timed alone (HBM-bound by design)
+    next_rows = {}
+    if not fwd_only:  # router backward (for a trained router) on this step's forward outputs
+        d_logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
+        rb_ms = timed(args.steps, lambda: blk.e4b_router_backward(d.dY, d_logits)) / args.steps
+        rb_b = router_bwd_bytes(cfg)
+        next_rows["router_backward"] = {
+            "launch_ms": rb_ms, "algorithmic_bytes": rb_b, "achieved": rb_b / (rb_ms / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rb_b / (rb_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "bound": "hbm", "note": "d(logits) [T,E] from dY and the forward's y_perm"}
+        del d_logits
+    nq = cfg.E * 2 * cfg.I * cfg.H  # the workload's gate_up stack, bf16 N(0, sigma_w)
+    gq = torch.Generator(device=dev).manual_seed(1234 + rank)
+    wq = (torch.randn(nq, generator=gq, device=dev) * cfg.sigma_w).to(torch.bfloat16)
+    pq = torch.empty(nq // 2, dtype=torch.uint8, device=dev)
+    aq = torch.empty(nq // 64, dtype=torch.float32, device=dev)
+    q_ms = timed(args.steps, lambda: e4b.e4b_nf4_quantize(wq, pq, aq)) / args.steps
+    q_b = quantize_bytes(nq)
+    next_rows["nf4_quantize"] = {
+        "launch_ms": q_ms, "weights": nq, "algorithmic_bytes": q_b, "achieved": q_b / (q_ms / 1e3) / 1e9,
+        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_b / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "bound": "hbm", "note": "bf16 gate_up stack [E,2I,H] -> packed NF4 + fp32 absmax"}
+    del wq, pq, aq
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -419,6 +457,7 @@ def main():
         "profiled_ms_per_step": prof_ms / args.steps,
         "e2e": e2e,
         "gpu_launches": launches,
+        "next_rows": next_rows,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -500,6 +500,22 @@ e4b_status e4b_lora_wgrad(const e4b_moe_dims* dims, int32_t T, const e4b_routing
   return E4B_OK;
 }
 
+e4b_status e4b_router_backward(const e4b_moe_dims* dims, int32_t T, const e4b_routing* routing,
+                               const e4b_bf16* y_perm, const e4b_bf16* dY, float* d_logits, float* dw,
+                               e4b_stream_t stream) {
+  E4B_TRY(check_dims(dims, T));
+  E4B_TRY(check_routing(routing));
+  if (!aligned16(y_perm) || !aligned16(dY) || !aligned16(d_logits)) return E4B_ERR_INVALID_ARG;
+  if (dw != nullptr && !aligned16(dw)) return E4B_ERR_INVALID_ARG;
+  if (T == 0) return E4B_OK;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  E4B_CUDA(launch_router_bwd(reinterpret_cast<const uint16_t*>(dY), reinterpret_cast<const uint16_t*>(y_perm),
+                             routing->row_of_slot, routing->topk_ids, routing->topk_w, T, dims->top_k, dims->H,
+                             dims->E, d_logits, dw, sms, (cudaStream_t)stream));
+  return E4B_OK;
+}
+
 e4b_status e4b_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n, e4b_bf16* out,
                            e4b_stream_t stream) {
   if (n < 0 || n % 64) return E4B_ERR_INVALID_ARG;

@@ -63,6 +63,9 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, 
 cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot, const float* topk_w, int T,
                            int k, int H, uint16_t* out, int num_sms, cudaStream_t stream);
 
+cudaError_t launch_router_bwd(const uint16_t* dY, const uint16_t* y_perm, const int32_t* row_of_slot,
+                              const int32_t* topk_ids, const float* topk_w, int T, int k, int H, int E,
+                              float* d_logits, float* dw, int num_sms, cudaStream_t stream);
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t n, uint8_t* packed, float* absmax, int num_sms,
                                 cudaStream_t stream);
 cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n, uint16_t* out,

@@ -358,6 +358,87 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   }
 }
 
+// Router backward, one warp per token.  dw_j = <dY[t], y_perm[row(t,j)]> in
+// fp32 (lanes across H in 16-byte pieces, the k rows of a batch loaded
+// together, then a butterfly sum), followed by the backward of the softmax
+// over the k selected logits: d_logit[ids_j] = w_j (dw_j - sum_i w_i dw_i);
+// every other logit of the row gets 0.
+constexpr int kRbwdSlots = 8;
+__global__ void __launch_bounds__(256) router_bwd_kernel(const uint16_t* __restrict__ dY,
+                                                         const uint16_t* __restrict__ y_perm,
+                                                         const int32_t* __restrict__ row_of_slot,
+                                                         const int32_t* __restrict__ topk_ids,
+                                                         const float* __restrict__ topk_w, int T, int k, int H,
+                                                         int E, float* __restrict__ d_logits,
+                                                         float* __restrict__ dw_out) {
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), nw = gridDim.x * (blockDim.x >> 5);
+  const int vec = H / 8;
+  for (int t = gw; t < T; t += nw) {
+    const int my_row = (lane < k) ? __ldg(row_of_slot + (size_t)t * k + lane) : 0;
+    const float my_w = (lane < k) ? __ldg(topk_w + (size_t)t * k + lane) : 0.0f;
+    const int my_id = (lane < k) ? __ldg(topk_ids + (size_t)t * k + lane) : 0;
+    const uint4* dyp = reinterpret_cast<const uint4*>(dY + (size_t)t * H);
+    float my_dw = 0.0f;
+    for (int j0 = 0; j0 < k; j0 += kRbwdSlots) {
+      const uint4* rp[kRbwdSlots];
+#pragma unroll
+      for (int j = 0; j < kRbwdSlots; ++j)
+        rp[j] = reinterpret_cast<const uint4*>(y_perm +
+                                               (size_t)__shfl_sync(0xffffffffu, my_row, (j0 + j) & 31) * H);
+      float acc[kRbwdSlots];
+#pragma unroll
+      for (int j = 0; j < kRbwdSlots; ++j) acc[j] = 0.0f;
+      for (int pc = lane; pc < vec; pc += 32) {
+        const uint4 d = __ldg(dyp + pc);
+        uint4 q[kRbwdSlots];
+#pragma unroll
+        for (int j = 0; j < kRbwdSlots; ++j)
+          if (j0 + j < k) q[j] = __ldg(rp[j] + pc);
+        const uint32_t* dp = reinterpret_cast<const uint32_t*>(&d);
+        float dv[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          dv[2 * c] = bf16lo_to_f32(dp[c]);
+          dv[2 * c + 1] = bf16hi_to_f32(dp[c]);
+        }
+#pragma unroll
+        for (int j = 0; j < kRbwdSlots; ++j)
+          if (j0 + j < k) {
+            const uint32_t* p = reinterpret_cast<const uint32_t*>(&q[j]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              acc[j] = fmaf(dv[2 * c], bf16lo_to_f32(p[c]), acc[j]);
+              acc[j] = fmaf(dv[2 * c + 1], bf16hi_to_f32(p[c]), acc[j]);
+            }
+          }
+      }
+#pragma unroll
+      for (int j = 0; j < kRbwdSlots; ++j) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        if (lane == j0 + j) my_dw = acc[j];
+      }
+    }
+    // sum_i w_i dw_i over the selected slots (lanes >= k contribute 0)
+    float mean = my_w * my_dw;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mean += __shfl_xor_sync(0xffffffffu, mean, o);
+    const float g = my_w * (my_dw - mean);
+    float* row = d_logits + (size_t)t * E;
+    if ((E & 3) == 0) {
+      for (int e = lane; e < E / 4; e += 32) reinterpret_cast<float4*>(row)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      for (int e = lane; e < E; e += 32) row[e] = 0.0f;
+    }
+    __syncwarp();  // the zeros are ordered before the selected entries
+    if (lane < k) {
+      row[my_id] = g;
+      if (dw_out != nullptr) dw_out[(size_t)t * k + lane] = my_dw;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restrict__ packed,
                                                           const float* __restrict__ absmax, int64_t nblocks,
                                                           uint16_t* __restrict__ out) {
@@ -374,43 +455,78 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restr
   }
 }
 
-// NF4 quantisation, one warp per block of 64 weights (lane l holds elements
-// 2l and 2l+1): absmax = max |w| over the block; each code is the level
-// nearest to w / absmax (IEEE float32 division and distances, an exact tie to
-// the lower code); a block whose absmax is not positive gets the code of the
-// level 0 (7).
-__device__ __forceinline__ uint32_t nf4_nearest_code(float x) {
-  uint32_t best = 0;
-  float bd = fabsf(__fsub_rn(x, nf4_level(0)));
-#pragma unroll
-  for (int c = 1; c < 16; ++c) {
-    const float d = fabsf(__fsub_rn(x, nf4_level(c)));
-    if (d < bd) {
-      bd = d;
-      best = (uint32_t)c;
-    }
-  }
-  return best;
+// NF4 quantisation.  The code of x = w / absmax (an IEEE float32 division)
+// is the level nearest to x in float32 distance |x - level|, an exact tie
+// going to the lower code; a block whose absmax is not positive gets the code
+// of the level 0 (7).  The levels ascend, so with c the number of levels
+// below x (a 4-step search of the level table) the nearest level is c-1 or c:
+// every other level is at least one level gap (> 0.07) further from x, far
+// more than float32 rounding of numbers below 2 can close, so comparing the
+// two distances takes the same decision as comparing all 16.  A NaN x ends
+// at c = 0 and gets code 0, as the full comparison gives.
+__device__ __forceinline__ uint32_t nf4_nearest_code(float x, const float* lv) {
+  int c = (lv[7] < x) ? 8 : 0;
+  c += (lv[c + 3] < x) ? 4 : 0;
+  c += (lv[c + 1] < x) ? 2 : 0;
+  c += (lv[c] < x) ? 1 : 0;
+  const int lo = c > 0 ? c - 1 : 0;
+  const float d_lo = fabsf(__fsub_rn(x, lv[lo]));
+  const float d_hi = fabsf(__fsub_rn(x, lv[c]));
+  return (uint32_t)(d_lo <= d_hi ? lo : c);
 }
 
-__global__ void __launch_bounds__(256) nf4_quantize_kernel(const uint32_t* __restrict__ w_pairs, int64_t nblocks,
-                                                           uint8_t* __restrict__ packed, float* __restrict__ absmax) {
+// Eight consecutive weights of one lane (a 16-byte piece); the 8 lanes of a
+// 64-element block take its absmax by a shuffle max.  Validity is uniform
+// over those 8 lanes; every lane takes part in the shuffles.
+__device__ __forceinline__ void nf4_quantize_piece(uint4 v, bool ok, int64_t p, int lane, const float* lv,
+                                                   uint32_t* __restrict__ packed4, float* __restrict__ absmax) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float w[8];
+  uint32_t m = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    w[2 * c] = bf16lo_to_f32(u[c]);
+    w[2 * c + 1] = bf16hi_to_f32(u[c]);
+  }
+  // |w| >= 0: its bit patterns order like unsigned integers (a NaN ranks above every number).
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = max(m, __float_as_uint(fabsf(w[i])));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  const float amax = __uint_as_float(m);
+  uint32_t out = 0x77777777u;
+  if (amax > 0.0f) {
+    out = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)  // element 2b in the high nibble of byte b
+      out |= nf4_nearest_code(__fdiv_rn(w[i], amax), lv) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+  }
+  if (ok) {
+    packed4[p] = out;
+    if ((lane & 7) == 0) absmax[p >> 3] = amax;
+  }
+}
+
+// A warp covers 4 blocks (32 pieces) per quad and loads two quads before
+// quantising either.
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const uint4* __restrict__ w8, int64_t nblocks,
+                                                           uint32_t* __restrict__ packed4,
+                                                           float* __restrict__ absmax) {
+  __shared__ float lv[16];
+  if (threadIdx.x < 16) lv[threadIdx.x] = nf4_level(threadIdx.x);
+  __syncthreads();
   const int lane = threadIdx.x & 31;
+  const int64_t n8 = nblocks * 8;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t b = gw; b < nblocks; b += nw) {
-    const uint32_t pr = __ldg(w_pairs + b * 32 + lane);
-    const float w0 = bf16lo_to_f32(pr), w1 = bf16hi_to_f32(pr);
-    // |w| >= 0: its bit patterns order like unsigned integers (a NaN ranks above every number).
-    const uint32_t m = max(__float_as_uint(fabsf(w0)), __float_as_uint(fabsf(w1)));
-    const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, m));
-    uint32_t c0 = 7, c1 = 7;
-    if (amax > 0.0f) {
-      c0 = nf4_nearest_code(__fdiv_rn(w0, amax));
-      c1 = nf4_nearest_code(__fdiv_rn(w1, amax));
-    }
-    packed[b * 32 + lane] = (uint8_t)((c0 << 4) | c1);
-    if (lane == 0) absmax[b] = amax;
+  for (int64_t q = gw * 2; q * 32 < n8; q += nw * 2) {
+    const int64_t p0 = q * 32 + lane, p1 = p0 + 32;
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    const uint4 a = (p0 < n8) ? __ldg(w8 + p0) : z;
+    const uint4 b = (p1 < n8) ? __ldg(w8 + p1) : z;
+    nf4_quantize_piece(a, p0 < n8, p0, lane, lv, packed4, absmax);
+    nf4_quantize_piece(b, p1 < n8, p1, lane, lv, packed4, absmax);
   }
 }
 
@@ -491,6 +607,16 @@ cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot,
   return cudaGetLastError();
 }
 
+cudaError_t launch_router_bwd(const uint16_t* dY, const uint16_t* y_perm, const int32_t* row_of_slot,
+                              const int32_t* topk_ids, const float* topk_w, int T, int k, int H, int E,
+                              float* d_logits, float* dw, int num_sms, cudaStream_t stream) {
+  const int blocks = (T + 7) / 8;  // 8 warps of 256 threads, a warp per token
+  const int grid = blocks < num_sms * 8 ? blocks : num_sms * 8;
+  LaunchScope scope("router_bwd", stream);
+  router_bwd_kernel<<<grid, 256, 0, stream>>>(dY, y_perm, row_of_slot, topk_ids, topk_w, T, k, H, E, d_logits, dw);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64_t n, uint16_t* out, int num_sms,
                                cudaStream_t stream) {
   const int64_t nblocks = n / 64;
@@ -505,11 +631,12 @@ cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int64
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t n, uint8_t* packed, float* absmax, int num_sms,
                                 cudaStream_t stream) {
   const int64_t nblocks = n / 64;
-  int64_t grid = (nblocks + 7) / 8;  // 8 warps of 256 threads, a warp per block
-  if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
+  int64_t grid = (nblocks + 63) / 64;  // 8 warps of 256 threads, 8 blocks per warp iteration
+  if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
   if (grid < 1) grid = 1;
   LaunchScope scope("nf4_quantize", stream);
-  nf4_quantize_kernel<<<(int)grid, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(w), nblocks, packed, absmax);
+  nf4_quantize_kernel<<<(int)grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(w), nblocks,
+                                                     reinterpret_cast<uint32_t*>(packed), absmax);
   return cudaGetLastError();
 }
 

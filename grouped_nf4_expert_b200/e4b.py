@@ -90,6 +90,8 @@ _SIGNATURES = {
     "e4b_lora_wgrad": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
                                ctypes.POINTER(FwdBuffers), ctypes.POINTER(BwdBuffers), c_vp, c_vp, c_vp, c_vp,
                                c_vp, c_sz, c_vp]),
+    "e4b_router_backward": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing), c_vp, c_vp, c_vp,
+                                    c_vp, c_vp]),
     "e4b_nf4_dequant": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "e4b_nf4_quantize": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_vp]),
     "e4b_debug_watchdog": (c_i32, [c_vp, c_sz, c_i64, c_vp]),
@@ -269,6 +271,11 @@ class Block:
                                     ctypes.byref(self._fwd), ctypes.byref(self._bwd), _ptr(self.dA_gu),
                                     _ptr(self.dB_gu), _ptr(self.dA_d), _ptr(self.dB_d), _ptr(self.ws),
                                     self.ws.numel(), _stream(stream)), "e4b_lora_wgrad")
+
+    def e4b_router_backward(self, dY, d_logits, dw=None, stream=None):
+        _check(lib().e4b_router_backward(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
+                                         _ptr(self.y_perm), _ptr(dY), _ptr(d_logits), _ptr(dw), _stream(stream)),
+               "e4b_router_backward")
 
     def check_device_error(self, stream=None) -> int:
         return e4b_check_device_error(self.ws, stream)

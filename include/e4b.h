@@ -226,6 +226,28 @@ e4b_status e4b_lora_wgrad(const e4b_moe_dims *dims, int32_t T, const e4b_routing
                           e4b_bf16 *dA_gu, e4b_bf16 *dB_gu, e4b_bf16 *dA_d, e4b_bf16 *dB_d,
                           void *ws, size_t ws_bytes, e4b_stream_t stream);
 
+/* Router-logit gradient, for a trained router (the router is frozen by
+ * default and its logits are inputs; this is the extra step that training it
+ * needs).  The top-k selection is piecewise constant, so the logits get a
+ * gradient through the routing weights only:
+ *   dw[t,j]  = <dY[t], y_perm[row(t,j)]>   (fp32 sum of bf16 products)
+ *   d_logits[t, ids[t,j]] = w[t,j] * (dw[t,j] - sum_i w[t,i] dw[t,i])
+ * and every other entry of d_logits is 0 (the whole [T, E] array is written).
+ * routing: what e4b_route_permute wrote for these T tokens (ids, weights,
+ * row_of_slot are read); y_perm: the unweighted expert outputs the forward
+ * wrote (e4b_fwd_buffers.y_perm); dY: bf16 [T, H], the upstream gradient the
+ * dgrad also takes.  d_logits: float32 [T, E]; dw: float32 [T, top_k] or NULL
+ * (not written).  All device pointers, 16-byte aligned, owned by the caller;
+ * invalid arguments -> E4B_ERR_INVALID_ARG / E4B_ERR_UNSUPPORTED with no
+ * launch; T == 0 launches nothing.  Needs no workspace.  Deterministic.
+ * Pages: "How do I QLoRA-train the fused experts of a MoE", section "The
+ * abstraction that fails, and what replaces it" (TRAIN_ROUTER trains the
+ * router `mlp.gate.weight`; the weights are the softmax over the selected
+ * logits). */
+e4b_status e4b_router_backward(const e4b_moe_dims *dims, int32_t T, const e4b_routing *routing,
+                               const e4b_bf16 *y_perm, const e4b_bf16 *dY, float *d_logits, float *dw,
+                               e4b_stream_t stream);
+
 /* Dequantises n NF4 elements (n a multiple of 64): packed uint8 [n/2],
  * absmax float32 [n/64] -> bf16 [n], with the same device routine the
  * grouped GEMMs decode with.  For bit-exact testing of the decode. */

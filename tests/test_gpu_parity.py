@@ -161,6 +161,15 @@ def test_nf4_quantize_bit_exact_special_blocks():
     blocks.append(blk * np.float32(0.5))
     for scale in (0.02, 1.0, 3.0):
         blocks += [(rng.standard_normal(64) * scale).astype(np.float32) for _ in range(200)]
+    # every bf16 value of [-amax, amax] next to a block maximum amax, for amax = 1 (x = w exactly) and
+    # amax = 1.5, 0.3 (x rounded by the division): every decision near every midpoint is taken
+    for amax in (1.0, 1.5, 0.3):
+        top = int(oracle.bf16_round_bits(np.array([amax], np.float32))[0])
+        vals = np.r_[np.arange(0, top + 1), np.arange(0x8000, 0x8000 + top + 1)].astype(np.uint16)
+        vals = inputs.bits_to_f32(vals)
+        vals = np.r_[vals, np.zeros((-vals.size) % 63, np.float32)].reshape(-1, 63)
+        blocks += list(np.c_[np.full((vals.shape[0], 1), inputs.bits_to_f32(np.array([top], np.uint16))[0]),
+                             vals].astype(np.float32))
     w = np.stack(blocks).reshape(-1)
     w_bits = oracle.bf16_round_bits(w)                # the bf16 weights both sides see
     w32 = inputs.bits_to_f32(w_bits)
@@ -382,3 +391,87 @@ def test_repeated_full_size_runs_are_bit_identical(name):
         else:
             for a, b in zip(ref, cur):
                 assert torch.equal(a, b)
+
+# --------------------------------------------------------------------- router backward (trained router)
+
+RBWD_TOL = 1e-4  # fp32 sums of exact bf16 products against float64
+
+
+def _router_bwd_gpu(blk, d, T, E, k):
+    d_logits = torch.full((T, E), float("nan"), dtype=torch.float32, device="cuda")
+    dw = torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda")
+    blk.e4b_router_backward(d.dY, d_logits, dw)
+    torch.cuda.synchronize()
+    return d_logits.cpu().numpy(), dw.cpu().numpy()
+
+
+def _check_router_rows(dl_gpu, dw_gpu, ref, rows, tol):
+    assert rel_err(dl_gpu[rows], ref["d_logits"][rows]) <= tol
+    assert rel_err(dw_gpu[rows], ref["dw"][rows]) <= tol
+    mask = np.zeros(ref["d_logits"].shape, dtype=bool)
+    np.put_along_axis(mask, ref["ids"].astype(np.int64), True, axis=1)
+    sel = mask[rows]
+    assert np.all(dl_gpu[rows][~sel] == 0.0)  # every unselected logit exactly 0
+    assert np.all(np.isfinite(dl_gpu[rows][sel]))
+
+
+@pytest.mark.parametrize("name", list(SMALL) + ["k1", "k32"])
+def test_router_backward_given_expert_outputs(name):
+    # The kernel alone: seeded per-slot expert outputs placed in y_perm, every row compared.
+    cfg = {"k1": inputs.Config("k1", E=8, H=128, I=64, top_k=1, T=70, r=8, alpha=16.0, routing="normal", seed=41),
+           "k32": inputs.Config("k32", E=40, H=192, I=64, top_k=32, T=45, r=8, alpha=16.0, routing="normal",
+                                seed=42)}.get(name) or SMALL[name]
+    prob, d, blk = run(cfg, fwd=False, dgrad=False, wgrad=False)
+    ros = check_routing(prob, blk)
+    T, E, k, H = cfg.T, cfg.E, cfg.top_k, cfg.H
+    yd = inputs.bf16_bits(np.random.default_rng(900 + cfg.seed).standard_normal((T * k, H), dtype=np.float32))
+    blk.y_perm[torch.from_numpy(ros).cuda()] = torch.from_numpy(yd.view(np.int16)).cuda().view(torch.bfloat16)
+    dl, dw = _router_bwd_gpu(blk, d, T, E, k)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    ref = oracle.topk_softmax_backward(prob.logits, k, dY, inputs.bits_to_f32(yd).astype(np.float64))
+    _check_router_rows(dl, dw, ref, np.arange(T), RBWD_TOL)
+    if k == 1:
+        assert np.all(dl == 0.0)
+
+
+def test_router_backward_full_size_sampled_tokens():
+    # train workload (E128 H2048 top-8, 8192 tokens): the whole launch, sampled rows compared
+    cfg = inputs.CONFIGS["train"]
+    prob, d, blk = run(cfg, fwd=False, dgrad=False, wgrad=False)
+    ros = blk.row_of_slot.cpu().numpy().astype(np.int64)
+    T, E, k, H = cfg.T, cfg.E, cfg.top_k, cfg.H
+    yd = inputs.bf16_bits(np.random.default_rng(950).standard_normal((T * k, H), dtype=np.float32))
+    blk.y_perm[torch.from_numpy(ros).cuda()] = torch.from_numpy(yd.view(np.int16)).cuda().view(torch.bfloat16)
+    dl, dw = _router_bwd_gpu(blk, d, T, E, k)
+    toks = _sample_tokens(T, 64, 102)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    ref = oracle.topk_softmax_backward(prob.logits, k, dY, {int(f): inputs.bits_to_f32(yd[f]).astype(np.float64)
+                                                            for t in toks for f in range(t * k, t * k + k)},
+                                       tokens=toks)
+    _check_router_rows(dl, dw, ref, toks, RBWD_TOL)
+    # properties at any size: every row has at most k nonzeros, all finite, sum ~ 0
+    assert np.all(np.isfinite(dl)) and np.all((dl != 0).sum(axis=1) <= k)
+    assert np.abs(dl.sum(axis=1)).max() <= 1e-4 * np.abs(dl).max()
+
+
+@pytest.mark.parametrize("name", ["medium", "stream_zipf_r64"])
+def test_router_backward_through_the_forward(name):
+    # End to end: the GPU forward's y_perm feeds the router backward; against the oracle's own forward.
+    cfg = SMALL[name]
+    prob, d, blk = run(cfg, dgrad=False, wgrad=False)
+    dl, dw = _router_bwd_gpu(blk, d, cfg.T, cfg.E, cfg.top_k)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    ref = oracle.router_backward(x, prob.logits, dY, oracle_experts(prob), cfg.top_k, cfg.alpha)
+    _check_router_rows(dl, dw, ref, np.arange(cfg.T), TOL)
+
+
+def test_router_backward_train_workload_sampled_tokens():
+    cfg = inputs.CONFIGS["train"]
+    prob, d, blk = run(cfg, dgrad=False, wgrad=False)
+    dl, dw = _router_bwd_gpu(blk, d, cfg.T, cfg.E, cfg.top_k)
+    toks = _sample_tokens(cfg.T, 12, 103)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    ref = oracle.router_backward(x, prob.logits, dY, oracle_experts(prob), cfg.top_k, cfg.alpha, tokens=toks)
+    _check_router_rows(dl, dw, ref, toks, TOL)

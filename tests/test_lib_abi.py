@@ -115,6 +115,17 @@ def test_null_and_misaligned_pointers_refused(so):
     bwd_ok = e4b.BwdBuffers(*p[26:31])
     assert so.e4b_lora_wgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(fwd), ctypes.byref(bwd_ok),
                              p[33], None, p[35], p[36], ws, wsb, None) == e4b.E4B_ERR_INVALID_ARG
+    # router backward: unaligned or missing tensors; dw optional; T == 0 launches nothing
+    assert so.e4b_router_backward(ctypes.byref(d), T, ctypes.byref(routing), p[24] + 2, p[31], p[37], None,
+                                  None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_router_backward(ctypes.byref(d), T, ctypes.byref(routing), p[24], None, p[37], None,
+                                  None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_router_backward(ctypes.byref(d), T, ctypes.byref(routing), p[24], p[31], p[37], p[38] + 4,
+                                  None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_router_backward(ctypes.byref(d), T, ctypes.byref(bad), p[24], p[31], p[37], None,
+                                  None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_router_backward(ctypes.byref(d), 0, ctypes.byref(routing), p[24], p[31], p[37], None,
+                                  None) == e4b.E4B_OK
     # unsupported dims are refused before pointers are looked at
     d.r = 12
     assert so.e4b_lora_wgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(fwd), ctypes.byref(bwd_ok),
