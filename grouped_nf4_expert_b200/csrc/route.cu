@@ -475,32 +475,81 @@ __device__ __forceinline__ uint32_t nf4_nearest_code(float x, const float* lv) {
   return (uint32_t)(d_lo <= d_hi ? lo : c);
 }
 
-// Eight consecutive weights of one lane (a 16-byte piece); the 8 lanes of a
-// 64-element block take its absmax by a shuffle max.  Validity is uniform
-// over those 8 lanes; every lane takes part in the shuffles.
+__device__ __forceinline__ float rcp_approx(float a) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(a));
+  return r;
+}
+
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+// The fast decision.  x' = w * rcp(a) is within 2^-21 of the float32
+// quotient x = fl(w / a) (|x| <= 1; the reciprocal is within 1 ulp, the
+// product within half an ulp).  The level nearest to x changes only at the
+// midpoints between adjacent levels (the float32 distance comparison agrees
+// with "x above the midpoint" except within a few ulps of it).  Buckets of
+// width 1/128 over [-1, 1] each hold the midpoint nearest to them, its
+// float32 bits with the low 4 bits replaced by the code just below it (an
+// error of at most 15 ulps, under 2^-20): code = that code + (x' above the
+// stored midpoint).  Midpoints are more than 0.07 apart, so no other midpoint
+// lies between x' and the stored one.  Whenever x' is within 2^-18 of the
+// stored midpoint the IEEE division decides instead; further away, x is on
+// the same side of the true midpoint as x' by more than 2^-20, far beyond
+// the rounding of the distances, so both decisions agree.  Blocks whose a is
+// outside [2^-125, 2^125], where the reciprocal may not be a normal number,
+// always divide.  Each lane reads its own copy of the table (bank = lane),
+// so the lookups never conflict.
+constexpr int kQBuckets = 257;
+constexpr float kQMargin = 3.814697265625e-06f;  // 2^-18
+constexpr float kQMagic = 12583040.0f;           // 1.5 * 2^23 + 128: bits = 0x4B400000 + 128 + round(128 x)
+
 __device__ __forceinline__ void nf4_quantize_piece(uint4 v, bool ok, int64_t p, int lane, const float* lv,
-                                                   uint32_t* __restrict__ packed4, float* __restrict__ absmax) {
+                                                   uint32_t tbl_lane, uint32_t* __restrict__ packed4,
+                                                   float* __restrict__ absmax) {
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-  float w[8];
-  uint32_t m = 0;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    w[2 * c] = bf16lo_to_f32(u[c]);
-    w[2 * c + 1] = bf16hi_to_f32(u[c]);
-  }
-  // |w| >= 0: its bit patterns order like unsigned integers (a NaN ranks above every number).
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m = max(m, __float_as_uint(fabsf(w[i])));
+  // absmax: |w| bf16 bit patterns order like unsigned integers (a NaN ranks above every number)
+  uint32_t m2 = __vmaxu2(u[0] & 0x7fff7fffu, u[1] & 0x7fff7fffu);
+  m2 = __vmaxu2(m2, __vmaxu2(u[2] & 0x7fff7fffu, u[3] & 0x7fff7fffu));
+  uint32_t m = max(m2 & 0xffffu, m2 >> 16) << 16;
   m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
   m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
   m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
   const float amax = __uint_as_float(m);
+  float w[8];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    w[2 * c] = __uint_as_float(mul_lo_u32(u[c], 65536u));  // low half: an integer multiply, off the ALU pipe
+    w[2 * c + 1] = bf16hi_to_f32(u[c]);
+  }
   uint32_t out = 0x77777777u;
   if (amax > 0.0f) {
-    out = 0;
+    bool exact = !(amax >= 2.350988701644575e-38f && amax <= 4.253529586511730793e+37f);  // 2^-125, 2^125
+    if (!exact) {
+      const float ra = rcp_approx(amax);
+      uint32_t near = 0;  // number of x' within the margin of their stored midpoint
+      out = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)  // element 2b in the high nibble of byte b
-      out |= nf4_nearest_code(__fdiv_rn(w[i], amax), lv) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+      for (int i = 0; i < 8; ++i) {  // element 2b in the high nibble of byte b
+        const float x = __fmul_rn(w[i], ra);
+        const float t = __fmaf_rn(x, 128.0f, kQMagic);
+        const float mid = ld_shared_f32(mad_lo_u32(__float_as_uint(t), 128u, tbl_lane));
+        const float d = __fsub_rn(mid, x);
+        const uint32_t code = mad_hi_u32(__float_as_uint(d), 2u, __float_as_uint(mid) & 15u);
+        near = mad_hi_u32(__float_as_uint(__fsub_rn(fabsf(d), kQMargin)), 2u, near);  // sign bit: |d| < margin
+        out = mad_lo_u32(code, 1u << (8 * (i >> 1) + ((i & 1) ? 0 : 4)), out);
+      }
+      exact = near != 0;
+    }
+    if (exact) {  // rare: some x' near a midpoint, or an extreme block scale
+      out = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        out |= nf4_nearest_code(__fdiv_rn(w[i], amax), lv) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+    }
   }
   if (ok) {
     packed4[p] = out;
@@ -514,19 +563,44 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const uint4* __restri
                                                            uint32_t* __restrict__ packed4,
                                                            float* __restrict__ absmax) {
   __shared__ float lv[16];
+  __shared__ float tbl[kQBuckets * 32];  // [bucket][lane]
   if (threadIdx.x < 16) lv[threadIdx.x] = nf4_level(threadIdx.x);
+  for (int e = threadIdx.x; e < kQBuckets; e += blockDim.x) {
+    const float center = (float)(e - 128) * 0.0078125f;
+    int best = 0;
+    float bm = 0.5f * (nf4_level(0) + nf4_level(1)), bd = fabsf(bm - center);
+    for (int c = 1; c < 15; ++c) {
+      const float mc = 0.5f * (nf4_level(c) + nf4_level(c + 1));
+      if (fabsf(mc - center) < bd) {
+        bd = fabsf(mc - center);
+        bm = mc;
+        best = c;
+      }
+    }
+    const float v = __uint_as_float((__float_as_uint(bm) & ~15u) | (uint32_t)best);
+    for (int l = 0; l < 32; ++l) tbl[e * 32 + l] = v;
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
+  // shared address of this lane's copy of bucket b is tbl + 128 b + 4 lane = bits(t) * 128 + tbl_lane
+  const uint32_t tbl_lane = (uint32_t)__cvta_generic_to_shared(tbl) + 4u * lane - 0x4B400000u * 128u;
   const int64_t n8 = nblocks * 8;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t q = gw * 2; q * 32 < n8; q += nw * 2) {
+  // the next iteration's two pieces are loaded before this iteration's are quantised
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  int64_t q = gw * 2;
+  uint4 a = (q * 32 + lane < n8) ? __ldg(w8 + q * 32 + lane) : z;
+  uint4 b = (q * 32 + 32 + lane < n8) ? __ldg(w8 + q * 32 + 32 + lane) : z;
+  for (; q * 32 < n8; q += nw * 2) {
     const int64_t p0 = q * 32 + lane, p1 = p0 + 32;
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    const uint4 a = (p0 < n8) ? __ldg(w8 + p0) : z;
-    const uint4 b = (p1 < n8) ? __ldg(w8 + p1) : z;
-    nf4_quantize_piece(a, p0 < n8, p0, lane, lv, packed4, absmax);
-    nf4_quantize_piece(b, p1 < n8, p1, lane, lv, packed4, absmax);
+    const int64_t n0 = p0 + nw * 64, n1 = n0 + 32;
+    const uint4 an = (n0 < n8) ? __ldg(w8 + n0) : z;
+    const uint4 bn = (n1 < n8) ? __ldg(w8 + n1) : z;
+    nf4_quantize_piece(a, p0 < n8, p0, lane, lv, tbl_lane, packed4, absmax);
+    nf4_quantize_piece(b, p1 < n8, p1, lane, lv, tbl_lane, packed4, absmax);
+    a = an;
+    b = bn;
   }
 }
 
@@ -632,7 +706,7 @@ cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t n, uint8_t* packed, f
                                 cudaStream_t stream) {
   const int64_t nblocks = n / 64;
   int64_t grid = (nblocks + 63) / 64;  // 8 warps of 256 threads, 8 blocks per warp iteration
-  if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
+  if (grid > (int64_t)num_sms * 6) grid = (int64_t)num_sms * 6;  // 33 KB of tables: 6 CTAs per SM
   if (grid < 1) grid = 1;
   LaunchScope scope("nf4_quantize", stream);
   nf4_quantize_kernel<<<(int)grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(w), nblocks,

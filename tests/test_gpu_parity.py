@@ -179,6 +179,36 @@ def test_nf4_quantize_bit_exact_special_blocks():
     assert np.array_equal(got_a.view(np.uint32), want_a[0].view(np.uint32))
 
 
+def _near_boundary_blocks(n_amax=400, seed=7):
+    # Blocks whose w / absmax (IEEE float32) falls within 2^-17 of a level or of a midpoint between two
+    # adjacent levels: the decisions a fast approximate quotient could get wrong.
+    lv = oracle.nf4_table().astype(np.float64)
+    pts = np.r_[lv, (lv[:-1] + lv[1:]) / 2.0]
+    rng = np.random.default_rng(seed)
+    tops = np.unique(oracle.bf16_round_bits(rng.uniform(0.01, 10.0, n_amax).astype(np.float32)))
+    blocks, hits = [], 0
+    for top in tops:
+        a = inputs.bits_to_f32(np.array([top], np.uint16))[0]
+        vals = inputs.bits_to_f32(np.r_[np.arange(1, top), np.arange(0x8001, 0x8000 + top)].astype(np.uint16))
+        x = (vals / a).astype(np.float64)  # float32 division, then exact widening
+        near = np.abs(x[:, None] - pts[None, :]).min(axis=1) <= 2.0 ** -17
+        v = vals[near][:63]
+        if v.size:
+            hits += v.size
+            blocks.append(np.r_[a, v, np.zeros(63 - v.size, np.float32)].astype(np.float32))
+    return blocks, hits
+
+
+def test_nf4_quantize_bit_exact_near_decision_boundaries():
+    blocks, hits = _near_boundary_blocks()
+    assert hits >= 500
+    w_bits = oracle.bf16_round_bits(np.stack(blocks).reshape(-1))
+    want_p, want_a = oracle.quantize_nf4(inputs.bits_to_f32(w_bits).reshape(1, -1))
+    got_p, got_a = _quantize_gpu(w_bits)
+    assert np.array_equal(got_p, want_p[0]), np.flatnonzero(got_p != want_p[0])[:10]
+    assert np.array_equal(got_a.view(np.uint32), want_a[0].view(np.uint32))
+
+
 def test_nf4_quantize_full_size_stack_sampled_blocks():
     # a gate_up-sized stack of the fine-grained workload (128 x 1536 x 2048 bf16, 805 MB), checked on sampled blocks
     E, R, K = 128, 1536, 2048
