@@ -332,11 +332,12 @@ def main():
     if st != e4b.E4B_OK:
         raise RuntimeError("device error after warm-up: %s" % e4b.STATUS.get(st, st))
 
-    def timed(K, body):
+    def timed(K, body, flush_l2=True):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         sync_all()
         for i in range(K):
-            flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
+            if flush_l2:
+                flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
             evs[i][0].record()
             body()
             evs[i][1].record()
@@ -421,28 +422,32 @@ def main():
     e2e = {"value": cfg.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
-    # ---- the rows next to the path, each timed alone (HBM-bound by design)
+    # ---- the rows next to the path, each timed alone (HBM-bound by design).  Both read more than the
+    # 126 MB L2 per launch, so they are timed back to back without the flush (whose dirty lines would
+    # be written back during the next launch).
     next_rows = {}
     if not fwd_only:  # router backward (for a trained router) on this step's forward outputs
         d_logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
-        rb_ms = timed(args.steps, lambda: blk.e4b_router_backward(d.dY, d_logits)) / args.steps
+        rb_ms = timed(args.steps, lambda: blk.e4b_router_backward(d.dY, d_logits), flush_l2=False) / args.steps
         rb_b = router_bwd_bytes(cfg)
         next_rows["router_backward"] = {
             "launch_ms": rb_ms, "algorithmic_bytes": rb_b, "achieved": rb_b / (rb_ms / 1e3) / 1e9,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rb_b / (rb_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "bound": "hbm", "note": "d(logits) [T,E] from dY and the forward's y_perm"}
+            "bound": "hbm", "l2": "not flushed: > 300 MB read per launch",
+            "note": "d(logits) [T,E] from dY and the forward's y_perm"}
         del d_logits
     nq = cfg.E * 2 * cfg.I * cfg.H  # the workload's gate_up stack, bf16 N(0, sigma_w)
     gq = torch.Generator(device=dev).manual_seed(1234 + rank)
     wq = (torch.randn(nq, generator=gq, device=dev) * cfg.sigma_w).to(torch.bfloat16)
     pq = torch.empty(nq // 2, dtype=torch.uint8, device=dev)
     aq = torch.empty(nq // 64, dtype=torch.float32, device=dev)
-    q_ms = timed(args.steps, lambda: e4b.e4b_nf4_quantize(wq, pq, aq)) / args.steps
+    q_ms = timed(args.steps, lambda: e4b.e4b_nf4_quantize(wq, pq, aq), flush_l2=False) / args.steps
     q_b = quantize_bytes(nq)
     next_rows["nf4_quantize"] = {
         "launch_ms": q_ms, "weights": nq, "algorithmic_bytes": q_b, "achieved": q_b / (q_ms / 1e3) / 1e9,
         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_b / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-        "bound": "hbm", "note": "bf16 gate_up stack [E,2I,H] -> packed NF4 + fp32 absmax"}
+        "bound": "hbm", "l2": "not flushed: > 800 MB read per launch",
+        "note": "bf16 gate_up stack [E,2I,H] -> packed NF4 + fp32 absmax"}
     del wq, pq, aq
 
     line = {
