@@ -7,6 +7,9 @@ epilogue, down, combine), the input gradient (down dgrad with the SwiGLU
 backward, gate_up dgrad, un-permute) and the LoRA weight gradients -- the
 four C-ABI calls of libe4b.so.  Default workload: E=128, H=2048, I=768,
 top-8, T=8192 tokens per GPU, LoRA r=64, alpha=128, Zipf(1.1) routing.
+A forward-only workload (``--workload decode``: 16 tokens) times the serving
+call e4b_moe_serve_fwd (routing + forward, nothing kept for a backward)
+replayed from a CUDA graph.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
 bounded token samples of the same workload instead.
@@ -308,13 +311,14 @@ def main():
     base, lora = d.base(), d.lora()
     grads = (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d)
 
-    fwd_only = cfg.passes == ("fwd",)  # decode-sized serving batch: the forward alone
+    fwd_only = cfg.passes == ("fwd",)  # decode-sized serving batch: the serving forward alone
 
     def step():
+        if fwd_only:  # routing + forward for inference, nothing kept for a backward
+            blk.e4b_moe_serve_fwd(d.logits, d.x, base, lora, keep_gu=False)
+            return
         blk.e4b_route_permute(d.logits, d.x)
         blk.e4b_grouped_nf4_lora_fwd(base, lora)
-        if fwd_only:
-            return
         blk.e4b_grouped_nf4_lora_dgrad(base, lora, d.dY)
         blk.e4b_lora_wgrad()
         if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
@@ -349,11 +353,31 @@ def main():
             ms = float(t.item())
         return ms
 
-    # ---- main timed region
-    launches0 = e4b.e4b_launch_count()
-    with ClockSampler(dev) as clocks:
-        total_ms = timed(args.steps, step)
-    launches = e4b.e4b_launch_count() - launches0
+    def capture(body):
+        """A CUDA graph of body() (the serving step: the library allocates and synchronises nothing),
+        and the number of library launches it holds."""
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        n0 = e4b.e4b_launch_count()
+        with torch.cuda.graph(g):
+            body()
+        n = e4b.e4b_launch_count() - n0
+        torch.cuda.synchronize(dev)
+        return g, n
+
+    # ---- main timed region (the serving step replays a CUDA graph of the call)
+    graphs = []
+    if fwd_only:
+        g_step, per_step = capture(step)
+        graphs.append(g_step)
+        with ClockSampler(dev) as clocks:
+            total_ms = timed(args.steps, g_step.replay)
+        launches = per_step * args.steps
+    else:
+        launches0 = e4b.e4b_launch_count()
+        with ClockSampler(dev) as clocks:
+            total_ms = timed(args.steps, step)
+        launches = e4b.e4b_launch_count() - launches0
     st = blk.check_device_error()
     if st != e4b.E4B_OK:
         raise RuntimeError("device error in the timed region: %s" % e4b.STATUS.get(st, st))
@@ -418,7 +442,12 @@ def main():
         for h, t in zip(houts, outs):
             h.copy_(t, non_blocking=True)
 
-    e2e_ms = timed(args.steps, e2e_step)
+    if fwd_only:  # the whole serving step, copies included, as one graph
+        g_e2e, _ = capture(e2e_step)
+        graphs.append(g_e2e)
+        e2e_ms = timed(args.steps, g_e2e.replay)
+    else:
+        e2e_ms = timed(args.steps, e2e_step)
     e2e = {"value": cfg.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
@@ -454,7 +483,9 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(cfg, world, "flushed between timed steps by a 256 MiB write"),
+        "config": dict(workload_config(cfg, world, "flushed between timed steps by a 256 MiB write"),
+                       cuda_graph=fwd_only, call=("e4b_moe_serve_fwd" if fwd_only else
+                                                  "route_permute + lora_fwd + lora_dgrad + lora_wgrad")),
         "tflops": flops * world / (ms_per_step / 1e3) / 1e12,
         "step_flop_per_gpu": flops,
         "roofline": roofline,
@@ -467,6 +498,7 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(prob, args.cpu_sample_tokens)
+    del graphs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -350,6 +350,85 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
   return E4B_OK;
 }
 
+e4b_status e4b_moe_serve_fwd(const e4b_moe_dims* dims, int32_t T, const float* logits, const e4b_bf16* x,
+                             const e4b_routing* routing, const e4b_nf4_experts* base, const e4b_lora* lora,
+                             const e4b_fwd_buffers* fwd, e4b_bf16* y, void* ws, size_t ws_bytes,
+                             e4b_stream_t stream) {
+  E4B_TRY(check_dims(dims, T));
+  E4B_TRY(check_ws(dims, T, ws, ws_bytes));
+  E4B_TRY(check_routing(routing));
+  E4B_TRY(check_base(base));
+  E4B_TRY(check_lora(lora));
+  if (fwd == nullptr || !aligned16(fwd->x_perm) || !aligned16(fwd->p_gu) || !aligned16(fwd->act) ||
+      !aligned16(fwd->p_d) || !aligned16(fwd->y_perm) || (fwd->gu != nullptr && !aligned16(fwd->gu)))
+    return E4B_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(x) || !aligned16(y)) return E4B_ERR_INVALID_ARG;
+  const int64_t N = (int64_t)T * dims->top_k;
+  if (!use_streaming_forward(N, dims->E)) {
+    // a prefill-sized batch: the training forward (it writes gu, so gu is required)
+    if (fwd->gu == nullptr) return E4B_ERR_INVALID_ARG;
+    E4B_TRY(e4b_route_permute(dims, T, logits, x, routing, fwd->x_perm, ws, ws_bytes, stream));
+    return e4b_grouped_nf4_lora_fwd(dims, T, routing, base, lora, fwd, y, ws, ws_bytes, stream);
+  }
+  if (T == 0) return E4B_OK;
+  int sms = 0;
+  E4B_CUDA(device_sms(&sms));
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int E = dims->E, H = dims->H, I = dims->I, r = dims->r, k = dims->top_k;
+  const float s = dims->alpha / (float)r;
+  int32_t* scratch = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sizeof(DeviceError));
+  E4B_CUDA(launch_route_serve(logits, T, E, H, k, routing->topk_ids, routing->topk_w, routing->counts,
+                              routing->offsets, routing->row_of_slot, routing->slot_of_row, routing->tiles,
+                              mtiles_cap(N, E), rows_cap(N, E), scratch, sms, st));
+  // x_perm[row] = x[token]; p_gu[row] = s * x A_gu[e]^T
+  E4B_CUDA(launch_lora_rows(reinterpret_cast<const uint16_t*>(x), true, routing->topk_ids, routing->row_of_slot,
+                            (int)N, k, H, lora->A_gu, r, s, fwd->x_perm, fwd->p_gu, sms, st));
+  Nf4GemmHost g{};
+  g.E = E;
+  g.H = H;
+  g.I = I;
+  g.r = r;
+  g.r_pad = r_padded(r);
+  g.tiles = routing->tiles;
+  g.rows_cap = rows_cap(N, E);
+  g.mt_cap = mtiles_cap(N, E);
+  g.err = static_cast<DeviceError*>(ws);
+  g.timeout_ns = kDefaultTimeoutNs;
+  // act = silu(gate) * up of W_gu x + p_gu B_gu^T (gu itself only when a buffer is given)
+  g.mode = kFwdGateUp;
+  g.nf4 = base->gate_up_nf4;
+  g.absmax = base->gate_up_absmax;
+  g.stored_rows = 2 * I;
+  g.stored_cols = H;
+  g.act_in = fwd->x_perm;
+  g.K = H;
+  g.n_dim = 2 * I;
+  g.lora_a_rows = fwd->p_gu;
+  g.lora_w = lora->B_gu;
+  g.out0 = fwd->gu;
+  g.out1 = fwd->act;
+  E4B_CUDA(launch_nf4_stream(g, sms, st));
+  // p_d[row] = s * act A_d[e]^T
+  E4B_CUDA(launch_lora_rows(fwd->act, false, routing->topk_ids, routing->row_of_slot, (int)N, k, I, lora->A_d, r,
+                            s, nullptr, fwd->p_d, sms, st));
+  // y_perm = W_d act + p_d B_d^T
+  g.mode = kFwdDown;
+  g.nf4 = base->down_nf4;
+  g.absmax = base->down_absmax;
+  g.stored_rows = H;
+  g.stored_cols = I;
+  g.act_in = fwd->act;
+  g.K = I;
+  g.n_dim = H;
+  g.lora_a_rows = fwd->p_d;
+  g.lora_w = lora->B_d;
+  g.out0 = fwd->y_perm;
+  g.out1 = nullptr;
+  E4B_CUDA(launch_nf4_stream(g, sms, st));
+  E4B_CUDA(launch_combine(fwd->y_perm, routing->row_of_slot, routing->topk_w, T, k, H, y, sms, st));
+  return E4B_OK;
+}
+
 e4b_status e4b_grouped_nf4_lora_dgrad(const e4b_moe_dims* dims, int32_t T, const e4b_routing* routing,
                                       const e4b_nf4_experts* base, const e4b_lora* lora,
                                       const e4b_fwd_buffers* fwd, const e4b_bf16* dY, const e4b_bwd_buffers* bwd,

@@ -54,6 +54,18 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
                          uint16_t* x_perm, int64_t rows_cap, int32_t* scratch, int num_sms,
                          cudaStream_t stream);
 
+// Routing tables for the serving forward (no x gather, no padding markers for
+// batches of at most kRouteTokensPerBlock tokens, which take one launch).
+cudaError_t launch_route_serve(const float* logits, int T, int E, int H, int k, int32_t* topk_ids, float* topk_w,
+                               int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* slot_of_row,
+                               int32_t* tiles, int64_t mt_cap, int64_t rows_cap, int32_t* scratch, int num_sms,
+                               cudaStream_t stream);
+// out[row(f)] = bf16(s * src_row(f) . A[e(f)]^T) per routed slot f on the CUDA cores; src_row is the token's
+// row (by_token) or the permuted row; copy_dst (optional) receives the source row at the permuted row.
+cudaError_t launch_lora_rows(const uint16_t* src, bool by_token, const int32_t* topk_ids, const int32_t* row_of_slot,
+                             int N, int k, int K, const uint16_t* A, int r, float s, uint16_t* copy_dst,
+                             uint16_t* out, int num_sms, cudaStream_t stream);
+
 // dst[row] = src[token of row] (optionally scaled by the slot's routing weight), zero for padding rows.
 cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, const int32_t* tiles,
                                const float* scale_w, int H, int k, int64_t rows_cap, uint16_t* dst,

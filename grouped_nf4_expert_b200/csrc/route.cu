@@ -226,6 +226,176 @@ __global__ void __launch_bounds__(32) route_rank_kernel(const int32_t* __restric
   }
 }
 
+// Routing of a batch of at most kRouteTokensPerBlock tokens in one CTA, for
+// the serving forward: top-k + softmax per token (as route_topk_kernel), the
+// expert counts, 128-aligned group offsets, the weight-streaming tile list
+// and the stable slot ranks (as route_scan_kernel and route_rank_kernel), in
+// one launch.  No padding markers and no m-tile lists: the serving forward
+// reads neither.
+template <int EPL>
+__global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                          int32_t* __restrict__ topk_ids,
+                                                          float* __restrict__ topk_w,
+                                                          int32_t* __restrict__ counts,
+                                                          int32_t* __restrict__ offsets,
+                                                          int32_t* __restrict__ row_of_slot,
+                                                          int32_t* __restrict__ tiles, int64_t st_offset) {
+  __shared__ int s_cnt[E4B_MAX_EXPERTS];
+  __shared__ int s_run[E4B_MAX_EXPERTS];
+  __shared__ int s_warp[32];
+  __shared__ int s_ids[kRouteTokensPerBlock * E4B_MAX_TOP_K];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int t = warp; t < T; t += nwarps) {
+    const float* row = logits + (size_t)t * E;
+    uint32_t key[EPL];
+    uint32_t live = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = (e < E) ? route_key(__ldg(row + e)) : 0u;
+      if (e < E) live |= 1u << i;
+    }
+    float my_v = 0.0f;
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+      uint32_t bk = 0u, bi = 0xffffffffu;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if ((live & (1u << i)) && (bi == 0xffffffffu || key[i] > bk)) {
+          bk = key[i];
+          bi = (uint32_t)(lane + 32 * i);
+        }
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t e_sel = __reduce_min_sync(0xffffffffu, (bk == kmax) ? bi : 0xffffffffu);
+      if ((int)(e_sel & 31u) == lane) live &= ~(1u << (e_sel >> 5));
+      if (lane == j) {
+        my_v = route_key_value(kmax);
+        my_e = (int)e_sel;
+      }
+    }
+    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const float z = (lane < k) ? expf(my_v - vmax) : 0.0f;
+    float sum = z;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) {
+      topk_ids[(size_t)t * k + lane] = my_e;
+      topk_w[(size_t)t * k + lane] = z / sum;
+      s_ids[t * k + lane] = my_e;
+      atomicAdd(&s_cnt[my_e], 1);
+    }
+  }
+  __syncthreads();
+  // one thread per expert: offsets and streaming tiles
+  const int e = threadIdx.x;
+  const int cnt = (e < E) ? s_cnt[e] : 0;
+  const int padded = (cnt + 127) / 128 * 128;
+  const int off = block_exclusive_scan(e < E ? padded : 0, s_warp);
+  const int n_st = (cnt + 31) / 32;
+  const int st_off = block_exclusive_scan(e < E ? n_st : 0, s_warp);
+  if (e < E) {
+    counts[e] = cnt;
+    offsets[e] = off;
+    s_run[e] = off;
+    int32_t* st = tiles + st_offset;
+    for (int i = 0; i < n_st; ++i) {
+      st[3 * (st_off + i)] = e;
+      st[3 * (st_off + i) + 1] = off + 32 * i;
+      st[3 * (st_off + i) + 2] = min(32, cnt - 32 * i);
+    }
+    if (e == E - 1) {
+      offsets[E] = off + padded;
+      tiles[0] = 0;  // no m-tile list
+      tiles[1] = off + padded;
+      tiles[2] = 0;  // no m-unit list
+      tiles[3] = st_off + n_st;
+    }
+  }
+  __syncthreads();
+  // stable ranks: warp 0 walks the slots in flat order, 32 at a time
+  if (warp == 0) {
+    const int N = T * k;
+    for (int f0 = 0; f0 < N; f0 += 32) {
+      const int f = f0 + lane;
+      const int ex = (f < N) ? s_ids[f] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, ex);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int leader = __ffs(peers) - 1;
+      if (ex >= 0) row_of_slot[f] = s_run[ex] + rank;
+      __syncwarp();
+      if (ex >= 0 && lane == leader) s_run[ex] += __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
+// LoRA down-projection of permuted rows on the CUDA cores, one CTA per routed
+// slot: out[row] = bf16(s * src_row . A[e]^T) over K, for the few rows of a
+// serving batch (the tensor-core projection is built for 128-row tiles).  The
+// source row is the token's row of `src` (by_token) or the slot's permuted
+// row; with `copy_dst` the source row is also copied to the slot's permuted
+// row (the x scatter of the serving forward).  fp32 products and sums.
+template <int R>
+__global__ void __launch_bounds__(256) lora_rows_kernel(const uint16_t* __restrict__ src, int by_token,
+                                                        const int32_t* __restrict__ topk_ids,
+                                                        const int32_t* __restrict__ row_of_slot, int N, int k,
+                                                        int K, const uint16_t* __restrict__ A, int r, float s,
+                                                        uint16_t* __restrict__ copy_dst,
+                                                        uint16_t* __restrict__ out) {
+  __shared__ float red[8][R];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int vec = K / 8;
+  for (int f = blockIdx.x; f < N; f += gridDim.x) {
+    const int e = __ldg(topk_ids + f), row = __ldg(row_of_slot + f);
+    const uint4* sp = reinterpret_cast<const uint4*>(src + (size_t)(by_token ? f / k : row) * K);
+    const uint4* ap = reinterpret_cast<const uint4*>(A + (size_t)e * r * K);
+    float acc[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j) acc[j] = 0.0f;
+    for (int pc = threadIdx.x; pc < vec; pc += blockDim.x) {
+      const uint4 q = __ldg(sp + pc);
+      if (copy_dst != nullptr) reinterpret_cast<uint4*>(copy_dst + (size_t)row * K)[pc] = q;
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(&q);
+      float xv[8];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        xv[2 * c] = bf16lo_to_f32(qw[c]);
+        xv[2 * c + 1] = bf16hi_to_f32(qw[c]);
+      }
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        if (j < r) {
+          const uint4 a = __ldg(ap + (size_t)j * vec + pc);
+          const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            acc[j] = fmaf(xv[2 * c], bf16lo_to_f32(aw[c]), acc[j]);
+            acc[j] = fmaf(xv[2 * c + 1], bf16hi_to_f32(aw[c]), acc[j]);
+          }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < R; ++j) red[warp][j] = acc[j];
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < r; j += blockDim.x) {  // r may exceed a one-warp block
+      float sum = 0.0f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w][j];
+      const __nv_bfloat16 h = __float2bfloat16_rn(s * sum);
+      out[(size_t)row * r + j] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+    __syncthreads();
+  }
+}
+
 __device__ __forceinline__ uint4 scale_bf16x8(uint4 q, float w) {
   uint32_t* p = reinterpret_cast<uint32_t*>(&q);
 #pragma unroll
@@ -281,11 +451,15 @@ constexpr int kRowsPerBatch = 8;
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ src_perm,
                                                       const int32_t* __restrict__ row_of_slot,
                                                       const float* __restrict__ topk_w, int T, int k, int H,
-                                                      uint16_t* __restrict__ out) {
+                                                      int split, uint16_t* __restrict__ out) {
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), nw = gridDim.x * (blockDim.x >> 5);
-  const int vec = H / 8;
-  for (int t = gw; t < T; t += nw) {
+  // a task is one of `split` equal column ranges of a token (split > 1 for small batches)
+  const int per = H / 8 / split;
+  for (int task = gw; task < T * split; task += nw) {
+    const int t = task / split;
+    const int pc0 = (task % split) * per;
+    const int vec = pc0 + per;
     // lane j < k holds slot j's permuted row and weight
     const int my_row = (lane < k) ? __ldg(row_of_slot + (size_t)t * k + lane) : 0;
     const float my_w = (lane < k) ? (topk_w ? __ldg(topk_w + (size_t)t * k + lane) : 1.0f) : 0.0f;
@@ -297,7 +471,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         rp[j] = reinterpret_cast<const uint4*>(src_perm + (size_t)__shfl_sync(0xffffffffu, my_row, j) * H);
         rw[j] = __shfl_sync(0xffffffffu, my_w, j);
       }
-      for (int pc = lane; pc < vec; pc += 32) {
+      for (int pc = pc0 + lane; pc < vec; pc += 32) {
         uint4 q[kRowsPerBatch];
 #pragma unroll
         for (int j = 0; j < kRowsPerBatch; ++j)
@@ -324,7 +498,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       }
       continue;
     }
-    for (int pc = lane; pc < vec; pc += 32) {
+    for (int pc = pc0 + lane; pc < vec; pc += 32) {
       float acc[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
@@ -659,7 +833,54 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
                                                   row_of_slot, slot_of_row);
   }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (x_perm == nullptr) return cudaSuccess;  // routing tables only
   return launch_gather_rows(x, slot_of_row, tiles, nullptr, H, k, rows_cap, x_perm, num_sms, stream);
+}
+
+cudaError_t launch_route_serve(const float* logits, int T, int E, int H, int k, int32_t* topk_ids, float* topk_w,
+                               int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* slot_of_row,
+                               int32_t* tiles, int64_t mt_cap, int64_t rows_cap, int32_t* scratch, int num_sms,
+                               cudaStream_t stream) {
+  if (T > kRouteTokensPerBlock)
+    return launch_route(logits, nullptr, T, E, H, k, topk_ids, topk_w, counts, offsets, row_of_slot, slot_of_row,
+                        tiles, mt_cap, nullptr, rows_cap, scratch, num_sms, stream);
+  const int64_t st_off = stiles_offset(mt_cap, E);
+  const int epl = (E + 31) / 32;
+  LaunchScope scope("route_small", stream);
+#define E4B_ROUTE_SMALL(P)                                                                                   \
+  route_small_kernel<P><<<1, 1024, 0, stream>>>(logits, T, E, k, topk_ids, topk_w, counts, offsets, row_of_slot, \
+                                                tiles, st_off)
+  if (epl <= 1)
+    E4B_ROUTE_SMALL(1);
+  else if (epl <= 2)
+    E4B_ROUTE_SMALL(2);
+  else if (epl <= 4)
+    E4B_ROUTE_SMALL(4);
+  else if (epl <= 8)
+    E4B_ROUTE_SMALL(8);
+  else if (epl <= 16)
+    E4B_ROUTE_SMALL(16);
+  else
+    E4B_ROUTE_SMALL(32);
+#undef E4B_ROUTE_SMALL
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_rows(const uint16_t* src, bool by_token, const int32_t* topk_ids, const int32_t* row_of_slot,
+                             int N, int k, int K, const uint16_t* A, int r, float s, uint16_t* copy_dst,
+                             uint16_t* out, int num_sms, cudaStream_t stream) {
+  const int pieces = K / 8;
+  const int threads = pieces >= 256 ? 256 : ((pieces + 31) / 32) * 32;
+  const int grid = N < num_sms * 8 ? N : num_sms * 8;
+  LaunchScope scope(copy_dst ? "scatter_lora_rows" : "lora_rows", stream);
+  const int bt = by_token ? 1 : 0;
+  if (r <= 16)
+    lora_rows_kernel<16><<<grid, threads, 0, stream>>>(src, bt, topk_ids, row_of_slot, N, k, K, A, r, s, copy_dst, out);
+  else if (r <= 32)
+    lora_rows_kernel<32><<<grid, threads, 0, stream>>>(src, bt, topk_ids, row_of_slot, N, k, K, A, r, s, copy_dst, out);
+  else
+    lora_rows_kernel<64><<<grid, threads, 0, stream>>>(src, bt, topk_ids, row_of_slot, N, k, K, A, r, s, copy_dst, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, const int32_t* tiles,
@@ -674,10 +895,14 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* slot_of_row, 
 
 cudaError_t launch_combine(const uint16_t* src_perm, const int32_t* row_of_slot, const float* topk_w, int T, int k,
                            int H, uint16_t* out, int num_sms, cudaStream_t stream) {
-  const int blocks = (T + 7) / 8;  // 8 warps of 256 threads, a warp per token
+  // a warp per token, or per 1/split of a token's columns when the batch has fewer tokens than 4 warps
+  // per SM (split divides the H/8 16-byte pieces and leaves at least 32 per task)
+  int split = 1;
+  while (T * split < num_sms * 4 && (H / 8) % (2 * split) == 0 && H / 8 / (2 * split) >= 32) split *= 2;
+  const int blocks = (T * split + 7) / 8;  // 8 warps of 256 threads
   const int grid = blocks < num_sms * 8 ? blocks : num_sms * 8;
   LaunchScope scope(topk_w ? "combine_y" : "combine_dx", stream);
-  combine_kernel<<<grid, 256, 0, stream>>>(src_perm, row_of_slot, topk_w, T, k, H, out);
+  combine_kernel<<<grid, 256, 0, stream>>>(src_perm, row_of_slot, topk_w, T, k, H, split, out);
   return cudaGetLastError();
 }
 

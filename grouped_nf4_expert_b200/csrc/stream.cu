@@ -413,10 +413,12 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
           for (int sl = 0; sl < 32; ++sl) epi[sl * 64 + (wrow - 64)] = v[sl];
           __syncwarp();
           if (lane == 0) mbar_arrive(epi_full);
+          if (p.out0 != nullptr) {  // gu is kept for a backward; a serving forward passes none
 #pragma unroll
-          for (int sl = 0; sl < 32; ++sl) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(v[sl]);
-            p.out0[(row0 + sl) * I2 + p.I + i] = *reinterpret_cast<const uint16_t*>(&h);
+            for (int sl = 0; sl < 32; ++sl) {
+              const __nv_bfloat16 h = __float2bfloat16_rn(v[sl]);
+              p.out0[(row0 + sl) * I2 + p.I + i] = *reinterpret_cast<const uint16_t*>(&h);
+            }
           }
         } else {
           ok = __all_sync(kFull, mbar_wait(epi_full, ti & 1, ctl, p.err, p.timeout_ns, 352));
@@ -426,7 +428,7 @@ __global__ void __launch_bounds__(nf4s::kThreads, 1)
             const float g = v[sl], uu = epi[sl * 64 + wrow];
             const __nv_bfloat16 hg = __float2bfloat16_rn(g);
             const __nv_bfloat16 ha = __float2bfloat16_rn(silu_f(g) * uu);
-            p.out0[(row0 + sl) * I2 + i] = *reinterpret_cast<const uint16_t*>(&hg);
+            if (p.out0 != nullptr) p.out0[(row0 + sl) * I2 + i] = *reinterpret_cast<const uint16_t*>(&hg);
             p.out1[(row0 + sl) * p.I + i] = *reinterpret_cast<const uint16_t*>(&ha);
           }
           __syncwarp();

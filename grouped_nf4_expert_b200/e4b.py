@@ -90,6 +90,9 @@ _SIGNATURES = {
     "e4b_lora_wgrad": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
                                ctypes.POINTER(FwdBuffers), ctypes.POINTER(BwdBuffers), c_vp, c_vp, c_vp, c_vp,
                                c_vp, c_sz, c_vp]),
+    "e4b_moe_serve_fwd": (c_i32, [ctypes.POINTER(MoeDims), c_i32, c_vp, c_vp, ctypes.POINTER(Routing),
+                                  ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora), ctypes.POINTER(FwdBuffers), c_vp,
+                                  c_vp, c_sz, c_vp]),
     "e4b_router_backward": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing), c_vp, c_vp, c_vp,
                                     c_vp, c_vp]),
     "e4b_nf4_dequant": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
@@ -246,6 +249,8 @@ class Block:
                                                            self.row_of_slot, self.slot_of_row, self.tiles)))
         self._fwd = FwdBuffers(*(t.data_ptr() for t in (self.x_perm, self.p_gu, self.gu, self.act, self.p_d,
                                                          self.y_perm)))
+        self._fwd_nogu = FwdBuffers(self.x_perm.data_ptr(), self.p_gu.data_ptr(), None, self.act.data_ptr(),
+                                    self.p_d.data_ptr(), self.y_perm.data_ptr())
         self._bwd = BwdBuffers(*(t.data_ptr() for t in (self.dyw, self.q_d, self.dgu, self.q_gu, self.dx_perm)))
 
     # -- the four hot-path calls -------------------------------------------------
@@ -271,6 +276,15 @@ class Block:
                                     ctypes.byref(self._fwd), ctypes.byref(self._bwd), _ptr(self.dA_gu),
                                     _ptr(self.dB_gu), _ptr(self.dA_d), _ptr(self.dB_d), _ptr(self.ws),
                                     self.ws.numel(), _stream(stream)), "e4b_lora_wgrad")
+
+    def e4b_moe_serve_fwd(self, logits, x, base: Nf4Experts, lora: Lora, keep_gu=True, stream=None):
+        """Routing + forward for inference into ``self.y``.  ``keep_gu=False`` passes no gu buffer
+        (allowed for decode-sized batches only; larger ones are refused without it)."""
+        fwd = self._fwd if keep_gu else self._fwd_nogu
+        _check(lib().e4b_moe_serve_fwd(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
+                                       ctypes.byref(self._routing), ctypes.byref(base), ctypes.byref(lora),
+                                       ctypes.byref(fwd), _ptr(self.y), _ptr(self.ws), self.ws.numel(),
+                                       _stream(stream)), "e4b_moe_serve_fwd")
 
     def e4b_router_backward(self, dY, d_logits, dw=None, stream=None):
         _check(lib().e4b_router_backward(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),

@@ -202,6 +202,31 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims *dims, int32_t T,
                                     const e4b_lora *lora, const e4b_fwd_buffers *fwd, e4b_bf16 *y,
                                     void *ws, size_t ws_bytes, e4b_stream_t stream);
 
+/* Serving forward: routing and the forward in one call, for inference
+ * (decode-sized batches above all): y = the block's output for x (bf16
+ * [T, H]) and logits (float32 [T, E]), the same arithmetic as
+ * e4b_route_permute + e4b_grouped_nf4_lora_fwd.  Batches with at most
+ * 16 * E routed slots take the serving pipeline: routing tables in one
+ * launch (T <= 64) or three, the x scatter fused with the LoRA projection
+ * s * x A_gu^T on the CUDA cores, the weight-streaming gate_up, the
+ * projection s * act A_d^T, the weight-streaming down and the weighted
+ * combine -- six launches, nothing kept for a backward: fwd->gu may be NULL
+ * (then not written), padding rows of the permuted buffers and
+ * routing->slot_of_row are left unspecified, and the m-tile lists in
+ * routing->tiles are not built, so the routing and buffers of a serving call
+ * must not be passed to e4b_grouped_nf4_lora_dgrad or e4b_lora_wgrad.
+ * Larger batches run e4b_route_permute + e4b_grouped_nf4_lora_fwd (fwd->gu
+ * is then required).  Argument checks, ownership and errors as for those two
+ * calls; the call allocates nothing and never synchronises, so it can be
+ * captured into a CUDA graph.
+ * Pages: section "Which project solves it" (grouped forward), section
+ * "Limitations" (the fast forward for inference) and METADATA "The package
+ * family" (one launch over the packed stacks). */
+e4b_status e4b_moe_serve_fwd(const e4b_moe_dims *dims, int32_t T, const float *logits, const e4b_bf16 *x,
+                             const e4b_routing *routing, const e4b_nf4_experts *base, const e4b_lora *lora,
+                             const e4b_fwd_buffers *fwd, e4b_bf16 *y, void *ws, size_t ws_bytes,
+                             e4b_stream_t stream);
+
 /* Input gradient for upstream dY (bf16 [T, H]): dyw = w * dY per slot,
  * q_d, the down-projection dgrad through the transposed re-dequantised base
  * plus LoRA with the SwiGLU backward fused in (dgu), q_gu, the gate_up dgrad

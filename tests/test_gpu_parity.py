@@ -505,3 +505,104 @@ def test_router_backward_train_workload_sampled_tokens():
     dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
     ref = oracle.router_backward(x, prob.logits, dY, oracle_experts(prob), cfg.top_k, cfg.alpha, tokens=toks)
     _check_router_rows(dl, dw, ref, toks, TOL)
+
+
+# --------------------------------------------------------------------- serving forward
+
+SERVE = ["tiny", "stream_r24", "stream_zipf_r64", "medium"]  # medium: a prefill-sized batch (training forward)
+
+
+def _serve(cfg, prob=None, keep_gu=False):
+    # keep_gu=False: no gu buffer, as a decode-sized serving call passes it
+    prob = prob if prob is not None else inputs.make_problem(cfg)
+    d = dv.upload(prob)
+    blk = e4b.Block(dv.dims_of(cfg), cfg.T)
+    blk.e4b_moe_serve_fwd(d.logits, d.x, d.base(), d.lora(), keep_gu=keep_gu)
+    assert blk.check_device_error() == e4b.E4B_OK
+    torch.cuda.synchronize()
+    return prob, d, blk
+
+
+def _check_serve_routing(prob, blk):
+    cfg = prob.cfg
+    ids, w = oracle.route_topk(prob.logits, cfg.top_k)
+    g = oracle.group_by_expert(ids, cfg.E)
+    assert np.array_equal(blk.topk_ids.cpu().numpy(), ids)
+    np.testing.assert_allclose(blk.topk_w.cpu().numpy(), w, rtol=4e-6, atol=1e-7)
+    assert np.array_equal(blk.counts.cpu().numpy(), g["counts"])
+    offsets = blk.offsets.cpu().numpy().astype(np.int64)
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), (g["counts"] + 127) // 128 * 128)
+    ros = blk.row_of_slot.cpu().numpy().astype(np.int64)
+    assert np.array_equal(ros - offsets[ids.reshape(-1)], g["rank"])
+    return ros
+
+
+@pytest.mark.parametrize("name", SERVE)
+def test_serve_forward_parity(name):
+    cfg = SMALL[name]
+    prob, _, blk = _serve(cfg, keep_gu=(name == "medium"))
+    ros = _check_serve_routing(prob, blk)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    fo = oracle.moe_forward(x, prob.logits, oracle_experts(prob), cfg.top_k, cfg.alpha)
+    slots = np.arange(cfg.N)
+    rows = ros[slots]
+    s = cfg.alpha / cfg.r
+    errs = {"y": rel_err(f64(blk.y), fo["y"])}
+    for key, buf, scale in [("act", blk.act, 1.0), ("p_gu", blk.p_gu, s), ("p_d", blk.p_d, s),
+                            ("yd", blk.y_perm, 1.0)]:
+        errs[key] = rel_err(f64(buf)[rows], np.stack([fo[key][f] for f in slots]) * scale)
+    assert np.array_equal(bits(blk.x_perm)[rows], prob.x[slots // cfg.top_k])
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, (bad, errs)
+
+
+def test_serve_decode_workload_full_and_gu_optional():
+    cfg = inputs.CONFIGS["decode"]
+    prob = inputs.make_problem(cfg)
+    _, _, a = _serve(cfg, prob, keep_gu=False)
+    _check_serve_routing(prob, a)
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    fo = oracle.moe_forward(x, prob.logits, oracle_experts(prob), cfg.top_k, cfg.alpha)
+    assert rel_err(f64(a.y), fo["y"]) <= TOL
+    assert np.all(bits(a.gu) == 0)  # never written without keep_gu
+    _, _, b = _serve(cfg, prob, keep_gu=True)
+    assert np.array_equal(bits(a.y), bits(b.y))  # gu is a by-product only
+    ros = b.row_of_slot.cpu().numpy().astype(np.int64)
+    gu = np.stack([fo["gu"][f] for f in range(cfg.N)])
+    assert rel_err(f64(b.gu)[ros], gu) <= TOL
+
+
+def test_serve_forward_cuda_graph_replay_is_bit_identical():
+    # the call allocates nothing and never synchronises: capture it once, replay it on new inputs
+    cfg = inputs.CONFIGS["decode"]
+    p1 = inputs.make_problem(cfg)
+    p2 = inputs.make_problem(cfg, data_rank=1)  # another batch over the same weights
+    d1, d2 = dv.upload(p1), dv.upload(p2)
+    blk = e4b.Block(dv.dims_of(cfg), cfg.T)
+    base, lora = d1.base(), d1.lora()
+    xs, ls = d1.x.clone(), d1.logits.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        blk.e4b_moe_serve_fwd(ls, xs, base, lora, keep_gu=False)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        blk.e4b_moe_serve_fwd(ls, xs, base, lora, keep_gu=False)
+    outs = []
+    for d in (d2, d1, d2):
+        xs.copy_(d.x)
+        ls.copy_(d.logits)
+        graph.replay()
+        torch.cuda.synchronize()
+        outs.append(bits(blk.y).copy())
+    eager = []
+    for d in (d2, d1):
+        blk.e4b_moe_serve_fwd(d.logits, d.x, base, lora, keep_gu=False)
+        torch.cuda.synchronize()
+        eager.append(bits(blk.y).copy())
+    assert blk.check_device_error() == e4b.E4B_OK
+    assert np.array_equal(outs[0], eager[0]) and np.array_equal(outs[2], eager[0])
+    assert np.array_equal(outs[1], eager[1]) and not np.array_equal(outs[0], outs[1])
+    del graph

@@ -115,6 +115,23 @@ def test_null_and_misaligned_pointers_refused(so):
     bwd_ok = e4b.BwdBuffers(*p[26:31])
     assert so.e4b_lora_wgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(fwd), ctypes.byref(bwd_ok),
                              p[33], None, p[35], p[36], ws, wsb, None) == e4b.E4B_ERR_INVALID_ARG
+    # serving forward: gu optional only for decode-sized batches; unaligned inputs; T == 0 launches nothing
+    nogu = e4b.FwdBuffers(p[19], p[20], None, p[22], p[23], p[24])
+    big = 33  # 66 routed slots > 16 * E
+    wsb_big = e4b.Sizes()
+    assert so.e4b_get_sizes(ctypes.byref(d), big, ctypes.byref(wsb_big)) == e4b.E4B_OK
+    assert wsb_big.workspace_bytes <= wsb
+    assert so.e4b_moe_serve_fwd(ctypes.byref(d), big, p[7], p[8], ctypes.byref(routing), ctypes.byref(base_ok),
+                                ctypes.byref(lora), ctypes.byref(nogu), p[25], ws, wsb,
+                                None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_moe_serve_fwd(ctypes.byref(d), T, p[7] + 4, p[8], ctypes.byref(routing), ctypes.byref(base_ok),
+                                ctypes.byref(lora), ctypes.byref(nogu), p[25], ws, wsb,
+                                None) == e4b.E4B_ERR_INVALID_ARG
+    assert so.e4b_moe_serve_fwd(ctypes.byref(d), T, p[7], p[8], ctypes.byref(routing), ctypes.byref(base),
+                                ctypes.byref(lora), ctypes.byref(nogu), p[25], ws, wsb,
+                                None) == e4b.E4B_ERR_INVALID_ARG  # base with a null member
+    assert so.e4b_moe_serve_fwd(ctypes.byref(d), 0, p[7], p[8], ctypes.byref(routing), ctypes.byref(base_ok),
+                                ctypes.byref(lora), ctypes.byref(nogu), p[25], ws, wsb, None) == e4b.E4B_OK
     # router backward: unaligned or missing tensors; dw optional; T == 0 launches nothing
     assert so.e4b_router_backward(ctypes.byref(d), T, ctypes.byref(routing), p[24] + 2, p[31], p[37], None,
                                   None) == e4b.E4B_ERR_INVALID_ARG
