@@ -317,8 +317,8 @@ def main():
         if fwd_only:  # routing + forward for inference, nothing kept for a backward
             blk.e4b_moe_serve_fwd(d.logits, d.x, base, lora, keep_gu=False)
             return
-        blk.e4b_route_permute(d.logits, d.x)
-        blk.e4b_grouped_nf4_lora_fwd(base, lora)
+        blk.e4b_route_permute(d.logits, d.x, gather=False)  # the forward gathers x with its first projection
+        blk.e4b_grouped_nf4_lora_fwd(base, lora, x=d.x)
         blk.e4b_grouped_nf4_lora_dgrad(base, lora, d.dY)
         blk.e4b_lora_wgrad()
         if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)

@@ -247,7 +247,8 @@ e4b_status e4b_route_permute(const e4b_moe_dims* dims, int32_t T, const float* l
   E4B_TRY(check_dims(dims, T));
   E4B_TRY(check_ws(dims, T, ws, ws_bytes));
   E4B_TRY(check_routing(routing));
-  if (!aligned16(logits) || !aligned16(x) || !aligned16(x_perm)) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(logits)) return E4B_ERR_INVALID_ARG;
+  if (x_perm != nullptr && (!aligned16(x) || !aligned16(x_perm))) return E4B_ERR_INVALID_ARG;
   if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
@@ -261,8 +262,9 @@ e4b_status e4b_route_permute(const e4b_moe_dims* dims, int32_t T, const float* l
 }
 
 e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e4b_routing* routing,
-                                    const e4b_nf4_experts* base, const e4b_lora* lora, const e4b_fwd_buffers* fwd,
-                                    e4b_bf16* y, void* ws, size_t ws_bytes, e4b_stream_t stream) {
+                                    const e4b_nf4_experts* base, const e4b_lora* lora, const e4b_bf16* x,
+                                    const e4b_fwd_buffers* fwd, e4b_bf16* y, void* ws, size_t ws_bytes,
+                                    e4b_stream_t stream) {
   E4B_TRY(check_dims(dims, T));
   E4B_TRY(check_ws(dims, T, ws, ws_bytes));
   E4B_TRY(check_routing(routing));
@@ -270,6 +272,7 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
   E4B_TRY(check_lora(lora));
   E4B_TRY(check_fwd(fwd));
   if (!aligned16(y)) return E4B_ERR_INVALID_ARG;
+  if (x != nullptr && !aligned16(x)) return E4B_ERR_INVALID_ARG;
   if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
@@ -302,13 +305,22 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
   g.err = err;
   g.timeout_ns = kDefaultTimeoutNs;
 
-  // p_gu = s * x_perm A_gu^T
+  // p_gu = s * x_perm A_gu^T; with x given, x_perm is gathered in the same pass
   lp.act_in = fwd->x_perm;
   lp.K = H;
   lp.w = lora->A_gu;
   lp.w_mn_major = false;
   lp.out = fwd->p_gu;
-  E4B_CUDA(launch_lora_proj(lp, sms, st));
+  if (x != nullptr) {
+    lp.gather_src = reinterpret_cast<const uint16_t*>(x);
+    lp.slot_of_row = routing->slot_of_row;
+    lp.gather_w = nullptr;
+    lp.k = k;
+    E4B_CUDA(launch_gather_proj(lp, sms, st));
+    lp.gather_src = nullptr;
+  } else {
+    E4B_CUDA(launch_lora_proj(lp, sms, st));
+  }
   // gu = W_gu x + p_gu B_gu^T ; act = silu(gate) * up
   g.mode = kFwdGateUp;
   g.nf4 = base->gate_up_nf4;
@@ -367,8 +379,8 @@ e4b_status e4b_moe_serve_fwd(const e4b_moe_dims* dims, int32_t T, const float* l
   if (!use_streaming_forward(N, dims->E)) {
     // a prefill-sized batch: the training forward (it writes gu, so gu is required)
     if (fwd->gu == nullptr) return E4B_ERR_INVALID_ARG;
-    E4B_TRY(e4b_route_permute(dims, T, logits, x, routing, fwd->x_perm, ws, ws_bytes, stream));
-    return e4b_grouped_nf4_lora_fwd(dims, T, routing, base, lora, fwd, y, ws, ws_bytes, stream);
+    E4B_TRY(e4b_route_permute(dims, T, logits, x, routing, nullptr, ws, ws_bytes, stream));
+    return e4b_grouped_nf4_lora_fwd(dims, T, routing, base, lora, x, fwd, y, ws, ws_bytes, stream);
   }
   if (T == 0) return E4B_OK;
   int sms = 0;
@@ -450,9 +462,6 @@ e4b_status e4b_grouped_nf4_lora_dgrad(const e4b_moe_dims* dims, int32_t T, const
   const float s = dims->alpha / (float)r;
   DeviceError* err = static_cast<DeviceError*>(ws);
 
-  // dyw[row] = w(slot) * dY[token]
-  E4B_CUDA(launch_gather_rows(dY, routing->slot_of_row, routing->tiles, routing->topk_w, H, k, rows_cap(N, E),
-                              bwd->dyw, sms, st));
   LoraProjHost lp{};
   lp.E = E;
   lp.r = r;
@@ -475,13 +484,17 @@ e4b_status e4b_grouped_nf4_lora_dgrad(const e4b_moe_dims* dims, int32_t T, const
   g.err = err;
   g.timeout_ns = kDefaultTimeoutNs;
 
-  // q_d = s * dyw B_d
+  // dyw[row] = w(slot) * dY[token] and q_d = s * dyw B_d, in one pass over the gathered rows
   lp.act_in = bwd->dyw;
   lp.K = H;
   lp.w = lora->B_d;
   lp.w_mn_major = true;
   lp.out = bwd->q_d;
-  E4B_CUDA(launch_lora_proj(lp, sms, st));
+  lp.gather_src = reinterpret_cast<const uint16_t*>(dY);
+  lp.slot_of_row = routing->slot_of_row;
+  lp.gather_w = routing->topk_w;
+  lp.k = k;
+  E4B_CUDA(launch_gather_proj(lp, sms, st));
   // dact = dyw W_d + q_d A_d ; dgu = SwiGLU backward(dact, gu)
   g.mode = kDgradDown;
   g.nf4 = base->down_nf4;

@@ -123,8 +123,15 @@ struct LoraProjHost {
   int64_t rows_cap, mt_cap;
   DeviceError* err;
   long long timeout_ns;
+  // launch_gather_proj only: act_in is written as act_in[row] = w(slot) * gather_src[token of row]
+  const uint16_t* gather_src;   // [T, K]
+  const int32_t* slot_of_row;   // [rows_cap]
+  const float* gather_w;        // [T*k] or nullptr
+  int k;
 };
 cudaError_t launch_lora_proj(const LoraProjHost& h, int num_sms, cudaStream_t stream);
+// The row gather fused with the projection: writes act_in (the gathered rows) and out.
+cudaError_t launch_gather_proj(const LoraProjHost& h, int num_sms, cudaStream_t stream);
 
 struct WgradHost {
   // four products dOut_g[e] = Act_g[e rows]^T * Low_g[e rows]

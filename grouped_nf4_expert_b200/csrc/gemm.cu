@@ -661,7 +661,8 @@ constexpr int B_BYTES = BK * E4B_MAX_RANK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 24 KB
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kTmemCols = 64;
+constexpr int kAccCols = 64;    // one accumulator: 128 rows x r_pad <= 64 fp32 columns
+constexpr int kTmemCols = 2 * kAccCols;  // two: a unit's MMAs overlap the previous unit's epilogue
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 }  // namespace lproj
 
@@ -684,19 +685,21 @@ __global__ void __launch_bounds__(lproj::kThreads)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* accfull = bars + 2 * STAGES;
-  uint64_t* accempty = accfull + 1;
-  uint64_t* drain = accfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 3);
-  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 4);
+  uint64_t* accfull = bars + 2 * STAGES;  // [2]
+  uint64_t* accempty = accfull + 2;       // [2]
+  uint64_t* drain = accfull + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 5);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 6);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accfull, 1);
-    mbar_init(accempty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
     mbar_init(drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -754,11 +757,13 @@ __global__ void __launch_bounds__(lproj::kThreads)
       const uint32_t idesc = make_idesc_bf16(BM, p.r_pad, false, W_MN);
       const uint32_t wswz = swz_for_row_bytes(2 * p.r_pad);
       int s = 0;
-      uint32_t ph = 0, tph = 0;
+      uint32_t ph = 0, ti = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        if (!(ok = mbar_wait(accempty, tph ^ 1, ctl, p.err, p.timeout_ns, 120))) break;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+        const uint32_t b = ti & 1, use = ti >> 1;
+        if (!(ok = mbar_wait(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 120))) break;
         tc_fence_after();
+        const uint32_t acc = tmem + b * kAccCols;
         for (int kc = 0; kc < kchunks; ++kc) {
           if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 121))) break;
           tc_fence_after();
@@ -768,7 +773,7 @@ __global__ void __launch_bounds__(lproj::kThreads)
             const uint64_t ad = make_sdesc(a0 + 32 * kk, 16, 1024, kSw128);
             const uint64_t bd = W_MN ? make_sdesc(b0 + 32 * p.r_pad * kk, b_bytes, 16 * p.r_pad, wswz)
                                      : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
-            umma_bf16(tmem, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(acc, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
           if (++s == STAGES) {
@@ -777,8 +782,7 @@ __global__ void __launch_bounds__(lproj::kThreads)
           }
         }
         if (!ok) break;
-        umma_commit(accfull);
-        tph ^= 1;
+        umma_commit(&accfull[b]);
       }
       umma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
@@ -787,12 +791,13 @@ __global__ void __launch_bounds__(lproj::kThreads)
     }
   } else {
     const int q = ((warp & 3) << 5) | lane;  // TMEM lane of this thread
-    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint32_t tph = 0;
+    uint32_t ti = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+      const uint32_t b = ti & 1, use = ti >> 1;
+      const uint32_t tl = tmem + b * kAccCols + ((uint32_t)(32 * (warp & 3)) << 16);
       const size_t row = (size_t)p.tiles[kTileHeader + 2 * u + 1] + q;
-      ok = mbar_wait(accfull, tph, ctl, p.err, p.timeout_ns, 130);
+      ok = mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 130);
       ok = __all_sync(kFull, ok);
       if (!ok) break;
       tc_fence_after();
@@ -809,13 +814,299 @@ __global__ void __launch_bounds__(lproj::kThreads)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty);
-      tph ^= 1;
+      if (lane == 0) mbar_arrive(&accempty[b]);
     }
   }
   __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the CTA barrier
   __syncthreads();
   if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// =============================================================================
+// Row gather fused with the LoRA projection:
+//   dst[row] = bf16(w(slot) * src[token of row])  (zero for padding rows)
+//   out[row] = bf16(scale * dst[row] . W_e)       over K, r outputs
+// The gathered 128-row x 64-column tile is built in shared memory (in the
+// UMMA's 128B-swizzled K-major layout) by eight producer warps, each loading
+// four rows' 128-byte pieces per instruction (8 lanes per row, coalesced);
+// the tensor core reads it as the A operand of the projection and a TMA bulk
+// store writes the same tile to dst, so the permuted rows are read from HBM
+// by no later projection.
+// =============================================================================
+namespace gproj {
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BK * E4B_MAX_RANK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 24 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+// warps 0-7 producers (16 tile rows each), 8 W loader, 9 UMMA issuer + TMEM owner, 10 tile storer,
+// 11-14 epilogue
+constexpr int kProdWarps = 8;
+constexpr int kWLoadWarp = 8, kIssueWarp = 9, kStoreWarp = 10, kEpiWarp0 = 11;
+constexpr int kThreads = 15 * 32;
+constexpr int kAccCols = 64;
+constexpr int kTmemCols = 2 * kAccCols;
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+}  // namespace gproj
+
+struct GatherProjParams {
+  const uint16_t* src;        // [T, K] token rows
+  const int32_t* slot_of_row;
+  const float* scale_w;       // [T*k] per-slot factor, or nullptr
+  const int32_t* tiles;
+  uint16_t* out;              // [rows_cap, r]
+  DeviceError* err;
+  long long timeout_ns;
+  float scale;
+  int K, r, r_pad, k;
+};
+
+template <bool W_MN>
+__global__ void __launch_bounds__(gproj::kThreads, 2)  // two CTAs per SM: <= 68 registers
+    gather_proj_kernel(const __grid_constant__ CUtensorMap map_dst, const __grid_constant__ CUtensorMap map_w,
+                       const GatherProjParams p) {
+  using namespace gproj;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = align1024(smem_dyn);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;                 // [STAGES] the producer warps + the W bytes
+  uint64_t* empty = bars + STAGES;       // [STAGES] the UMMAs read the slot
+  uint64_t* stored = bars + 2 * STAGES;  // [STAGES] the bulk store read the tile
+  uint64_t* accfull = bars + 3 * STAGES;  // [2]
+  uint64_t* accempty = accfull + 2;       // [2]
+  uint64_t* drain = accfull + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 5);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 6);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], kProdWarps + 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&stored[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kIssueWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_units = p.tiles[0];
+  const int rows_used = p.tiles[1];
+  const int kchunks = p.K / BK;
+  const uint32_t b_bytes = BK * p.r_pad * 2;
+
+  if (warp < kProdWarps) {
+    // ------------------------------------------------ producers: warp w builds rows 16w..16w+15; per
+    // instruction i lane l moves 16-byte piece l%8 of row 16w + 4i + l/8
+    const int c = lane & 7;
+    uint32_t s = 0, ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int row0 = p.tiles[kTileHeader + 2 * u + 1];
+      const uint4* src[4];
+      float w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = row0 + 16 * warp + 4 * i + (lane >> 3);
+        const int slot = (row < rows_used) ? __ldg(p.slot_of_row + row) : -1;
+        src[i] = (slot >= 0) ? reinterpret_cast<const uint4*>(p.src + (size_t)(slot / p.k) * p.K) + c : nullptr;
+        w[i] = (slot >= 0 && p.scale_w != nullptr) ? __ldg(p.scale_w + slot) : 1.0f;
+      }
+      // Two k-chunks per round: all eight loads are issued before the round's
+      // proxy fence, which waits for this thread's outstanding memory accesses.
+      for (int kc = 0; kc < kchunks; kc += 2) {
+        const bool two = kc + 1 < kchunks;
+        uint4 v[2][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[0][i] = src[i] ? __ldg(src[i] + 8 * kc) : make_uint4(0u, 0u, 0u, 0u);
+          v[1][i] = (src[i] && two) ? __ldg(src[i] + 8 * (kc + 1)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t slots[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !two) break;
+          // warp-uniform waits: every lane leaves the loop together on a timeout
+          if (!(ok = __all_sync(kFull, mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 60)))) break;
+          if (!(ok = __all_sync(kFull, mbar_wait(&stored[s], ph ^ 1, ctl, p.err, p.timeout_ns, 61)))) break;
+          uint8_t* tile = smem + s * STAGE_BYTES;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int q = 16 * warp + 4 * i + (lane >> 3);  // tile row
+            uint4 x = v[h][i];
+            if (p.scale_w != nullptr) {
+              uint32_t* xw = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                xw[e] = pack_bf16x2(w[i] * bf16lo_to_f32(xw[e]), w[i] * bf16hi_to_f32(xw[e]));
+            }
+            *reinterpret_cast<uint4*>(tile + (q >> 3) * 1024 + (q & 7) * 128 + ((c ^ (q & 7)) << 4)) = x;
+          }
+          slots[h] = s;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        fence_proxy_async_smem();  // visible to the tensor core and the bulk store
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full[slots[0]]);
+          if (two) mbar_arrive(&full[slots[1]]);
+        }
+      }
+    }
+  } else if (warp == kWLoadWarp) {
+    // ------------------------------------------------ LoRA factor chunks (TMA, one lane)
+    if (lane == 0) {
+      tma_prefetch_desc(&map_w);
+      uint32_t s = 0, ph = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int e = p.tiles[kTileHeader + 2 * u];
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 62))) break;
+          uint8_t* st = smem + s * STAGE_BYTES + A_BYTES;
+          mbar_arrive_expect_tx(&full[s], b_bytes);
+          if (W_MN)
+            tma_load_3d(st, &map_w, &full[s], 0, kc * BK, e);
+          else
+            tma_load_3d(st, &map_w, &full[s], kc * BK, 0, e);
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {  // let issued copies land before shared memory goes away
+        for (int i = 0; i < STAGES; ++i)
+          if (issued & (1u << i)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[i], (last_par >> i) & 1u) &&
+                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+            }
+          }
+      }
+    }
+  } else if (warp == kIssueWarp) {
+    // ------------------------------------------------ UMMA issuer (one lane)
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(BM, p.r_pad, false, W_MN);
+      const uint32_t wswz = swz_for_row_bytes(2 * p.r_pad);
+      uint32_t s = 0, ph = 0, ti = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+        const uint32_t b = ti & 1, use = ti >> 1;
+        if (!(ok = mbar_wait(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 63))) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + b * kAccCols;
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 64))) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES), b0 = a0 + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = make_sdesc(a0 + 32 * kk, 16, 1024, kSw128);
+            const uint64_t bd = W_MN ? make_sdesc(b0 + 32 * p.r_pad * kk, b_bytes, 16 * p.r_pad, wswz)
+                                     : make_sdesc(b0 + 32 * kk, 16, 1024, kSw128);
+            umma_bf16(acc, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&accfull[b]);
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+      }
+    }
+  } else if (warp == kStoreWarp) {
+    // ------------------------------------------------ gathered tiles -> dst (TMA bulk stores, one lane)
+    // A slot is handed back once its store's shared-memory reads are done,
+    // checked when the store kStoreLag chunks later has been issued (up to
+    // kStoreLag + 1 stores in flight; kStoreLag < STAGES).
+    constexpr int kStoreLag = 2;
+    if (lane == 0) {
+      tma_prefetch_desc(&map_dst);
+      uint32_t s = 0, ph = 0, pend[kStoreLag];
+      int n_pend = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int row0 = p.tiles[kTileHeader + 2 * u + 1];
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 65))) break;
+          tma_store_2d(&map_dst, smem_u32(smem + s * STAGE_BYTES), kc * BK, row0);
+          bulk_commit();
+          if (n_pend == kStoreLag) {
+            bulk_wait_read<kStoreLag>();  // the oldest pending store has read its slot
+            mbar_arrive(&stored[pend[0]]);
+#pragma unroll
+            for (int i = 0; i + 1 < kStoreLag; ++i) pend[i] = pend[i + 1];
+            --n_pend;
+          }
+          pend[n_pend++] = s;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      bulk_wait<0>();  // reads and writes of every store done
+      for (int i = 0; i < n_pend; ++i) mbar_arrive(&stored[pend[i]]);
+    }
+  } else {
+    // ------------------------------------------------ epilogue: TMEM -> bf16(scale * acc) rows
+    const int q = ((warp & 3) << 5) | lane;  // TMEM lane of this thread
+    uint32_t ti = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
+      const uint32_t b = ti & 1, use = ti >> 1;
+      const uint32_t tl = tmem + b * kAccCols + ((uint32_t)(32 * (warp & 3)) << 16);
+      const size_t row = (size_t)p.tiles[kTileHeader + 2 * u + 1] + q;
+      ok = mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 66);
+      ok = __all_sync(kFull, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int j = 0; j < p.r_pad; j += 16) {
+        float v[16];
+        tmem_ld16(tl + j, v);
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(p.scale * v[2 * i], p.scale * v[2 * i + 1]);
+        uint4* d = reinterpret_cast<uint4*>(p.out + row * p.r + j);
+        if (j < p.r) d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (j + 8 < p.r) d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[b]);
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if (warp == kIssueWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -831,7 +1122,8 @@ constexpr int B_BYTES = BK * E4B_MAX_RANK * 2;  // 64 rows x r_pad, MN-major
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
 constexpr int kThreads = 192;
-constexpr int kTmemCols = 64;
+constexpr int kAccCols = 64;             // one accumulator: 128 features x r_pad <= 64 fp32 columns
+constexpr int kTmemCols = 2 * kAccCols;  // two: a unit's MMAs overlap the previous unit's epilogue
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 }  // namespace wg
 
@@ -883,19 +1175,21 @@ __global__ void __launch_bounds__(wg::kThreads)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* accfull = bars + 2 * STAGES;
-  uint64_t* accempty = accfull + 1;
-  uint64_t* drain = accfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 3);
-  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 4);
+  uint64_t* accfull = bars + 2 * STAGES;  // [2]
+  uint64_t* accempty = accfull + 2;       // [2]
+  uint64_t* drain = accfull + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 5);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 6);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accfull, 1);
-    mbar_init(accempty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
     mbar_init(drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -951,12 +1245,14 @@ __global__ void __launch_bounds__(wg::kThreads)
       const uint32_t idesc = make_idesc_bf16(BM, p.r_pad, true, true);
       const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
       int s = 0;
-      uint32_t ph = 0, tph = 0;
+      uint32_t ph = 0, ti = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
         const WgradUnit w = wgrad_unit(p, u);
-        if (!(ok = mbar_wait(accempty, tph ^ 1, ctl, p.err, p.timeout_ns, 220))) break;
+        const uint32_t b = ti & 1, use = ti >> 1;
+        if (!(ok = mbar_wait(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 220))) break;
         tc_fence_after();
+        const uint32_t acc = tmem + b * kAccCols;
         for (int kc = 0; kc < w.nk; ++kc) {
           if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 221))) break;
           tc_fence_after();
@@ -965,7 +1261,7 @@ __global__ void __launch_bounds__(wg::kThreads)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = make_sdesc(a0 + 2048 * kk, A_BYTES / 2, 1024, kSw128);
             const uint64_t bd = make_sdesc(b0 + 32 * p.r_pad * kk, b_bytes, 16 * p.r_pad, lswz);
-            umma_bf16(tmem, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(acc, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
           if (++s == STAGES) {
@@ -974,8 +1270,7 @@ __global__ void __launch_bounds__(wg::kThreads)
           }
         }
         if (!ok) break;
-        umma_commit(accfull);
-        tph ^= 1;
+        umma_commit(&accfull[b]);
       }
       umma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
@@ -984,12 +1279,13 @@ __global__ void __launch_bounds__(wg::kThreads)
     }
   } else {
     const int q = ((warp & 3) << 5) | lane;
-    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint32_t tph = 0;
+    uint32_t ti = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ti) {
       const WgradUnit w = wgrad_unit(p, u);
-      ok = mbar_wait(accfull, tph, ctl, p.err, p.timeout_ns, 230);
+      const uint32_t b = ti & 1, use = ti >> 1;
+      const uint32_t tl = tmem + b * kAccCols + ((uint32_t)(32 * (warp & 3)) << 16);
+      ok = mbar_wait(&accfull[b], use & 1, ctl, p.err, p.timeout_ns, 230);
       ok = __all_sync(kFull, ok);
       if (!ok) break;
       tc_fence_after();
@@ -1026,8 +1322,7 @@ __global__ void __launch_bounds__(wg::kThreads)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty);
-      tph ^= 1;
+      if (lane == 0) mbar_arrive(&accempty[b]);
     }
   }
   __syncwarp();  // reconverge each warp (its lane 0 ran a role loop) before the CTA barrier
@@ -1183,6 +1478,43 @@ cudaError_t launch_lora_proj(const LoraProjHost& h, int num_sms, cudaStream_t st
   } else {
     if ((err = set_smem(lora_proj_kernel<false>, smem)) != cudaSuccess) return err;
     lora_proj_kernel<false><<<grid, lproj::kThreads, smem, stream>>>(mact, mw, p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_proj(const LoraProjHost& h, int num_sms, cudaStream_t stream) {
+  CUtensorMap mdst, mw;
+  cudaError_t err;
+  if ((err = map_bf16_2d(&mdst, h.act_in, h.K, h.rows_cap, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+    return err;
+  if (h.w_mn_major)
+    err = map_bf16_3d(&mw, h.w, h.r, h.K, h.E, h.r_pad, 64, swizzle_for_bytes(2 * h.r_pad));
+  else
+    err = map_bf16_3d(&mw, h.w, h.K, h.r, h.E, 64, h.r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (err != cudaSuccess) return err;
+  GatherProjParams p;
+  p.src = h.gather_src;
+  p.slot_of_row = h.slot_of_row;
+  p.scale_w = h.gather_w;
+  p.tiles = h.tiles;
+  p.out = h.out;
+  p.err = h.err;
+  p.timeout_ns = h.timeout_ns;
+  p.scale = h.scale;
+  p.K = h.K;
+  p.r = h.r;
+  p.r_pad = h.r_pad;
+  p.k = h.k;
+  const int64_t cap = (int64_t)num_sms * 2;
+  const int grid = (int)(h.mt_cap < cap ? h.mt_cap : cap);
+  const int smem = gproj::SMEM_BYTES;
+  LaunchScope scope(h.gather_w ? "gather_proj_dyw" : "gather_proj_x", stream);
+  if (h.w_mn_major) {
+    if ((err = set_smem(gather_proj_kernel<true>, smem)) != cudaSuccess) return err;
+    gather_proj_kernel<true><<<grid, gproj::kThreads, smem, stream>>>(mdst, mw, p);
+  } else {
+    if ((err = set_smem(gather_proj_kernel<false>, smem)) != cudaSuccess) return err;
+    gather_proj_kernel<false><<<grid, gproj::kThreads, smem, stream>>>(mdst, mw, p);
   }
   return cudaGetLastError();
 }

@@ -81,7 +81,7 @@ _SIGNATURES = {
     "e4b_route_permute": (c_i32, [ctypes.POINTER(MoeDims), c_i32, c_vp, c_vp, ctypes.POINTER(Routing), c_vp,
                                   c_vp, c_sz, c_vp]),
     "e4b_grouped_nf4_lora_fwd": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
-                                         ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora),
+                                         ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora), c_vp,
                                          ctypes.POINTER(FwdBuffers), c_vp, c_vp, c_sz, c_vp]),
     "e4b_grouped_nf4_lora_dgrad": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
                                            ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora),
@@ -254,16 +254,18 @@ class Block:
         self._bwd = BwdBuffers(*(t.data_ptr() for t in (self.dyw, self.q_d, self.dgu, self.q_gu, self.dx_perm)))
 
     # -- the four hot-path calls -------------------------------------------------
-    def e4b_route_permute(self, logits, x, stream=None):
+    def e4b_route_permute(self, logits, x, gather=True, stream=None):
+        """Routing tables; with ``gather`` also ``x_perm`` (else the forward gathers, given ``x``)."""
         _check(lib().e4b_route_permute(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
-                                       ctypes.byref(self._routing), _ptr(self.x_perm), _ptr(self.ws),
-                                       self.ws.numel(), _stream(stream)), "e4b_route_permute")
+                                       ctypes.byref(self._routing), _ptr(self.x_perm) if gather else None,
+                                       _ptr(self.ws), self.ws.numel(), _stream(stream)), "e4b_route_permute")
 
-    def e4b_grouped_nf4_lora_fwd(self, base: Nf4Experts, lora: Lora, stream=None):
+    def e4b_grouped_nf4_lora_fwd(self, base: Nf4Experts, lora: Lora, x=None, stream=None):
+        """Forward; with ``x`` the call also writes ``x_perm`` (fused with the first projection)."""
         _check(lib().e4b_grouped_nf4_lora_fwd(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
-                                              ctypes.byref(base), ctypes.byref(lora), ctypes.byref(self._fwd),
-                                              _ptr(self.y), _ptr(self.ws), self.ws.numel(), _stream(stream)),
-               "e4b_grouped_nf4_lora_fwd")
+                                              ctypes.byref(base), ctypes.byref(lora), _ptr(x),
+                                              ctypes.byref(self._fwd), _ptr(self.y), _ptr(self.ws),
+                                              self.ws.numel(), _stream(stream)), "e4b_grouped_nf4_lora_fwd")
 
     def e4b_grouped_nf4_lora_dgrad(self, base: Nf4Experts, lora: Lora, dY, stream=None):
         _check(lib().e4b_grouped_nf4_lora_dgrad(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),

@@ -162,7 +162,10 @@ e4b_status e4b_check_device_error(const void *ws, e4b_stream_t stream);
  * expert id, NaN lowest), the softmax over them, the stable grouping of the
  * T*top_k slots by expert (ascending flat slot within an expert), the device
  * work list, and x_perm[row] = x[token of row] (zero for padding rows).
- * logits: float32 [T, E]; x: bf16 [T, H]; x_perm: [rows_cap, H].
+ * logits: float32 [T, E]; x: bf16 [T, H]; x_perm: [rows_cap, H].  With
+ * x_perm NULL only the routing tables are written (x is not read and may be
+ * NULL): the permutation is then left to e4b_grouped_nf4_lora_fwd, which
+ * gathers the rows in the same pass as its first LoRA projection.
  * Deterministic: identical inputs give identical bits.
  * Pages: same page, section "Which project solves it" (grouped execution);
  * the router's logits are inputs (router frozen, section "The abstraction
@@ -193,14 +196,17 @@ e4b_status e4b_route_permute_noalloc(const e4b_moe_dims *dims, int32_t T, const 
 
 /* Forward: p_gu, gu/act (SiLU-gated epilogue), p_d, y_perm, then the
  * router-weighted un-permute y[t] = sum_j w[t,j] * y_perm[row(t,j)] (fp32
- * sum in j order, rounded once to bf16).  fwd->x_perm must hold what
- * e4b_route_permute wrote.  y: bf16 [T, H].
+ * sum in j order, rounded once to bf16).  y: bf16 [T, H].  With x (bf16
+ * [T, H]) given, the call writes fwd->x_perm itself (x_perm[row] = x[token of
+ * row], zero for padding rows, as e4b_route_permute would) in the same pass
+ * as p_gu, so the permuted rows are not read back from memory; with x NULL,
+ * fwd->x_perm must hold what e4b_route_permute wrote.
  * Pages: section "The abstraction that fails" (pre-activation delta) and
  * section "Why it happens" (the LoRA term); METADATA "The package family". */
 e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims *dims, int32_t T,
                                     const e4b_routing *routing, const e4b_nf4_experts *base,
-                                    const e4b_lora *lora, const e4b_fwd_buffers *fwd, e4b_bf16 *y,
-                                    void *ws, size_t ws_bytes, e4b_stream_t stream);
+                                    const e4b_lora *lora, const e4b_bf16 *x, const e4b_fwd_buffers *fwd,
+                                    e4b_bf16 *y, void *ws, size_t ws_bytes, e4b_stream_t stream);
 
 /* Serving forward: routing and the forward in one call, for inference
  * (decode-sized batches above all): y = the block's output for x (bf16

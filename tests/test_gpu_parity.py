@@ -72,13 +72,15 @@ def oracle_experts(prob):
                           f(prob.A_gu), f(prob.B_gu), f(prob.A_d), f(prob.B_d))
 
 
-def run(cfg, fwd=True, dgrad=True, wgrad=True, prob=None):
+def run(cfg, fwd=True, dgrad=True, wgrad=True, prob=None, fused_gather=True):
+    # fused_gather: x_perm is written by the forward (with its first projection), else by the routing call
     prob = prob if prob is not None else inputs.make_problem(cfg)
     d = dv.upload(prob)
     blk = e4b.Block(dv.dims_of(cfg), cfg.T)
-    blk.e4b_route_permute(d.logits, d.x)
+    fused = fused_gather and fwd
+    blk.e4b_route_permute(d.logits, d.x, gather=not fused)
     if fwd:
-        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora())
+        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora(), x=d.x if fused else None)
     if dgrad:
         blk.e4b_grouped_nf4_lora_dgrad(d.base(), d.lora(), d.dY)
     if wgrad:
@@ -257,10 +259,10 @@ def test_routing_ties_and_deterministic():
 
 # --------------------------------------------------------------------- full block, small sizes
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_block_parity_small(name):
+@pytest.mark.parametrize("name,fused", [(n, True) for n in SMALL] + [("medium", False), ("stream_r24", False)])
+def test_block_parity_small(name, fused):
     cfg = SMALL[name]
-    prob, _, blk = run(cfg)
+    prob, _, blk = run(cfg, fused_gather=fused)
     ros = check_routing(prob, blk)
     ex = oracle_experts(prob)
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
@@ -408,8 +410,8 @@ def test_repeated_full_size_runs_are_bit_identical(name):
     backward = "dgrad" in cfg.passes
     ref = None
     for _ in range(6 if name == "finegrained" else 3):
-        blk.e4b_route_permute(d.logits, d.x)
-        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora())
+        blk.e4b_route_permute(d.logits, d.x, gather=False)
+        blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora(), x=d.x)
         if backward:
             blk.e4b_grouped_nf4_lora_dgrad(d.base(), d.lora(), d.dY)
             blk.e4b_lora_wgrad()

@@ -105,8 +105,15 @@ def test_null_and_misaligned_pointers_refused(so):
     lora = e4b.Lora(*p[15:19])
     fwd = e4b.FwdBuffers(*p[19:25])
     assert so.e4b_grouped_nf4_lora_fwd(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(base),
-                                       ctypes.byref(lora), ctypes.byref(fwd), p[25], ws, wsb,
+                                       ctypes.byref(lora), None, ctypes.byref(fwd), p[25], ws, wsb,
                                        None) == e4b.E4B_ERR_INVALID_ARG
+    # a misaligned x to gather from
+    assert so.e4b_grouped_nf4_lora_fwd(ctypes.byref(d), T, ctypes.byref(routing),
+                                       ctypes.byref(e4b.Nf4Experts(*p[11:15])), ctypes.byref(lora), p[8] + 2,
+                                       ctypes.byref(fwd), p[25], ws, wsb, None) == e4b.E4B_ERR_INVALID_ARG
+    # routing tables only (no x_perm): x is not needed; nothing to do for T == 0
+    assert so.e4b_route_permute(ctypes.byref(d), 0, p[7], None, ctypes.byref(routing), None, ws, wsb,
+                                None) == e4b.E4B_OK
     bwd = e4b.BwdBuffers(*p[26:30], p[30] + 8)
     base_ok = e4b.Nf4Experts(*p[11:15])
     assert so.e4b_grouped_nf4_lora_dgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(base_ok),
