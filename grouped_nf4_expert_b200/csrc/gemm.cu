@@ -829,12 +829,13 @@ __global__ void __launch_bounds__(lproj::kThreads)
 // Row gather fused with the LoRA projection:
 //   dst[row] = bf16(w(slot) * src[token of row])  (zero for padding rows)
 //   out[row] = bf16(scale * dst[row] . W_e)       over K, r outputs
-// The gathered 128-row x 64-column tile is built in shared memory (in the
-// UMMA's 128B-swizzled K-major layout) by eight producer warps, each loading
-// four rows' 128-byte pieces per instruction (8 lanes per row, coalesced);
-// the tensor core reads it as the A operand of the projection and a TMA bulk
-// store writes the same tile to dst, so the permuted rows are read from HBM
-// by no later projection.
+// The gathered 128-row x 64-column tile is copied into shared memory (in the
+// UMMA's 128B-swizzled K-major layout) by four loader warps with cp.async
+// (8 lanes per 128-byte row piece, coalesced; zero-filled for padding rows),
+// as many k-chunks ahead as there are free slots; for a weighted gather four
+// more warps scale the landed tile in place.  The tensor core reads the tile
+// as the A operand of the projection and a TMA bulk store writes the same tile
+// to dst, so the permuted rows are read from HBM by no later projection.
 // =============================================================================
 namespace gproj {
 constexpr int BM = 128, BK = 64, STAGES = 4;
@@ -842,9 +843,9 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BK * E4B_MAX_RANK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 24 KB
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
-// warps 0-7 producers (16 tile rows each), 8 W loader, 9 UMMA issuer + TMEM owner, 10 tile storer,
-// 11-14 epilogue
-constexpr int kProdWarps = 8;
+// warps 0-3 row loaders (32 tile rows each), 4-7 scalers (weighted gather only), 8 W loader,
+// 9 UMMA issuer + TMEM owner, 10 tile storer, 11-14 epilogue
+constexpr int kLoadWarps = 4, kScaleWarp0 = 4, kScaleWarps = 4;
 constexpr int kWLoadWarp = 8, kIssueWarp = 9, kStoreWarp = 10, kEpiWarp0 = 11;
 constexpr int kThreads = 15 * 32;
 constexpr int kAccCols = 64;
@@ -865,27 +866,31 @@ struct GatherProjParams {
 };
 
 template <bool W_MN>
-__global__ void __launch_bounds__(gproj::kThreads, 2)  // two CTAs per SM: <= 68 registers
+__global__ void __launch_bounds__(gproj::kThreads, 2)  // two CTAs per SM: <= 64 registers
     gather_proj_kernel(const __grid_constant__ CUtensorMap map_dst, const __grid_constant__ CUtensorMap map_w,
                        const GatherProjParams p) {
   using namespace gproj;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align1024(smem_dyn);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* full = bars;                 // [STAGES] the producer warps + the W bytes
+  uint64_t* full = bars;                 // [STAGES] tile complete (+ the W bytes)
   uint64_t* empty = bars + STAGES;       // [STAGES] the UMMAs read the slot
   uint64_t* stored = bars + 2 * STAGES;  // [STAGES] the bulk store read the tile
-  uint64_t* accfull = bars + 3 * STAGES;  // [2]
+  uint64_t* landed = bars + 3 * STAGES;  // [STAGES] (weighted gather) the row copies landed
+  uint64_t* accfull = bars + 4 * STAGES;  // [2]
   uint64_t* accempty = accfull + 2;       // [2]
   uint64_t* drain = accfull + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 5);
   CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 6);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    const bool scaled = p.scale_w != nullptr;
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full[i], kProdWarps + 1);
+      // each loader thread's cp.async arrival (.noinc) counts once; the W loader's expect_tx once
+      mbar_init(&full[i], (scaled ? kScaleWarps : kLoadWarps * 32) + 1);
       mbar_init(&empty[i], 1);
       mbar_init(&stored[i], 1);
+      mbar_init(&landed[i], kLoadWarps * 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
@@ -908,65 +913,78 @@ __global__ void __launch_bounds__(gproj::kThreads, 2)  // two CTAs per SM: <= 68
   const int kchunks = p.K / BK;
   const uint32_t b_bytes = BK * p.r_pad * 2;
 
-  if (warp < kProdWarps) {
-    // ------------------------------------------------ producers: warp w builds rows 16w..16w+15; per
-    // instruction i lane l moves 16-byte piece l%8 of row 16w + 4i + l/8
+  if (warp < kLoadWarps) {
+    // ------------------------------------------------ row loaders: warp w copies rows 32w..32w+31; per
+    // instruction i lane l copies 16-byte piece l%8 of row 32w + 4i + l/8 (cp.async, no registers held)
     const int c = lane & 7;
+    uint64_t* done = (p.scale_w != nullptr) ? landed : full;
     uint32_t s = 0, ph = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const int row0 = p.tiles[kTileHeader + 2 * u + 1];
-      const uint4* src[4];
-      float w[4];
+      const uint16_t* src[8];
+      uint32_t nbytes[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = row0 + 16 * warp + 4 * i + (lane >> 3);
+      for (int i = 0; i < 8; ++i) {
+        const int row = row0 + 32 * warp + 4 * i + (lane >> 3);
         const int slot = (row < rows_used) ? __ldg(p.slot_of_row + row) : -1;
-        src[i] = (slot >= 0) ? reinterpret_cast<const uint4*>(p.src + (size_t)(slot / p.k) * p.K) + c : nullptr;
-        w[i] = (slot >= 0 && p.scale_w != nullptr) ? __ldg(p.scale_w + slot) : 1.0f;
+        src[i] = p.src + ((slot >= 0) ? (size_t)(slot / p.k) * p.K : 0) + 8 * c;
+        nbytes[i] = (slot >= 0) ? 16u : 0u;  // padding rows: zero fill, nothing read
       }
-      // Two k-chunks per round: all eight loads are issued before the round's
-      // proxy fence, which waits for this thread's outstanding memory accesses.
-      for (int kc = 0; kc < kchunks; kc += 2) {
-        const bool two = kc + 1 < kchunks;
-        uint4 v[2][4];
+      for (int kc = 0; kc < kchunks; ++kc) {
+        // warp-uniform waits: every lane leaves the loop together on a timeout
+        if (!(ok = __all_sync(kFull, mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 60)))) break;
+        if (!(ok = __all_sync(kFull, mbar_wait(&stored[s], ph ^ 1, ctl, p.err, p.timeout_ns, 61)))) break;
+        uint8_t* tile = smem + s * STAGE_BYTES;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[0][i] = src[i] ? __ldg(src[i] + 8 * kc) : make_uint4(0u, 0u, 0u, 0u);
-          v[1][i] = (src[i] && two) ? __ldg(src[i] + 8 * (kc + 1)) : make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < 8; ++i) {
+          const int q = 32 * warp + 4 * i + (lane >> 3);  // tile row
+          cp_async_16_zfill(tile + (q >> 3) * 1024 + (q & 7) * 128 + ((c ^ (q & 7)) << 4), src[i] + kc * BK,
+                            nbytes[i]);
         }
-        uint32_t slots[2];
+        cp_async_arrive_noinc(&done[s]);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+  } else if (warp < kScaleWarp0 + kScaleWarps) {
+    // ------------------------------------------------ scalers (weighted gather): row *= w(slot) in place
+    if (p.scale_w != nullptr) {
+      const int sw = warp - kScaleWarp0, c = lane & 7;
+      uint32_t s = 0, ph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int row0 = p.tiles[kTileHeader + 2 * u + 1];
+        float w[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h == 1 && !two) break;
-          // warp-uniform waits: every lane leaves the loop together on a timeout
-          if (!(ok = __all_sync(kFull, mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 60)))) break;
-          if (!(ok = __all_sync(kFull, mbar_wait(&stored[s], ph ^ 1, ctl, p.err, p.timeout_ns, 61)))) break;
+        for (int i = 0; i < 8; ++i) {
+          const int row = row0 + 32 * sw + 4 * i + (lane >> 3);
+          const int slot = (row < rows_used) ? __ldg(p.slot_of_row + row) : -1;
+          w[i] = (slot >= 0) ? __ldg(p.scale_w + slot) : 0.0f;
+        }
+        for (int kc = 0; kc < kchunks; ++kc) {
+          if (!(ok = __all_sync(kFull, mbar_wait(&landed[s], ph, ctl, p.err, p.timeout_ns, 67)))) break;
           uint8_t* tile = smem + s * STAGE_BYTES;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int q = 16 * warp + 4 * i + (lane >> 3);  // tile row
-            uint4 x = v[h][i];
-            if (p.scale_w != nullptr) {
-              uint32_t* xw = reinterpret_cast<uint32_t*>(&x);
+          for (int i = 0; i < 8; ++i) {
+            const int q = 32 * sw + 4 * i + (lane >> 3);
+            uint4* pc = reinterpret_cast<uint4*>(tile + (q >> 3) * 1024 + (q & 7) * 128 + ((c ^ (q & 7)) << 4));
+            uint4 x = *pc;
+            uint32_t* xw = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                xw[e] = pack_bf16x2(w[i] * bf16lo_to_f32(xw[e]), w[i] * bf16hi_to_f32(xw[e]));
-            }
-            *reinterpret_cast<uint4*>(tile + (q >> 3) * 1024 + (q & 7) * 128 + ((c ^ (q & 7)) << 4)) = x;
+            for (int e = 0; e < 4; ++e)
+              xw[e] = pack_bf16x2(w[i] * bf16lo_to_f32(xw[e]), w[i] * bf16hi_to_f32(xw[e]));
+            *pc = x;
           }
-          slots[h] = s;
+          fence_proxy_async_smem();  // visible to the tensor core and the bulk store
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[s]);
           if (++s == STAGES) {
             s = 0;
             ph ^= 1;
           }
-        }
-        if (!ok) break;
-        fence_proxy_async_smem();  // visible to the tensor core and the bulk store
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&full[slots[0]]);
-          if (two) mbar_arrive(&full[slots[1]]);
         }
       }
     }
@@ -1056,6 +1074,7 @@ __global__ void __launch_bounds__(gproj::kThreads, 2)  // two CTAs per SM: <= 68
         const int row0 = p.tiles[kTileHeader + 2 * u + 1];
         for (int kc = 0; kc < kchunks; ++kc) {
           if (!(ok = mbar_wait(&full[s], ph, ctl, p.err, p.timeout_ns, 65))) break;
+          fence_proxy_async_smem();
           tma_store_2d(&map_dst, smem_u32(smem + s * STAGE_BYTES), kc * BK, row0);
           bulk_commit();
           if (n_pend == kStoreLag) {
