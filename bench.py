@@ -62,14 +62,21 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def nf4_gemm_source_hash():
+    """Hash of the grouped NF4 GEMM kernel's source text: gemm.cu from its namespace to the next
+    kernel's section (the kernel, its parameters and its constants)."""
+    import hashlib
+    gemm = open(os.path.join(ROOT, "grouped_nf4_expert_b200", "csrc", "gemm.cu"), "rb").read()
+    i = gemm.index(b"namespace nf4g {")
+    j = gemm.index(b"// LoRA projection: out[rows, r]", i)
+    return hashlib.sha256(gemm[i:j]).hexdigest()[:16]
+
+
 def profiled_traffic():
     """DRAM bytes per step of the nf4_gemm launches from the committed ncu summary, if the kernel
     source still hashes to what was profiled; else None."""
-    import hashlib
     import re
-    src = b"".join(open(os.path.join(ROOT, "grouped_nf4_expert_b200", "csrc", f), "rb").read()
-                   for f in ("gemm.cu", "e4b_device.cuh"))
-    sha = hashlib.sha256(src).hexdigest()[:16]
+    sha = nf4_gemm_source_hash()
     try:
         text = open(os.path.join(ROOT, "profiles", "nf4_gemm_train_ncu.md")).read()
     except OSError:
