@@ -245,6 +245,7 @@ e4b_status e4b_route_permute(const e4b_moe_dims* dims, int32_t T, const float* l
                              const e4b_routing* routing, e4b_bf16* x_perm, void* ws, size_t ws_bytes,
                              e4b_stream_t stream) {
   E4B_TRY(check_dims(dims, T));
+  if (T == 0) return E4B_OK;  // nothing is read or written: T-sized pointers may be NULL
   E4B_TRY(check_ws(dims, T, ws, ws_bytes));
   E4B_TRY(check_routing(routing));
   if (!aligned16(logits)) return E4B_ERR_INVALID_ARG;
@@ -266,6 +267,7 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
                                     const e4b_fwd_buffers* fwd, e4b_bf16* y, void* ws, size_t ws_bytes,
                                     e4b_stream_t stream) {
   E4B_TRY(check_dims(dims, T));
+  if (T == 0) return E4B_OK;  // nothing is read or written: T-sized pointers may be NULL
   E4B_TRY(check_ws(dims, T, ws, ws_bytes));
   E4B_TRY(check_routing(routing));
   E4B_TRY(check_base(base));
@@ -367,6 +369,7 @@ e4b_status e4b_moe_serve_fwd(const e4b_moe_dims* dims, int32_t T, const float* l
                              const e4b_fwd_buffers* fwd, e4b_bf16* y, void* ws, size_t ws_bytes,
                              e4b_stream_t stream) {
   E4B_TRY(check_dims(dims, T));
+  if (T == 0) return E4B_OK;  // nothing is read or written: T-sized pointers may be NULL
   E4B_TRY(check_ws(dims, T, ws, ws_bytes));
   E4B_TRY(check_routing(routing));
   E4B_TRY(check_base(base));
@@ -446,6 +449,7 @@ e4b_status e4b_grouped_nf4_lora_dgrad(const e4b_moe_dims* dims, int32_t T, const
                                       const e4b_fwd_buffers* fwd, const e4b_bf16* dY, const e4b_bwd_buffers* bwd,
                                       e4b_bf16* dx, void* ws, size_t ws_bytes, e4b_stream_t stream) {
   E4B_TRY(check_dims(dims, T));
+  if (T == 0) return E4B_OK;  // nothing is read or written: T-sized pointers may be NULL
   E4B_TRY(check_ws(dims, T, ws, ws_bytes));
   E4B_TRY(check_routing(routing));
   E4B_TRY(check_base(base));
@@ -596,6 +600,7 @@ e4b_status e4b_router_backward(const e4b_moe_dims* dims, int32_t T, const e4b_ro
                                const e4b_bf16* y_perm, const e4b_bf16* dY, float* d_logits, float* dw,
                                e4b_stream_t stream) {
   E4B_TRY(check_dims(dims, T));
+  if (T == 0) return E4B_OK;  // nothing is read or written: T-sized pointers may be NULL
   E4B_TRY(check_routing(routing));
   if (!aligned16(y_perm) || !aligned16(dY) || !aligned16(d_logits)) return E4B_ERR_INVALID_ARG;
   if (dw != nullptr && !aligned16(dw)) return E4B_ERR_INVALID_ARG;

@@ -498,7 +498,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       }
       continue;
     }
-    for (int pc = pc0 + lane; pc < vec; pc += 32) {
+    // k > 8: the row indices and weights come by shuffles inside the loop, so every lane runs
+    // every iteration (the loop bound is warp-uniform) and only the loads and stores are guarded.
+    for (int pb = pc0; pb < vec; pb += 32) {
+      const int pc = pb + lane;
+      const bool live = pc < vec;
       float acc[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
@@ -507,7 +511,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 #pragma unroll
         for (int j = 0; j < kRowsPerBatch; ++j) {
           const int r = __shfl_sync(0xffffffffu, my_row, (j0 + j) & 31);
-          if (j0 + j < k) q[j] = __ldg(reinterpret_cast<const uint4*>(src_perm + (size_t)r * H) + pc);
+          q[j] = (live && j0 + j < k) ? __ldg(reinterpret_cast<const uint4*>(src_perm + (size_t)r * H) + pc)
+                                      : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int j = 0; j < kRowsPerBatch; ++j) {
@@ -527,7 +532,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       o.y = pack_bf16x2(acc[2], acc[3]);
       o.z = pack_bf16x2(acc[4], acc[5]);
       o.w = pack_bf16x2(acc[6], acc[7]);
-      reinterpret_cast<uint4*>(out + (size_t)t * H)[pc] = o;
+      if (live) reinterpret_cast<uint4*>(out + (size_t)t * H)[pc] = o;
     }
   }
 }

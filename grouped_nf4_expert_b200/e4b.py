@@ -131,7 +131,13 @@ def _check(status: int, where: str):
 
 
 def _ptr(t) -> Optional[int]:
-    return None if t is None else t.data_ptr()
+    """Device address of a tensor's first element; for an empty view, the address it would have in its
+    storage (torch reports 0 for empty tensors)."""
+    if t is None:
+        return None
+    if t.numel() == 0:
+        return t.untyped_storage().data_ptr() + t.storage_offset() * t.element_size() or None
+    return t.data_ptr()
 
 
 def _stream(stream) -> Optional[int]:
@@ -245,10 +251,10 @@ class Block:
         self.ws = z((int(sz.workspace_bytes),), torch.uint8)
         e4b_workspace_init(self.ws)
         self._dims_c = dims.c()
-        self._routing = Routing(*(t.data_ptr() for t in (self.topk_ids, self.topk_w, self.counts, self.offsets,
-                                                           self.row_of_slot, self.slot_of_row, self.tiles)))
-        self._fwd = FwdBuffers(*(t.data_ptr() for t in (self.x_perm, self.p_gu, self.gu, self.act, self.p_d,
-                                                         self.y_perm)))
+        self._routing = Routing(*(_ptr(t) for t in (self.topk_ids, self.topk_w, self.counts, self.offsets,
+                                                      self.row_of_slot, self.slot_of_row, self.tiles)))
+        self._fwd = FwdBuffers(*(_ptr(t) for t in (self.x_perm, self.p_gu, self.gu, self.act, self.p_d,
+                                                    self.y_perm)))
         self._fwd_nogu = FwdBuffers(self.x_perm.data_ptr(), self.p_gu.data_ptr(), None, self.act.data_ptr(),
                                     self.p_d.data_ptr(), self.y_perm.data_ptr())
         self._bwd = BwdBuffers(*(t.data_ptr() for t in (self.dyw, self.q_d, self.dgu, self.q_gu, self.dx_perm)))

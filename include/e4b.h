@@ -34,7 +34,10 @@
  *     enqueued on `stream` in order.
  *   - bfloat16 tensors are passed as e4b_bf16 (their 16-bit patterns).
  *   - Arguments are validated on the host before anything is launched; a
- *     failed check returns a status and launches nothing.
+ *     failed check returns a status and launches nothing.  With T == 0 the
+ *     calls return E4B_OK without reading or writing anything (pointers to
+ *     T-sized arrays may then be NULL); e4b_lora_wgrad still writes its
+ *     all-zero gradients.
  *   - A launch failure returns E4B_ERR_CUDA.  Device-side waits are bounded:
  *     a wait that runs out records E4B_ERR_DEVICE_TIMEOUT in the workspace,
  *     the kernel ends cleanly, and e4b_check_device_error reports it.

@@ -259,9 +259,52 @@ def test_routing_ties_and_deterministic():
 
 # --------------------------------------------------------------------- full block, small sizes
 
+# Degenerate shapes: one token (a 128-row tile holding 2 rows), every expert selected (k = E),
+# a single expert, and k = 32 (the combine's long path) with H not a multiple of 128.
+EDGE = {
+    "one_token": inputs.Config("one_token", E=4, H=64, I=64, top_k=2, T=1, r=8, alpha=16.0,
+                               routing="normal", seed=51),
+    "k_equals_E": inputs.Config("k_equals_E", E=8, H=128, I=128, top_k=8, T=40, r=16, alpha=32.0,
+                                routing="normal", seed=52),
+    "one_expert": inputs.Config("one_expert", E=1, H=128, I=192, top_k=1, T=200, r=8, alpha=16.0,
+                                routing="normal", seed=53),
+    "k32_ragged": inputs.Config("k32_ragged", E=40, H=192, I=64, top_k=32, T=45, r=8, alpha=16.0,
+                                routing="zipf", seed=54),
+}
+
+
+@pytest.mark.parametrize("name", list(EDGE))
+def test_block_parity_edge_shapes(name):
+    _check_block(EDGE[name], True)
+
+
+def test_zero_tokens_is_a_no_op_with_zero_gradients():
+    cfg = inputs.Config("zero", E=4, H=64, I=64, top_k=2, T=0, r=8, alpha=16.0, routing="normal", seed=55)
+    prob = inputs.make_problem(cfg)
+    d = dv.upload(prob)
+    blk = e4b.Block(dv.dims_of(cfg), 0)
+    for t in (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d):
+        t.fill_(1.0)
+    # [0, .] token tensors still need valid aligned pointers
+    x = torch.zeros((1, cfg.H), dtype=torch.bfloat16, device="cuda")
+    logits = torch.zeros((1, cfg.E), dtype=torch.float32, device="cuda")
+    blk.e4b_route_permute(logits, x, gather=False)
+    blk.e4b_grouped_nf4_lora_fwd(d.base(), d.lora(), x=x)
+    blk.e4b_grouped_nf4_lora_dgrad(d.base(), d.lora(), x)
+    blk.e4b_lora_wgrad()
+    blk.e4b_moe_serve_fwd(logits, x, d.base(), d.lora())
+    torch.cuda.synchronize()
+    assert blk.check_device_error() == e4b.E4B_OK
+    for t in (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d):
+        assert torch.count_nonzero(t).item() == 0
+
+
 @pytest.mark.parametrize("name,fused", [(n, True) for n in SMALL] + [("medium", False), ("stream_r24", False)])
 def test_block_parity_small(name, fused):
-    cfg = SMALL[name]
+    _check_block(SMALL[name], fused)
+
+
+def _check_block(cfg, fused):
     prob, _, blk = run(cfg, fused_gather=fused)
     ros = check_routing(prob, blk)
     ex = oracle_experts(prob)
