@@ -542,8 +542,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 // together, then a butterfly sum), followed by the backward of the softmax
 // over the k selected logits: d_logit[ids_j] = w_j (dw_j - sum_i w_i dw_i);
 // every other logit of the row gets 0.
-constexpr int kRbwdSlots = 8;
-__global__ void __launch_bounds__(256) router_bwd_kernel(const uint16_t* __restrict__ dY,
+constexpr int kRbwdSlots = 4;
+__global__ void __launch_bounds__(256, 4) router_bwd_kernel(const uint16_t* __restrict__ dY,
                                                          const uint16_t* __restrict__ y_perm,
                                                          const int32_t* __restrict__ row_of_slot,
                                                          const int32_t* __restrict__ topk_ids,
