@@ -651,3 +651,31 @@ def test_serve_forward_cuda_graph_replay_is_bit_identical():
     assert np.array_equal(outs[0], eager[0]) and np.array_equal(outs[2], eager[0])
     assert np.array_equal(outs[1], eager[1]) and not np.array_equal(outs[0], outs[1])
     del graph
+
+
+# --------------------------------------------------------------------- expert parallel (owner side)
+
+def test_expert_parallel_owner_forward_matches_expert_outputs():
+    # The owner's computation for rows it received: top-1 onto the given local experts, weight 1,
+    # through the library; each output row must be that expert's output for the row (the oracle's yd).
+    from grouped_nf4_expert_b200 import parallel
+    cfg = SMALL["medium"]
+    prob = inputs.make_problem(cfg)
+    d = dv.upload(prob)
+    ids, _ = oracle.route_topk(prob.logits, cfg.top_k)
+    flat = ids.reshape(-1)
+    lo, hi = 2, 6  # this owner's experts
+    slots = np.flatnonzero((flat >= lo) & (flat < hi))
+    rows = d.x[torch.from_numpy(slots // cfg.top_k).cuda()].contiguous()
+    local_ids = torch.from_numpy((flat[slots] - lo).astype(np.int32)).cuda()
+    sl = slice(lo, hi)
+    base = e4b.nf4_experts(d.gate_up_nf4[sl].contiguous(), d.gate_up_absmax[sl].contiguous(),
+                           d.down_nf4[sl].contiguous(), d.down_absmax[sl].contiguous())
+    keep = [d.A_gu[sl].contiguous(), d.B_gu[sl].contiguous(), d.A_d[sl].contiguous(), d.B_d[sl].contiguous()]
+    blk = parallel.ep_local_forward(e4b.Dims(E=hi - lo, H=cfg.H, I=cfg.I, top_k=1, r=cfg.r, alpha=cfg.alpha),
+                                    rows, local_ids, base, e4b.lora_factors(*keep))
+    assert blk.check_device_error() == e4b.E4B_OK
+    x = inputs.bits_to_f32(prob.x).astype(np.float64)
+    fo = oracle.moe_forward(x, prob.logits, oracle_experts(prob), cfg.top_k, cfg.alpha)
+    want = np.stack([fo["yd"][int(f)] for f in slots])
+    assert rel_err(f64(blk.y), want) <= TOL
