@@ -119,8 +119,20 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
 }
 
 // One CTA of 1024 threads, one thread per expert: counts, 128-aligned group
-// offsets, per-(CTA, expert) scatter bases, padding markers, the m-tile list
-// and the experts in descending-count order.
+// offsets, per-(CTA, expert) scatter bases and the experts in descending-count
+// order; then the whole CTA writes the padding markers and the three work
+// lists (m-tiles, 256-row m-units, 32-slot streaming tiles) as flat index
+// spaces, each entry's expert found by a binary search of the per-expert
+// prefix sums, so that no thread walks a heavy expert's entries alone.
+__device__ __forceinline__ int owner_of(const int* prefix, int E, int i) {  // last e with prefix[e] <= i
+  int lo = 0, hi = E;  // prefix[lo] <= i < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= i) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ block_counts, int nblk,
                                                           int E, int32_t* __restrict__ block_base,
                                                           int32_t* __restrict__ counts,
@@ -129,6 +141,9 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
                                                           int32_t* __restrict__ tiles, int64_t mt_cap) {
   __shared__ int s_warp[32];
   __shared__ int s_cnt[E4B_MAX_EXPERTS];
+  __shared__ int s_off[E4B_MAX_EXPERTS];
+  __shared__ int s_pmt[E4B_MAX_EXPERTS + 1], s_pmu[E4B_MAX_EXPERTS + 1], s_pst[E4B_MAX_EXPERTS + 1];
+  __shared__ int s_ppad[E4B_MAX_EXPERTS + 1];
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E)
@@ -140,8 +155,14 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   const int mu_off = block_exclusive_scan(e < E ? n_mu : 0, s_warp);
   const int n_st = (cnt + 31) / 32;
   const int st_off = block_exclusive_scan(e < E ? n_st : 0, s_warp);
+  const int pad_off = block_exclusive_scan(e < E ? padded - cnt : 0, s_warp);
   if (e < E) {
     s_cnt[e] = cnt;
+    s_off[e] = off;
+    s_pmt[e] = mt_off;
+    s_pmu[e] = mu_off;
+    s_pst[e] = st_off;
+    s_ppad[e] = pad_off;
     counts[e] = cnt;
     offsets[e] = off;
     int run = off;
@@ -149,24 +170,11 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
       block_base[(size_t)b * E + e] = run;
       run += block_counts[(size_t)b * E + e];
     }
-    for (int r = off + cnt; r < off + padded; ++r) slot_of_row[r] = -1;
-    for (int i = 0; i < padded / 128; ++i) {
-      tiles[kTileHeader + 2 * (mt_off + i)] = e;
-      tiles[kTileHeader + 2 * (mt_off + i) + 1] = off + 128 * i;
-    }
-    int32_t* mu = tiles + kTileHeader + 2 * mt_cap + E;
-    for (int i = 0; i < n_mu; ++i) {
-      mu[3 * (mu_off + i)] = e;
-      mu[3 * (mu_off + i) + 1] = off + 256 * i;
-      mu[3 * (mu_off + i) + 2] = min(256, padded - 256 * i);
-    }
-    int32_t* st = tiles + kTileHeader + 2 * mt_cap + E + 3 * mt_cap;
-    for (int i = 0; i < n_st; ++i) {
-      st[3 * (st_off + i)] = e;
-      st[3 * (st_off + i) + 1] = off + 32 * i;
-      st[3 * (st_off + i) + 2] = min(32, cnt - 32 * i);
-    }
     if (e == E - 1) {
+      s_pmt[E] = mt_off + padded / 128;
+      s_pmu[E] = mu_off + n_mu;
+      s_pst[E] = st_off + n_st;
+      s_ppad[E] = pad_off + padded - cnt;
       offsets[E] = off + padded;
       tiles[0] = mt_off + padded / 128;
       tiles[1] = off + padded;
@@ -179,6 +187,30 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
     int rank = 0;
     for (int o = 0; o < E; ++o) rank += (s_cnt[o] > cnt) || (s_cnt[o] == cnt && o < e);
     tiles[kTileHeader + 2 * mt_cap + rank] = e;
+  }
+  for (int i = threadIdx.x; i < s_ppad[E]; i += blockDim.x) {
+    const int x = owner_of(s_ppad, E, i);
+    slot_of_row[s_off[x] + s_cnt[x] + (i - s_ppad[x])] = -1;
+  }
+  for (int i = threadIdx.x; i < s_pmt[E]; i += blockDim.x) {
+    const int x = owner_of(s_pmt, E, i);
+    tiles[kTileHeader + 2 * i] = x;
+    tiles[kTileHeader + 2 * i + 1] = s_off[x] + 128 * (i - s_pmt[x]);
+  }
+  int32_t* mu = tiles + kTileHeader + 2 * mt_cap + E;
+  for (int i = threadIdx.x; i < s_pmu[E]; i += blockDim.x) {
+    const int x = owner_of(s_pmu, E, i), q = i - s_pmu[x];
+    const int pad_x = (s_cnt[x] + 127) / 128 * 128;
+    mu[3 * i] = x;
+    mu[3 * i + 1] = s_off[x] + 256 * q;
+    mu[3 * i + 2] = min(256, pad_x - 256 * q);
+  }
+  int32_t* st = tiles + kTileHeader + 2 * mt_cap + E + 3 * mt_cap;
+  for (int i = threadIdx.x; i < s_pst[E]; i += blockDim.x) {
+    const int x = owner_of(s_pst, E, i), q = i - s_pst[x];
+    st[3 * i] = x;
+    st[3 * i + 1] = s_off[x] + 32 * q;
+    st[3 * i + 2] = min(32, s_cnt[x] - 32 * q);
   }
 }
 
