@@ -1,14 +1,17 @@
 // Grouped GEMMs on the 5th-generation tensor cores (tcgen05, TMEM
 // accumulators, TMA-fed shared memory) for the NF4 expert block:
 //
-//  * nf4_gemm_kernel: one 128x128 output tile per work unit of a grouped
-//    GEMM whose B operand is a frozen NF4 expert matrix, dequantised into
-//    shared memory by a decode warpgroup (bit-exact bf16 weights), with the
-//    LoRA term as an extra K = r MMA into the same TMEM accumulator.  Four
-//    modes: forward gate_up (SiLU-gated epilogue), forward down, down dgrad
-//    (transposed base, SwiGLU backward epilogue), gate_up dgrad.
+//  * nf4_gemm_kernel: persistent CTA pairs, one 256x256 output tile per work
+//    unit (cta_group::2 UMMAs) of a grouped GEMM whose B operand is a frozen
+//    NF4 expert matrix, dequantised into shared memory by four decode groups
+//    (bit-exact bf16 weights), with the LoRA term as an extra K = r MMA into
+//    the same TMEM accumulator.  Four modes: forward gate_up (SiLU-gated
+//    epilogue), forward down, down dgrad (transposed base, SwiGLU backward
+//    epilogue), gate_up dgrad.
 //  * lora_proj_kernel: s * (rows x LoRA factor) -> [rows, r], the low-rank
 //    projections p = s x A^T and q = s dy B.
+//  * gather_proj_kernel: the row gather of x (or w * dY) into the permuted
+//    buffer fused with its LoRA projection.
 //  * wgrad_kernel: variable-K grouped GEMM for the LoRA weight gradients
 //    (K = the rows of one expert).
 //
