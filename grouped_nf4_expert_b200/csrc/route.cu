@@ -1,7 +1,9 @@
 // Routing and permutation kernels: top-k + softmax, expert histogram, prefix
 // sums with per-expert padding, the device work list, a deterministic stable
-// scatter, row gathers and the weighted un-permute combine.  Also the NF4
-// dequantisation test kernel and the watchdog self-test.
+// scatter, row gathers and the weighted un-permute combine; the serving call's
+// one-CTA routing and CUDA-core LoRA row projections; the router backward
+// (d logits of a trained router); the NF4 quantiser and the dequantisation
+// test kernel; the watchdog self-test.
 //
 // Pages: "How do I QLoRA-train the fused experts of a MoE", section "Which
 // project solves it" (grouped execution of the routed experts) and section

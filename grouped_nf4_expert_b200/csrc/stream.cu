@@ -2,10 +2,10 @@
 //
 // When a batch routes only a few slots to each expert, the block's cost is
 // reading every touched expert's NF4 weights once.  Here the weights are the
-// UMMA M operand (128 weight rows per tile, decoded into shared memory) and
-// up to 32 routed slots of one expert are the N operand, so each weight byte is
-// fetched and decoded once per 32 slots.  Decoded tiles go to tensor memory,
-// which the UMMA reads as its A operand.  A code stage holds 4 k-chunks, so
+// UMMA M operand (128 weight rows per tile) and up to 32 routed slots of one
+// expert are the N operand, so each weight byte is fetched and decoded once
+// per 32 slots.  Decoded tiles go straight to tensor memory, which the UMMA
+// reads as its A operand.  A code stage holds 4 k-chunks, so
 // every weight row contributes one whole 128-byte line (and one 16-byte run
 // of block scales) per stage; rings of code stages and of activation-row tiles
 // keep enough memory traffic in flight.
@@ -15,8 +15,8 @@
 // the decoded rows of its stage's four k-chunks straight into its own A
 // buffer in tensor memory, and one warp issues every stage's UMMAs in order
 // with those tiles as the A operand read from tensor memory.  Outputs match the training tiles (gu /
-// act for gate_up, y_perm for down), with the LoRA term as K = r UMMAs into
-// the same accumulator.
+// act for gate_up, y_perm for down; the serving call skips gu), with the LoRA
+// term as K = r UMMAs into the same accumulator.
 //
 // Pages: "How do I QLoRA-train the fused experts of a MoE", section "The
 // abstraction that fails" (per-expert delta before the activation) and
