@@ -94,6 +94,7 @@ constexpr int LB_OFF = LA_OFF + LA_BYTES;
 constexpr int kEpiTileBytes = 32 * 16 * 2;
 constexpr int kEpiStepBytes = 3 * kEpiTileBytes;
 constexpr int kEpiWarpBytes = 2 * kEpiStepBytes;
+static_assert(kEpiWarpBytes >= 3 * 2 * kEpiTileBytes, "three 2-tile buffers for the plain epilogue");
 constexpr int EPI_OFF = LB_OFF + LB_BYTES;
 constexpr int BAR_OFF = EPI_OFF + 4 * kEpiWarpBytes;
 constexpr int BAR_BYTES = 1024;
@@ -607,21 +608,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           }
         }
       } else {
+        // 32-column steps (n_dim is a multiple of 64): two 16-column tiles per step from a ring of
+        // three 2 KB buffers, so that a unit's accumulator is drained in 8 steps, each with one
+        // TMEM wait and one proxy fence (in the down projection's short units the epilogue would
+        // otherwise hold the accumulator past the next unit's start).
         const int c0 = nt * 256;
 #pragma unroll 1
-        for (int jj = 0; jj < 256; jj += 16) {
+        for (int jj = 0; jj < 256; jj += 32) {
           if (c0 + jj >= p.n_dim) break;
-          float v[16];
-          tmem_ld16(tl + jj, v);
+          float v[32];
+          tmem_ld32(tl + jj, v);
           if (!store) continue;
-          uint32_t w[8];
+          uint32_t w0[8], w1[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          const uint32_t buf = step_buffer();
-          stage(buf, 0, w);
+          for (int i = 0; i < 8; ++i) {
+            w0[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            w1[i] = pack_bf16x2(v[16 + 2 * i], v[16 + 2 * i + 1]);
+          }
+          if (lane == 0) bulk_wait_read<2>();
+          __syncwarp();
+          const uint32_t buf = ebuf + (step % 3) * (2 * kEpiTileBytes);
+          stage(buf, 0, w0);
+          stage(buf, 1, w1);
           publish();
           if (lane == 0) {
             tma_store_2d(&map_o0, buf, c0 + jj, wrow0);
+            tma_store_2d(&map_o0, buf + kEpiTileBytes, c0 + jj + 16, wrow0);
             bulk_commit();
           }
           ++step;
