@@ -964,6 +964,9 @@ __global__ void __launch_bounds__(gproj::kThreads, 2)  // two CTAs per SM: <= 64
         }
       }
     }
+    // every copy of this thread has landed before the CTA's shared memory can go away (a timeout
+    // elsewhere may end the loops with copies still in flight)
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp < kScaleWarp0 + kScaleWarps) {
     // ------------------------------------------------ scalers (weighted gather): row *= w(slot) in place
     if (p.scale_w != nullptr) {
