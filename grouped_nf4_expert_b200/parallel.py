@@ -120,3 +120,14 @@ def ep_local_forward(dims_local, rows, local_ids, base_local, lora_local):
     blk.e4b_route_permute(logits, rows, gather=False)
     blk.e4b_grouped_nf4_lora_fwd(base_local, lora_local, x=rows)
     return blk
+
+
+def ep_local_backward(blk, dyw_rows, base_local, lora_local):
+    """The owner's backward for the rows it received: ``dyw_rows`` bf16 [R, H] are the received
+    w * dY rows (the routing weight applied by the sender), run through the library's input
+    gradient and LoRA weight gradients with the top-1, weight-1 routing of :func:`ep_local_forward`
+    (``blk`` is the block it returned).  Returns ``blk``: ``dx`` [R, H] holds each row's input
+    gradient (to be sent back), ``dA_gu``/``dB_gu``/``dA_d``/``dB_d`` the owner's expert gradients."""
+    blk.e4b_grouped_nf4_lora_dgrad(base_local, lora_local, dyw_rows)
+    blk.e4b_lora_wgrad()
+    return blk

@@ -655,7 +655,7 @@ def test_serve_forward_cuda_graph_replay_is_bit_identical():
 
 # --------------------------------------------------------------------- expert parallel (owner side)
 
-def test_expert_parallel_owner_forward_matches_expert_outputs():
+def test_expert_parallel_owner_forward_and_backward():
     # The owner's computation for rows it received: top-1 onto the given local experts, weight 1,
     # through the library; each output row must be that expert's output for the row (the oracle's yd).
     from grouped_nf4_expert_b200 import parallel
@@ -679,3 +679,22 @@ def test_expert_parallel_owner_forward_matches_expert_outputs():
     fo = oracle.moe_forward(x, prob.logits, oracle_experts(prob), cfg.top_k, cfg.alpha)
     want = np.stack([fo["yd"][int(f)] for f in slots])
     assert rel_err(f64(blk.y), want) <= TOL
+    # the owner's backward: received w * dY rows -> each row's input gradient and its experts' gradients
+    _, w = oracle.route_topk(prob.logits, cfg.top_k)
+    dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
+    wf = w.reshape(-1)
+    dyw_bits = oracle.bf16_round_bits((wf[slots, None] * dY[slots // cfg.top_k]).astype(np.float32))
+    dyw = torch.from_numpy(dyw_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    parallel.ep_local_backward(blk, dyw, base, e4b.lora_factors(*keep))
+    assert blk.check_device_error() == e4b.E4B_OK
+    # the oracle on the same rows: top-1 onto the local experts, weight 1, upstream = the bf16 rows sent
+    sub = oracle_experts(prob)
+    sub = oracle.Experts(*(getattr(sub, f)[sl] for f in ("gate_up_nf4", "gate_up_absmax", "down_nf4",
+                                                          "down_absmax", "A_gu", "B_gu", "A_d", "B_d")))
+    lg = np.full((len(slots), hi - lo), -1e30, dtype=np.float32)
+    lg[np.arange(len(slots)), flat[slots] - lo] = 0.0
+    bo = oracle.moe_backward(x[slots // cfg.top_k], lg, inputs.bits_to_f32(dyw_bits).astype(np.float64), sub, 1,
+                             cfg.alpha)
+    assert rel_err(f64(blk.dx), bo["dx"]) <= TOL
+    for key, buf in [("dA_gu", blk.dA_gu), ("dB_gu", blk.dB_gu), ("dA_d", blk.dA_d), ("dB_d", blk.dB_d)]:
+        assert rel_err(f64(buf), bo[key]) <= TOL, key
