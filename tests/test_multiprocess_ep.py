@@ -22,6 +22,8 @@ from grouped_nf4_expert_b200 import inputs
 from grouped_nf4_expert_b200 import parallel
 
 CFG = inputs.Config("ep", E=4, H=64, I=64, top_k=2, T=13, r=8, alpha=16.0, routing="zipf", seed=57)
+# four ranks, two experts each, skewed routing and few tokens: some rank pairs exchange no rows
+CFG4 = inputs.Config("ep4", E=8, H=64, I=64, top_k=3, T=5, r=8, alpha=16.0, routing="zipf", seed=58)
 KEYS = ("dA_gu", "dB_gu", "dA_d", "dB_d")
 
 
@@ -37,7 +39,9 @@ def _onehot_logits(local_ids, n):
     return lg
 
 
-def _worker(rank, world, port, out_q):
+def _worker(rank, world, port, out_q, cfg_name="ep"):
+    global CFG
+    CFG = CFG4 if cfg_name == "ep4" else CFG
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     import datetime
@@ -68,7 +72,8 @@ def _worker(rank, world, port, out_q):
             grads = [np.zeros_like(getattr(local, a)) for a in ("A_gu", "B_gu", "A_d", "B_d")]
         dx = parallel.ep_combine(parallel.ep_return(torch.from_numpy(dx_rows), plan2),
                                  torch.ones_like(w_t)).double().numpy()
-        out_q.put((rank, y, dx, grads, int(plan.send_counts[1 - rank]), int(plan.recv_counts[1 - rank])))
+        out_q.put((rank, y, dx, grads, sum(plan.send_counts) - plan.send_counts[rank],
+                   sum(plan.recv_counts) - plan.recv_counts[rank]))
     finally:
         dist.destroy_process_group()
 
@@ -80,11 +85,26 @@ def _free_port():
 
 
 def test_two_rank_expert_parallel_equals_full_block():
-    world = 2
+    _run_and_check(2, CFG, "ep", require_exchange=True)
+
+
+def test_four_rank_expert_parallel_with_empty_exchanges():
+    # the case really has a rank that sends no rows to another
+    counts = []
+    for r in range(4):
+        ids, _ = oracle.route_topk(inputs.make_problem(CFG4, data_rank=r).logits, CFG4.top_k)
+        counts.append(np.bincount(ids.reshape(-1) // (CFG4.E // 4), minlength=4))
+    assert (np.array(counts) == 0).any()
+    _run_and_check(4, CFG4, "ep4", require_exchange=False)
+
+
+def _run_and_check(world, cfg, cfg_name, require_exchange):
+    global CFG
+    CFG = cfg
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, cfg_name)) for r in range(world)]
     for p in procs:
         p.start()
     results = {}
@@ -105,7 +125,8 @@ def test_two_rank_expert_parallel_equals_full_block():
         y, dx, _, sent, recvd = results[r]
         np.testing.assert_allclose(y, fo["y"], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dx, bo["dx"], rtol=1e-10, atol=1e-12)
-        assert sent > 0 and recvd > 0  # rows really crossed between the ranks
+        if require_exchange:
+            assert sent > 0 and recvd > 0  # rows really crossed between the ranks
         for k in KEYS:
             grads_union[k] = grads_union[k] + bo[k]
     e_loc = CFG.E // world
