@@ -168,3 +168,14 @@ def test_dequant_and_watchdog_argument_checks(so):
     assert so.e4b_nf4_quantize(p[0], 0, p[1], p[2], None) == e4b.E4B_OK  # nothing to do
     assert so.e4b_debug_watchdog(p[0], 256, 0, None) == e4b.E4B_ERR_INVALID_ARG
     assert so.e4b_debug_watchdog(p[0], 8, 1000, None) == e4b.E4B_ERR_INVALID_ARG
+
+
+def test_binding_pointer_of_empty_views_is_their_storage_address():
+    # torch reports address 0 for empty tensors; the binding passes where the view would start, so
+    # that a T = 0 call sees valid (aligned) pointers rather than NULL
+    import torch
+    buf = torch.zeros(64)
+    assert e4b._ptr(buf[:0]) == buf.data_ptr()
+    assert e4b._ptr(buf[16:16]) == buf.data_ptr() + 16 * 4
+    assert e4b._ptr(buf[4:]) == buf.data_ptr() + 16
+    assert e4b._ptr(None) is None
