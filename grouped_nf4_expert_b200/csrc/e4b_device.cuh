@@ -172,10 +172,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier in any CTA of the cluster (address from mapa_shared).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
 
 // Non-blocking signal to another CTA of the cluster: stores `v` to the word at
 // `remote_word` and performs complete_tx(4 bytes) on the mbarrier at
@@ -451,16 +447,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Whole warp: 8 consecutive 32-bit columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 // Whole warp: each thread writes 32 consecutive 32-bit columns of its own
 // TMEM lane (the warp's 32-lane quadrant), then waits for the writes.
@@ -668,17 +654,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Writes 64 bf16 (one 128-byte row of a 128B-swizzled atom) to shared memory:
-// row `row` of the 8-row group starting at `base` + (row/8)*1024; 16-byte chunk
-// c goes to chunk c ^ (row % 8).
-__device__ __forceinline__ void st_swizzled_row128(uint8_t* base, int row, const uint32_t (&v)[32]) {
-  uint8_t* rp = base + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 q = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-    *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = q;
-  }
-}
 
 // silu and the logistic sigmoid with the fast exponential and the fast
 // (reciprocal-based) division: a few ulp, far below bf16 output rounding.  For
