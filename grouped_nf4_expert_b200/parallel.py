@@ -131,3 +131,30 @@ def ep_local_backward(blk, dyw_rows, base_local, lora_local):
     blk.e4b_grouped_nf4_lora_dgrad(base_local, lora_local, dyw_rows)
     blk.e4b_lora_wgrad()
     return blk
+
+
+def ep_block_forward(ids, w, x, E: int, local_forward, group=None):
+    """Expert-parallel forward of this rank's tokens.
+
+    ``ids``/``w`` [T, k]: this rank's routing over all E experts; ``x`` [T, H].  ``local_forward(rows,
+    local_ids)`` computes the owner's expert outputs for the rows it received (for instance through
+    :func:`ep_local_forward`: its block's ``y``).  Returns ``(y, state)``: y [T, H] in fp32 (fp64 for
+    fp64 rows), and the state :func:`ep_block_backward` needs.
+    """
+    rows, local_ids, plan = ep_dispatch(ids, x, E, group)
+    yd = local_forward(rows, local_ids)
+    y = ep_combine(ep_return(yd, plan, group), w)
+    return y, (rows, local_ids)
+
+
+def ep_block_backward(ids, w, dY, E: int, local_backward, group=None):
+    """Expert-parallel input gradient of this rank's tokens: w * dY rows go to the owners,
+    ``local_backward(dyw_rows, local_ids)`` returns each received row's input gradient (the owner
+    keeps its experts' LoRA gradients), and the rows come back summed per token: dx [T, H]."""
+    import torch
+    T, k = w.shape
+    dt = torch.promote_types(torch.float32, dY.dtype)  # the product in fp32, rounded once (as the library)
+    dyw = (w.to(dt).unsqueeze(2) * dY.to(dt).unsqueeze(1)).to(dY.dtype).reshape(T * k, -1)
+    rows, local_ids, plan = ep_dispatch(ids, dyw, E, group)
+    dx_rows = local_backward(rows, local_ids)
+    return ep_combine(ep_return(dx_rows, plan, group), torch.ones_like(w))

@@ -55,25 +55,36 @@ def _worker(rank, world, port, out_q, cfg_name="ep"):
         dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
         ids, w = oracle.route_topk(prob.logits, CFG.top_k)
         ids_t, w_t = torch.from_numpy(ids.astype(np.int64)), torch.from_numpy(w)
-        # forward: rows out, expert outputs back, weighted combine
-        rx, rid, plan = parallel.ep_dispatch(ids_t, torch.from_numpy(x), CFG.E)
-        lg = _onehot_logits(rid.numpy(), e_loc)
-        yd = oracle.moe_forward(rx.numpy(), lg, local, 1, CFG.alpha)["y"] if len(rid) else np.zeros((0, CFG.H))
-        y = parallel.ep_combine(parallel.ep_return(torch.from_numpy(yd), plan), w_t).double().numpy()
-        # backward: w * dY rows out, slot input gradients back, summed per token
-        dyw = torch.from_numpy((w[:, :, None] * dY[:, None, :]).reshape(-1, CFG.H))
-        rdy, rid2, plan2 = parallel.ep_dispatch(ids_t, dyw, CFG.E)
-        assert torch.equal(rid, rid2)
-        if len(rid):
-            bo = oracle.moe_backward(rx.numpy(), lg, rdy.numpy(), local, 1, CFG.alpha)
-            dx_rows, grads = bo["dx"], [bo[k] for k in KEYS]
-        else:
-            dx_rows = np.zeros((0, CFG.H))
-            grads = [np.zeros_like(getattr(local, a)) for a in ("A_gu", "B_gu", "A_d", "B_d")]
-        dx = parallel.ep_combine(parallel.ep_return(torch.from_numpy(dx_rows), plan2),
-                                 torch.ones_like(w_t)).double().numpy()
-        out_q.put((rank, y, dx, grads, sum(plan.send_counts) - plan.send_counts[rank],
-                   sum(plan.recv_counts) - plan.recv_counts[rank]))
+        # the owner's computation for received rows: top-1 onto the local expert, weight 1 (the oracle)
+        seen = {}
+
+        def local_forward(rows, local_ids):
+            seen["x"], seen["ids"] = rows.numpy(), local_ids.numpy()
+            if not len(local_ids):
+                return torch.zeros((0, CFG.H), dtype=torch.float64)
+            lg = _onehot_logits(local_ids.numpy(), e_loc)
+            return torch.from_numpy(oracle.moe_forward(rows.numpy(), lg, local, 1, CFG.alpha)["y"])
+
+        def local_backward(dyw_rows, local_ids):
+            assert np.array_equal(local_ids.numpy(), seen["ids"])  # same rows, same order as the forward
+            if not len(local_ids):
+                seen["grads"] = [np.zeros_like(getattr(local, a)) for a in ("A_gu", "B_gu", "A_d", "B_d")]
+                return torch.zeros((0, CFG.H), dtype=torch.float64)
+            lg = _onehot_logits(local_ids.numpy(), e_loc)
+            bo = oracle.moe_backward(seen["x"], lg, dyw_rows.numpy(), local, 1, CFG.alpha)
+            seen["grads"] = [bo[k] for k in KEYS]
+            return torch.from_numpy(bo["dx"])
+
+        y, _ = parallel.ep_block_forward(ids_t, w_t, torch.from_numpy(x), CFG.E, local_forward)
+        dx = parallel.ep_block_backward(ids_t, w_t, torch.from_numpy(dY), CFG.E, local_backward)
+        # rows that crossed between ranks (counted from the routing, as the dispatch plans them)
+        owner = parallel.expert_owner(ids_t.reshape(-1), CFG.E, world)
+        sent = int((owner != rank).sum())
+        counts = torch.bincount(owner, minlength=world)
+        recv = torch.empty_like(counts)
+        dist.all_to_all_single(recv, counts)
+        recvd = int(recv.sum() - recv[rank])
+        out_q.put((rank, y.double().numpy(), dx.double().numpy(), seen["grads"], sent, recvd))
     finally:
         dist.destroy_process_group()
 
