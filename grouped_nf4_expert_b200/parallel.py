@@ -1,8 +1,14 @@
-"""Data-parallel plumbing: one process per GPU, each running the whole block on its own tokens.
+"""Multi-GPU plumbing, one process per GPU over torch.distributed (NCCL over NVLink on GPUs; the
+tests use gloo on CPU).
 
-The frozen NF4 base is replicated and has no gradient, so the only exchange
-of a data-parallel training step is the sum of the four LoRA gradient tensors
-over all ranks (NCCL over NVLink on GPUs; any torch.distributed backend works).
+Data parallel: every rank runs the whole block on its own tokens.  The frozen NF4 base is
+replicated and has no gradient, so the only exchange of a training step is the sum of the four
+LoRA gradient tensors over all ranks (:func:`allreduce_lora_grads`).
+
+Expert parallel: the experts are split across the ranks and the routed rows travel to their
+experts' owners and back (:func:`ep_dispatch`, :func:`ep_return`, :func:`ep_combine`,
+:func:`ep_block_forward`, :func:`ep_block_backward`); the owner computes through the library with
+:func:`ep_local_forward` / :func:`ep_local_backward`.
 """
 
 from __future__ import annotations
