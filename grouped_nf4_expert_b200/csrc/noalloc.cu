@@ -64,14 +64,14 @@ extern "C" e4b_status e4b_route_permute_noalloc(const e4b_moe_dims* dims, int32_
   e4b_sizes sz;
   const e4b_status st = e4b_get_sizes(dims, T, &sz);  // validates dims and T
   if (st != E4B_OK) return st;
+  if (T == 0) return E4B_OK;  // nothing is read or written: T-sized pointers may be NULL
   if (routing == nullptr || !aligned16(routing->topk_ids) || !aligned16(routing->topk_w) ||
       !aligned16(routing->counts) || !aligned16(routing->offsets) || !aligned16(routing->row_of_slot) ||
-      !aligned16(routing->slot_of_row) || !aligned16(routing->tiles) || !aligned16(logits) || !aligned16(x) ||
-      !aligned16(x_perm))
+      !aligned16(routing->slot_of_row) || !aligned16(routing->tiles) || !aligned16(logits) ||
+      (x_perm != nullptr && (!aligned16(x) || !aligned16(x_perm))))
     return E4B_ERR_INVALID_ARG;
   const int64_t nblk = ((int64_t)T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock;
   if (2 * nblk * (int64_t)dims->E > kNoallocScratchInts) return E4B_ERR_UNSUPPORTED;
-  if (T == 0) return E4B_OK;
   int32_t* scratch = nullptr;
   int sms = 0;
   if (setup_current_device(&scratch, &sms) != cudaSuccess) {

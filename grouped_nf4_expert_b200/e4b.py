@@ -80,6 +80,8 @@ _SIGNATURES = {
     "e4b_check_device_error": (c_i32, [c_vp, c_vp]),
     "e4b_route_permute": (c_i32, [ctypes.POINTER(MoeDims), c_i32, c_vp, c_vp, ctypes.POINTER(Routing), c_vp,
                                   c_vp, c_sz, c_vp]),
+    "e4b_route_permute_noalloc": (c_i32, [ctypes.POINTER(MoeDims), c_i32, c_vp, c_vp, ctypes.POINTER(Routing),
+                                          c_vp, c_vp]),
     "e4b_grouped_nf4_lora_fwd": (c_i32, [ctypes.POINTER(MoeDims), c_i32, ctypes.POINTER(Routing),
                                          ctypes.POINTER(Nf4Experts), ctypes.POINTER(Lora), c_vp,
                                          ctypes.POINTER(FwdBuffers), c_vp, c_vp, c_sz, c_vp]),
@@ -265,6 +267,13 @@ class Block:
         _check(lib().e4b_route_permute(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
                                        ctypes.byref(self._routing), _ptr(self.x_perm) if gather else None,
                                        _ptr(self.ws), self.ws.numel(), _stream(stream)), "e4b_route_permute")
+
+    def e4b_route_permute_noalloc(self, logits, x, gather=True, stream=None):
+        """As ``e4b_route_permute``, with the library's fixed scratch instead of ``ws`` (capturable in
+        a global-mode CUDA graph once a first call on the device has been made)."""
+        _check(lib().e4b_route_permute_noalloc(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
+                                               ctypes.byref(self._routing), _ptr(self.x_perm) if gather else None,
+                                               _stream(stream)), "e4b_route_permute_noalloc")
 
     def e4b_grouped_nf4_lora_fwd(self, base: Nf4Experts, lora: Lora, x=None, stream=None):
         """Forward; with ``x`` the call also writes ``x_perm`` (fused with the first projection)."""

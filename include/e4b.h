@@ -185,14 +185,16 @@ e4b_status e4b_route_permute(const e4b_moe_dims *dims, int32_t T, const float *l
  * counterpart; this is an addition of this library.
  * Scratch lives in a fixed 4 MiB array in the library's own device memory
  * (held on every GPU that loads the library until the process exits); calls
- * whose 2 * ceil(T / 256) * E int32 scratch entries exceed 1,048,576 are
+ * whose 2 * ceil(T / 64) * E int32 scratch entries exceed 1,048,576 are
  * refused with E4B_ERR_UNSUPPORTED.  Allocates nothing (no cudaMalloc,
  * cudaFree or allocating library call).  The first call on a device looks
  * up the array's device address (a one-time set-up per device, made with
  * that device current); make that first call before any stream capture.
  * All calls share the one array: calls whose work overlaps on the GPU (other
  * streams, other host threads) race on it and must be serialised by the
- * caller.  Nothing in the array needs to start at zero. */
+ * caller.  Nothing in the array needs to start at zero.  As with
+ * e4b_route_permute, x_perm NULL writes the routing tables only (x unread),
+ * and T == 0 returns E4B_OK with nothing launched. */
 e4b_status e4b_route_permute_noalloc(const e4b_moe_dims *dims, int32_t T, const float *logits,
                                      const e4b_bf16 *x, const e4b_routing *routing, e4b_bf16 *x_perm,
                                      e4b_stream_t stream);

@@ -114,6 +114,14 @@ def test_null_and_misaligned_pointers_refused(so):
     # routing tables only (no x_perm): x is not needed; nothing to do for T == 0
     assert so.e4b_route_permute(ctypes.byref(d), 0, p[7], None, ctypes.byref(routing), None, ws, wsb,
                                 None) == e4b.E4B_OK
+    # the allocation-free variant validates the same way, before any CUDA call
+    na = so.e4b_route_permute_noalloc
+    assert na(ctypes.byref(d), 0, None, None, None, None, None) == e4b.E4B_OK
+    assert na(ctypes.byref(d), T, p[7], p[8] + 2, ctypes.byref(routing), p[9], None) == e4b.E4B_ERR_INVALID_ARG
+    assert na(ctypes.byref(d), T, p[7], None, None, None, None) == e4b.E4B_ERR_INVALID_ARG
+    big = e4b.Dims(E=1024, H=64, I=64, top_k=2, r=8, alpha=16.0).c()
+    assert na(ctypes.byref(big), 256 * 600, p[7], None, ctypes.byref(routing), None,
+              None) == e4b.E4B_ERR_UNSUPPORTED
     bwd = e4b.BwdBuffers(*p[26:30], p[30] + 8)
     base_ok = e4b.Nf4Experts(*p[11:15])
     assert so.e4b_grouped_nf4_lora_dgrad(ctypes.byref(d), T, ctypes.byref(routing), ctypes.byref(base_ok),

@@ -8,7 +8,8 @@ through the C ABI twice in a row, on two different batches, and checks each
 result against ``e4b_route_permute`` on the same inputs: routing ids, counts,
 offsets, permutation and the permuted rows must be identical, and the routing
 weights within the parity tests' tolerance (they come out bit-identical).
-It also checks that a problem too large for the fixed array is refused.
+A third call writes the routing tables only (no permuted rows), through the
+binding.  It also checks that a problem too large for the fixed array is refused.
 This file is named to be collected last.
 """
 
@@ -54,6 +55,12 @@ def test_noalloc_routing_matches_workspace_routing_twice_in_a_row():
         assert torch.equal(out.slot_of_row[:used], ref.slot_of_row[:used]), batch
         assert torch.equal(out.x_perm[:used], ref.x_perm[:used]), batch
         np.testing.assert_allclose(out.topk_w.cpu().numpy(), ref.topk_w.cpu().numpy(), rtol=1e-6, atol=0)
+    # tables only (no x_perm), through the binding: the same tables again
+    tab = e4b.Block(dims, cfg.T)
+    tab.e4b_route_permute_noalloc(d.logits, None, gather=False)
+    torch.cuda.synchronize()
+    for name in ("topk_ids", "counts", "offsets", "row_of_slot", "tiles"):
+        assert torch.equal(getattr(tab, name), getattr(ref, name)), name
 
 
 def test_noalloc_refuses_problems_beyond_its_fixed_scratch():
