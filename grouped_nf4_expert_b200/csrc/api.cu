@@ -250,7 +250,6 @@ e4b_status e4b_route_permute(const e4b_moe_dims* dims, int32_t T, const float* l
   E4B_TRY(check_routing(routing));
   if (!aligned16(logits)) return E4B_ERR_INVALID_ARG;
   if (x_perm != nullptr && (!aligned16(x) || !aligned16(x_perm))) return E4B_ERR_INVALID_ARG;
-  if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
   const int64_t N = (int64_t)T * dims->top_k;
@@ -275,7 +274,6 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims* dims, int32_t T, const e
   E4B_TRY(check_fwd(fwd));
   if (!aligned16(y)) return E4B_ERR_INVALID_ARG;
   if (x != nullptr && !aligned16(x)) return E4B_ERR_INVALID_ARG;
-  if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
   const cudaStream_t st = (cudaStream_t)stream;
@@ -385,7 +383,6 @@ e4b_status e4b_moe_serve_fwd(const e4b_moe_dims* dims, int32_t T, const float* l
     E4B_TRY(e4b_route_permute(dims, T, logits, x, routing, nullptr, ws, ws_bytes, stream));
     return e4b_grouped_nf4_lora_fwd(dims, T, routing, base, lora, x, fwd, y, ws, ws_bytes, stream);
   }
-  if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
   const cudaStream_t st = (cudaStream_t)stream;
@@ -457,7 +454,6 @@ e4b_status e4b_grouped_nf4_lora_dgrad(const e4b_moe_dims* dims, int32_t T, const
   E4B_TRY(check_fwd(fwd));
   E4B_TRY(check_bwd(bwd));
   if (!aligned16(dY) || !aligned16(dx)) return E4B_ERR_INVALID_ARG;
-  if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
   const cudaStream_t st = (cudaStream_t)stream;
@@ -604,7 +600,6 @@ e4b_status e4b_router_backward(const e4b_moe_dims* dims, int32_t T, const e4b_ro
   E4B_TRY(check_routing(routing));
   if (!aligned16(y_perm) || !aligned16(dY) || !aligned16(d_logits)) return E4B_ERR_INVALID_ARG;
   if (dw != nullptr && !aligned16(dw)) return E4B_ERR_INVALID_ARG;
-  if (T == 0) return E4B_OK;
   int sms = 0;
   E4B_CUDA(device_sms(&sms));
   E4B_CUDA(launch_router_bwd(reinterpret_cast<const uint16_t*>(dY), reinterpret_cast<const uint16_t*>(y_perm),
