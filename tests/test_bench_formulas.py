@@ -1,5 +1,5 @@
 """The algorithmic work counts bench.py divides by (the roofline numerators), checked against
-operation-by-operation tallies of the block on small shapes."""
+operation-by-operation tallies of the block on small shapes; and the reference arm's JSON line."""
 
 import importlib.util
 import os
@@ -57,3 +57,30 @@ def test_router_backward_and_quantiser_bytes():
     assert bench.router_bwd_bytes(CFG) == T * per_token
     n = 128  # two blocks
     assert bench.quantize_bytes(n) == n * 2 + n // 2 + 2 * 4
+
+
+def _run_bench(extra_env, *args):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ, **extra_env)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], env=env, cwd=ROOT,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_prints_one_contract_line_on_rank_0_only():
+    args = ("--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1")
+    (line,) = _run_bench({"RANK": "0"}, *args)
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    for key in ("metric", "value", "n_gpus", "steps", "warmup", "ms_per_step", "scaling", "vs_baseline", "dtype",
+                "data", "config"):
+        assert key in line, key
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert "workload" in line["config"]
+    assert _run_bench({"RANK": "1"}, *args) == []   # other ranks exit 0 without work
