@@ -5,6 +5,13 @@ Every function here forwards to the entry point of the same name in
 are torch CUDA tensors (PyTorch supplies device memory and streams).  A
 non-OK status raises :class:`E4BError`.  There is no fallback: if the library
 is missing, :func:`lib` raises.
+
+The library sees raw device addresses only, so before each call the binding
+checks what the addresses cannot carry: every tensor is a contiguous CUDA
+tensor of the dtype the header names, on one device, holding at least the
+elements the call reads or writes (``TypeError`` / ``ValueError`` otherwise).
+Alignment, shapes the build refuses and workspace size are the library's own
+checks.
 """
 
 from __future__ import annotations
@@ -149,6 +156,62 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
+def _torch_dtype(name):
+    import torch
+    return {"bf16": torch.bfloat16, "f32": torch.float32, "i32": torch.int32, "u8": torch.uint8}[name]
+
+
+def _dev(t, dtype: str, min_numel: int, name: str, device=None, optional=None, where=True) -> Optional[int]:
+    """Device address of ``t`` after checking that it is a contiguous CUDA tensor of ``dtype``
+    holding at least ``min_numel`` elements (on ``device`` when given).  ``None`` passes where the
+    header allows NULL: by default where nothing is read or written (``min_numel == 0``)."""
+    import torch
+    if optional is None:
+        optional = min_numel == 0
+    if t is None:
+        if optional:
+            return None
+        raise ValueError("%s: a tensor is required" % name)
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s: expected a torch.Tensor, got %s" % (name, type(t).__name__))
+    if t.dtype != _torch_dtype(dtype):
+        raise TypeError("%s: dtype %s, expected %s" % (name, t.dtype, _torch_dtype(dtype)))
+    if not t.is_contiguous():
+        raise ValueError("%s: must be contiguous" % name)
+    if t.numel() < min_numel:
+        raise ValueError("%s: %d elements, the call needs %d" % (name, t.numel(), min_numel))
+    if not where:  # the caller checks the devices of all its tensors together (_one_cuda_device)
+        return _ptr(t)
+    if t.device.type != "cuda":
+        raise ValueError("%s: must be a CUDA tensor, got one on %s" % (name, t.device))
+    if device is not None and t.device != device:
+        raise ValueError("%s: on %s, expected %s" % (name, t.device, device))
+    return _ptr(t)
+
+
+def _numel_of(t, name: str) -> int:
+    import torch
+    if t is None:
+        raise ValueError("%s: a tensor is required" % name)
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s: expected a torch.Tensor, got %s" % (name, type(t).__name__))
+    return t.numel()
+
+
+def _one_cuda_device(**tensors):
+    """The one CUDA device that all the given tensors are on (None entries are skipped)."""
+    devs = set()
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if t.device.type != "cuda":
+            raise ValueError("%s: must be a CUDA tensor, got one on %s" % (name, t.device))
+        devs.add(t.device)
+    if len(devs) > 1:
+        raise ValueError("tensors on several devices: %s" % sorted(str(d) for d in devs))
+    return devs.pop() if devs else None
+
+
 @dataclass(frozen=True)
 class Dims:
     E: int
@@ -176,27 +239,38 @@ def e4b_nf4_levels():
 
 
 def e4b_workspace_init(ws, stream=None):
-    _check(lib().e4b_workspace_init(_ptr(ws), ws.numel(), _stream(stream)), "e4b_workspace_init")
+    p = _dev(ws, "u8", 1, "ws")
+    _check(lib().e4b_workspace_init(p, ws.numel(), _stream(stream)), "e4b_workspace_init")
 
 
 def e4b_check_device_error(ws, stream=None) -> int:
     """Synchronises the stream; returns the status (does not raise)."""
-    return lib().e4b_check_device_error(_ptr(ws), _stream(stream))
+    return lib().e4b_check_device_error(_dev(ws, "u8", 1, "ws"), _stream(stream))
 
 
 def e4b_nf4_dequant(packed, absmax, out, stream=None):
-    _check(lib().e4b_nf4_dequant(_ptr(packed), _ptr(absmax), out.numel(), _ptr(out), _stream(stream)),
-           "e4b_nf4_dequant")
+    """packed NF4 codes [n/2] u8 and absmax [n/64] f32 -> bf16 [n] (n = out.numel())."""
+    n = _numel_of(out, "out")
+    pp = _dev(packed, "u8", n // 2, "packed", where=False)
+    pa = _dev(absmax, "f32", n // 64, "absmax", where=False)
+    po = _dev(out, "bf16", 0, "out", optional=False, where=False)
+    _one_cuda_device(packed=packed, absmax=absmax, out=out)
+    _check(lib().e4b_nf4_dequant(pp, pa, n, po, _stream(stream)), "e4b_nf4_dequant")
 
 
 def e4b_nf4_quantize(w, packed, absmax, stream=None):
     """bf16 weights (n elements, n % 64 == 0) -> packed NF4 codes [n/2] u8 and absmax [n/64] f32."""
-    _check(lib().e4b_nf4_quantize(_ptr(w), w.numel(), _ptr(packed), _ptr(absmax), _stream(stream)),
-           "e4b_nf4_quantize")
+    n = _numel_of(w, "w")
+    pp = _dev(packed, "u8", n // 2, "packed", where=False)
+    pa = _dev(absmax, "f32", n // 64, "absmax", where=False)
+    pw = _dev(w, "bf16", 0, "w", optional=False, where=False)
+    _one_cuda_device(w=w, packed=packed, absmax=absmax)
+    _check(lib().e4b_nf4_quantize(pw, n, pp, pa, _stream(stream)), "e4b_nf4_quantize")
 
 
 def e4b_debug_watchdog(ws, timeout_ns: int, stream=None):
-    _check(lib().e4b_debug_watchdog(_ptr(ws), ws.numel(), int(timeout_ns), _stream(stream)), "e4b_debug_watchdog")
+    p = _dev(ws, "u8", 1, "ws")
+    _check(lib().e4b_debug_watchdog(p, ws.numel(), int(timeout_ns), _stream(stream)), "e4b_debug_watchdog")
 
 
 def e4b_profiler_enable(on: bool):
@@ -226,7 +300,10 @@ class Block:
 
     def __init__(self, dims: Dims, T: int, device="cuda"):
         import torch
-        self.dims, self.T, self.device = dims, T, torch.device(device)
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.dims, self.T, self.device = dims, T, dev
         sz = e4b_get_sizes(dims, T)
         self.sizes = sz
         E, H, I, k, r = dims.E, dims.H, dims.I, dims.top_k, dims.r
@@ -261,31 +338,58 @@ class Block:
                                     self.p_d.data_ptr(), self.y_perm.data_ptr())
         self._bwd = BwdBuffers(*(t.data_ptr() for t in (self.dyw, self.q_d, self.dgu, self.q_gu, self.dx_perm)))
 
+    # -- argument checks (see the module docstring) ----------------------------
+    def _rows(self, t, dtype, cols, name, required=True):
+        """A [T, cols] token tensor of this problem (at least T * cols elements)."""
+        return _dev(t, dtype, self.T * cols, name, self.device, optional=not required or self.T == 0)
+
+    def _base(self, base: Nf4Experts):
+        """The NF4 base struct; when made by :func:`nf4_experts`, its sizes and device are checked
+        against this problem."""
+        d = self.dims
+        need = {"gate_up_nf4": d.E * 2 * d.I * d.H // 2, "gate_up_absmax": d.E * 2 * d.I * d.H // 64,
+                "down_nf4": d.E * d.H * d.I // 2, "down_absmax": d.E * d.H * d.I // 64}
+        _check_struct(base, need, self.device, "base")
+        return ctypes.byref(base)
+
+    def _lora(self, lora: Lora):
+        d = self.dims
+        need = {"A_gu": d.E * d.r * d.H, "B_gu": d.E * 2 * d.I * d.r, "A_d": d.E * d.r * d.I,
+                "B_d": d.E * d.H * d.r}
+        _check_struct(lora, need, self.device, "lora")
+        return ctypes.byref(lora)
+
     # -- the four hot-path calls -------------------------------------------------
     def e4b_route_permute(self, logits, x, gather=True, stream=None):
         """Routing tables; with ``gather`` also ``x_perm`` (else the forward gathers, given ``x``)."""
-        _check(lib().e4b_route_permute(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
+        pl = self._rows(logits, "f32", self.dims.E, "logits")
+        px = self._rows(x, "bf16", self.dims.H, "x", required=gather)
+        _check(lib().e4b_route_permute(ctypes.byref(self._dims_c), self.T, pl, px,
                                        ctypes.byref(self._routing), _ptr(self.x_perm) if gather else None,
                                        _ptr(self.ws), self.ws.numel(), _stream(stream)), "e4b_route_permute")
 
     def e4b_route_permute_noalloc(self, logits, x, gather=True, stream=None):
         """As ``e4b_route_permute``, with the library's fixed scratch instead of ``ws`` (capturable in
         a global-mode CUDA graph once a first call on the device has been made)."""
-        _check(lib().e4b_route_permute_noalloc(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
+        pl = self._rows(logits, "f32", self.dims.E, "logits")
+        px = self._rows(x, "bf16", self.dims.H, "x", required=gather)
+        _check(lib().e4b_route_permute_noalloc(ctypes.byref(self._dims_c), self.T, pl, px,
                                                ctypes.byref(self._routing), _ptr(self.x_perm) if gather else None,
                                                _stream(stream)), "e4b_route_permute_noalloc")
 
     def e4b_grouped_nf4_lora_fwd(self, base: Nf4Experts, lora: Lora, x=None, stream=None):
         """Forward; with ``x`` the call also writes ``x_perm`` (fused with the first projection)."""
+        px = self._rows(x, "bf16", self.dims.H, "x", required=False)
         _check(lib().e4b_grouped_nf4_lora_fwd(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
-                                              ctypes.byref(base), ctypes.byref(lora), _ptr(x),
+                                              self._base(base), self._lora(lora), px,
                                               ctypes.byref(self._fwd), _ptr(self.y), _ptr(self.ws),
                                               self.ws.numel(), _stream(stream)), "e4b_grouped_nf4_lora_fwd")
 
     def e4b_grouped_nf4_lora_dgrad(self, base: Nf4Experts, lora: Lora, dY, stream=None):
+        pdy = self._rows(dY, "bf16", self.dims.H, "dY")
         _check(lib().e4b_grouped_nf4_lora_dgrad(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
-                                                ctypes.byref(base), ctypes.byref(lora), ctypes.byref(self._fwd),
-                                                _ptr(dY), ctypes.byref(self._bwd), _ptr(self.dx), _ptr(self.ws),
+                                                self._base(base), self._lora(lora), ctypes.byref(self._fwd),
+                                                pdy, ctypes.byref(self._bwd), _ptr(self.dx), _ptr(self.ws),
                                                 self.ws.numel(), _stream(stream)), "e4b_grouped_nf4_lora_dgrad")
 
     def e4b_lora_wgrad(self, stream=None):
@@ -298,24 +402,55 @@ class Block:
         """Routing + forward for inference into ``self.y``.  ``keep_gu=False`` passes no gu buffer
         (allowed for decode-sized batches only; larger ones are refused without it)."""
         fwd = self._fwd if keep_gu else self._fwd_nogu
-        _check(lib().e4b_moe_serve_fwd(ctypes.byref(self._dims_c), self.T, _ptr(logits), _ptr(x),
-                                       ctypes.byref(self._routing), ctypes.byref(base), ctypes.byref(lora),
+        pl = self._rows(logits, "f32", self.dims.E, "logits")
+        px = self._rows(x, "bf16", self.dims.H, "x")
+        _check(lib().e4b_moe_serve_fwd(ctypes.byref(self._dims_c), self.T, pl, px,
+                                       ctypes.byref(self._routing), self._base(base), self._lora(lora),
                                        ctypes.byref(fwd), _ptr(self.y), _ptr(self.ws), self.ws.numel(),
                                        _stream(stream)), "e4b_moe_serve_fwd")
 
     def e4b_router_backward(self, dY, d_logits, dw=None, stream=None):
+        pdy = self._rows(dY, "bf16", self.dims.H, "dY")
+        pdl = self._rows(d_logits, "f32", self.dims.E, "d_logits")
+        pdw = self._rows(dw, "f32", self.dims.top_k, "dw", required=False)
         _check(lib().e4b_router_backward(ctypes.byref(self._dims_c), self.T, ctypes.byref(self._routing),
-                                         _ptr(self.y_perm), _ptr(dY), _ptr(d_logits), _ptr(dw), _stream(stream)),
+                                         _ptr(self.y_perm), pdy, pdl, pdw, _stream(stream)),
                "e4b_router_backward")
 
     def check_device_error(self, stream=None) -> int:
         return e4b_check_device_error(self.ws, stream)
 
 
+def _make_struct(cls, tensors, dtypes):
+    """A pointer struct over contiguous CUDA tensors on one device.  The struct keeps the tensors
+    alive (it holds their raw addresses) and records their sizes for the calls' checks."""
+    names = [f[0] for f in cls._fields_]
+    st = cls(*(_dev(t, dt, 1, n, where=False) for t, dt, n in zip(tensors, dtypes, names)))
+    dev = _one_cuda_device(**dict(zip(names, tensors)))
+    st._keep, st._device = tuple(tensors), dev
+    st._numel = {n: t.numel() for n, t in zip(names, tensors)}
+    return st
+
+
+def _check_struct(st, need, device, what):
+    """Sizes and device of a struct made by :func:`nf4_experts` / :func:`lora_factors` against a
+    problem (a struct built field by field carries no sizes and is passed as is)."""
+    numel = getattr(st, "_numel", None)
+    if numel is None:
+        return
+    if st._device != device:
+        raise ValueError("%s: tensors on %s, the problem is on %s" % (what, st._device, device))
+    for name, n in need.items():
+        if numel[name] < n:
+            raise ValueError("%s.%s: %d elements, the dims need %d" % (what, name, numel[name], n))
+
+
 def nf4_experts(gate_up_nf4, gate_up_absmax, down_nf4, down_absmax) -> Nf4Experts:
-    return Nf4Experts(gate_up_nf4.data_ptr(), gate_up_absmax.data_ptr(), down_nf4.data_ptr(),
-                      down_absmax.data_ptr())
+    """The frozen NF4 base: codes u8 [E,2I,H/2] and [E,H,I/2], block absmax f32 [E,2I,H/64] and
+    [E,H,I/64]."""
+    return _make_struct(Nf4Experts, (gate_up_nf4, gate_up_absmax, down_nf4, down_absmax), ("u8", "f32", "u8", "f32"))
 
 
 def lora_factors(A_gu, B_gu, A_d, B_d) -> Lora:
-    return Lora(A_gu.data_ptr(), B_gu.data_ptr(), A_d.data_ptr(), B_d.data_ptr())
+    """The per-expert LoRA factors, bf16 [E,r,H], [E,2I,r], [E,r,I], [E,H,r]."""
+    return _make_struct(Lora, (A_gu, B_gu, A_d, B_d), ("bf16",) * 4)

@@ -187,3 +187,43 @@ def test_binding_pointer_of_empty_views_is_their_storage_address():
     assert e4b._ptr(buf[16:16]) == buf.data_ptr() + 16 * 4
     assert e4b._ptr(buf[4:]) == buf.data_ptr() + 16
     assert e4b._ptr(None) is None
+
+
+def test_binding_checks_tensors_before_calling_the_library():
+    # The binding refuses what raw addresses cannot carry (dtype, layout, size, device) before any
+    # library call; CPU tensors exercise every check up to the device one.
+    import torch
+    n = 256
+    packed = torch.zeros(n // 2, dtype=torch.uint8)
+    absmax = torch.zeros(n // 64, dtype=torch.float32)
+    out = torch.zeros(n, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="out: dtype"):
+        e4b.e4b_nf4_dequant(packed, absmax, out.float())
+    with pytest.raises(ValueError, match="packed: 64 elements, the call needs 128"):
+        e4b.e4b_nf4_dequant(packed[:64], absmax, out)
+    with pytest.raises(ValueError, match="absmax: must be contiguous"):
+        e4b.e4b_nf4_dequant(packed, torch.zeros(8, dtype=torch.float32)[::2], out)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        e4b.e4b_nf4_dequant(packed, absmax, out)
+    with pytest.raises(ValueError, match="w: a tensor is required"):
+        e4b.e4b_nf4_quantize(None, packed, absmax)
+    with pytest.raises(ValueError, match="absmax: 2 elements, the call needs 4"):
+        e4b.e4b_nf4_quantize(out, packed, absmax[:2])
+    with pytest.raises(TypeError, match="gate_up_nf4: dtype"):
+        e4b.nf4_experts(absmax, absmax, packed, absmax)
+    with pytest.raises(TypeError, match="expected a torch.Tensor"):
+        e4b.lora_factors(np.zeros(4), out, out, out)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        e4b.lora_factors(out, out, out, out)
+
+
+def test_binding_checks_struct_sizes_against_the_dims():
+    class Fake:  # what nf4_experts / lora_factors record
+        _device = "cuda:0"
+        _numel = {"A_gu": 100}
+    e4b._check_struct(Fake(), {"A_gu": 100}, "cuda:0", "lora")
+    with pytest.raises(ValueError, match="lora.A_gu: 100 elements, the dims need 101"):
+        e4b._check_struct(Fake(), {"A_gu": 101}, "cuda:0", "lora")
+    with pytest.raises(ValueError, match="on cuda:0, the problem is on cuda:1"):
+        e4b._check_struct(Fake(), {"A_gu": 1}, "cuda:1", "lora")
+    e4b._check_struct(e4b.Lora(), {"A_gu": 10 ** 9}, "cuda:0", "lora")  # built field by field: not checked
