@@ -316,7 +316,7 @@ def main():
     d = dv.upload(prob, dev)
     blk = e4b.Block(dv.dims_of(cfg), cfg.T, dev)
     base, lora = d.base(), d.lora()
-    grads = (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d)
+    grads = (blk.lora_grads,)  # dA_gu, dB_gu, dA_d, dB_d are views of this one buffer: one all-reduce
 
     fwd_only = cfg.passes == ("fwd",)  # decode-sized serving batch: the serving forward alone
 

@@ -325,8 +325,16 @@ class Block:
         self.dyw, self.q_d, self.dgu = z((R, H), bf), z((R, r), bf), z((R, 2 * I), bf)
         self.q_gu, self.dx_perm = z((R, r), bf), z((R, H), bf)
         self.y, self.dx = z((T, H), bf), z((T, H), bf)
-        self.dA_gu, self.dB_gu = z((E, r, H), bf), z((E, 2 * I, r), bf)
-        self.dA_d, self.dB_d = z((E, r, I), bf), z((E, H, r), bf)
+        # the four LoRA gradients are views of one flat buffer, so that a data-parallel step sums them
+        # with one collective and no packing copy (every size is a multiple of 8 elements: r % 8 == 0)
+        gshapes = ((E, r, H), (E, 2 * I, r), (E, r, I), (E, H, r))
+        gsizes = [a * b * c for a, b, c in gshapes]
+        self.lora_grads = z((sum(gsizes),), bf)
+        views, o = [], 0
+        for shp, n in zip(gshapes, gsizes):
+            views.append(self.lora_grads[o:o + n].view(*shp))
+            o += n
+        self.dA_gu, self.dB_gu, self.dA_d, self.dB_d = views
         self.ws = z((int(sz.workspace_bytes),), torch.uint8)
         e4b_workspace_init(self.ws)
         self._dims_c = dims.c()

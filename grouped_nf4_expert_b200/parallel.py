@@ -15,7 +15,9 @@ from __future__ import annotations
 
 
 def allreduce_lora_grads(grads, group=None):
-    """Sums each gradient tensor over all ranks of ``group``, in place."""
+    """Sums each gradient tensor over all ranks of ``group``, in place.  A
+    :class:`~grouped_nf4_expert_b200.e4b.Block` holds its four LoRA gradients as views of one flat
+    buffer (``Block.lora_grads``): passing that buffer sums all four in one collective."""
     import torch.distributed as dist
     for g in grads:
         dist.all_reduce(g, op=dist.ReduceOp.SUM, group=group)

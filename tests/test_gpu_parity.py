@@ -397,6 +397,19 @@ def test_binding_refuses_mismatched_tensors_before_any_launch():
     assert e4b.e4b_launch_count() == n0
 
 
+def test_lora_gradients_are_views_of_one_flat_buffer():
+    # a data-parallel step reduces the four gradients with one collective over this buffer
+    cfg = inputs.CONFIGS["train"]
+    blk = e4b.Block(dv.dims_of(cfg), 1)
+    grads = (blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d)
+    addr = blk.lora_grads.data_ptr()
+    for g in grads:
+        assert g.is_contiguous() and g.data_ptr() % 16 == 0
+        assert g.data_ptr() == addr
+        addr += g.numel() * 2
+    assert addr == blk.lora_grads.data_ptr() + blk.lora_grads.numel() * 2
+
+
 def test_watchdog_times_out_cleanly_and_context_survives():
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     e4b.e4b_workspace_init(ws)
