@@ -165,6 +165,14 @@ LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : name_(name), s
   g_launches.fetch_add(1, std::memory_order_relaxed);
   std::lock_guard<std::mutex> lock(g_prof_mu);
   if (!g_prof_on) return;
+  // A launch being captured into a CUDA graph is counted but not timed: its
+  // events would only be recorded when the graph replays.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream_, &capture) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return;
+  }
+  if (capture != cudaStreamCaptureStatusNone) return;
   std::pair<cudaEvent_t, cudaEvent_t> ev;
   if (!g_prof_pool.empty()) {
     ev = g_prof_pool.back();

@@ -319,7 +319,8 @@ e4b_status e4b_debug_watchdog(void *ws, size_t ws_bytes, int64_t timeout_ns, e4b
  * launches is bracketed by two CUDA events recorded on that launch's stream;
  * e4b_profiler_read waits for the recorded events, returns per-kernel launch
  * counts and summed device times, and clears the record.  Off by default; it
- * creates CUDA events (host handles), never device buffers. */
+ * creates CUDA events (host handles), never device buffers.  Launches made
+ * while their stream is being captured into a CUDA graph are not timed. */
 typedef struct {
   char name[48];      /* kernel (and mode) name */
   int64_t launches;   /* launches recorded */
