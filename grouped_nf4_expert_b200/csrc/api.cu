@@ -19,7 +19,7 @@ namespace e4b {
 namespace {
 
 constexpr int kMaxDevices = 64;
-int g_num_sms[kMaxDevices] = {0};
+std::atomic<int> g_num_sms[kMaxDevices] = {};  // per device, filled on first use (any host thread)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -28,13 +28,13 @@ cudaError_t device_sms(int* out) {
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (g_num_sms[dev] == 0) {
-    int n = 0;
+  int n = g_num_sms[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (err != cudaSuccess) return err;
-    g_num_sms[dev] = n;
+    g_num_sms[dev].store(n, std::memory_order_relaxed);
   }
-  *out = g_num_sms[dev];
+  *out = n;
   return cudaSuccess;
 }
 
