@@ -17,10 +17,10 @@
 //
 // Pages: "How do I QLoRA-train the fused experts of a MoE", section "The
 // abstraction that fails" (pre-activation per-expert delta over the fused
-// stacks), section "Why it happens" (scaling * (x @ A.T) @ B.T; the base is
-// re-dequantised in backward), section "Which project solves it" (grouped
-// forward and a dgrad kernel); package METADATA "The package family"
-// (in-register decode of 4-bit stacks, fp32 accumulation).
+// stacks), section "Why it happens" (scaling * (x @ A.T) @ B.T; the backward
+// decodes the 4-bit base again), section "Which project solves it" (grouped
+// forward and a dgrad kernel); package METADATA "The package family" (4-bit
+// codes decoded in registers, fp32 sums).
 #include <math.h>
 
 #include "e4b_device.cuh"

@@ -3,8 +3,8 @@
  * hand-written for NVIDIA B200 (sm_100a).
  *
  * The block is the routed-expert MoE layer over a frozen, NF4-quantised,
- * fused expert stack with a trainable low-rank delta per expert applied
- * before that expert's activation:
+ * fused expert stack; each expert carries a trainable low-rank delta that is
+ * added to its pre-activation (inside the activation, not after it):
  *
  *     y[t] = sum_j w[t,j] * yd(t, e = ids[t,j])
  *     gu   = W_gu[e] x + s * B_gu[e] (A_gu[e] x)         s = alpha / r
@@ -14,18 +14,19 @@
  * Sources (page title, section):
  *   "How do I QLoRA-train the fused experts of a MoE (per-expert LoRA on
  *   4-bit experts)?", section "The abstraction that fails, and what replaces
- *   it": the fused 3-D stacks gate_up_proj [E,2I,H] and down_proj [E,H,I];
- *   the delta act(W_e x + B[e] A[e] x) is applied per routed expert BEFORE
+ *   it": the fused 3-D stacks (gate_up_proj [E,2I,H], down_proj [E,H,I]);
+ *   each routed expert computes act(W_e x + B[e] A[e] x), the delta inside
  *   the activation; the base is frozen and B starts at zero.
  *   Same page, section "Why it happens": the LoRA term is
- *   scaling * (x @ A[e].T) @ B[e].T with stacked per-expert A and B; the base
- *   re-dequantises in backward, so no dequantised weight is ever stored.
+ *   scaling * (x @ A[e].T) @ B[e].T with stacked per-expert A and B; the
+ *   backward decodes the 4-bit base again, so no bf16 copy of a weight is
+ *   ever kept.
  *   Same page, sections "Which project solves it" and "Limitations": a
  *   grouped forward, an input-gradient (dgrad) kernel, the stock epilogue
  *   act(gate) * up, and loud refusal instead of a silent fallback.
- *   experts4bit-qlora package METADATA, section "The package family": one
- *   launch over 4-bit packed expert stacks, in-register decode, fp32
- *   accumulation.
+ *   experts4bit-qlora package METADATA, section "The package family": a
+ *   single kernel launch covers all the packed 4-bit experts, decoding in
+ *   registers and summing in fp32.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major
@@ -232,7 +233,7 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims *dims, int32_t T,
  * captured into a CUDA graph.
  * Pages: section "Which project solves it" (grouped forward), section
  * "Limitations" (the fast forward for inference) and METADATA "The package
- * family" (one launch over the packed stacks). */
+ * family" (a single launch covers all packed experts). */
 e4b_status e4b_moe_serve_fwd(const e4b_moe_dims *dims, int32_t T, const float *logits, const e4b_bf16 *x,
                              const e4b_routing *routing, const e4b_nf4_experts *base, const e4b_lora *lora,
                              const e4b_fwd_buffers *fwd, e4b_bf16 *y, void *ws, size_t ws_bytes,

@@ -12,14 +12,14 @@ Sources (page title, section):
 
 * "How do I QLoRA-train the fused experts of a MoE (per-expert LoRA on 4-bit
   experts)?" -- §"The abstraction that fails, and what replaces it" (fused
-  3-D stacks ``gate_up_proj [E,2I,H]``, ``down_proj [E,H,I]``; the delta is
-  applied per routed expert before the activation; B starts at zero; the
-  base is frozen), §"Why it happens" (the LoRA term is
-  ``scaling * (x @ A[e].T) @ B[e].T``; the base re-dequantises in backward;
-  the reference forward is a per-expert loop), §"Limitations" (the stock
-  epilogue ``act(gate) * up``).
-* experts4bit-qlora package METADATA -- §"The package family" (4-bit packed
-  expert stacks, decoded in-register, fp32 accumulation).
+  3-D stacks ``gate_up_proj [E,2I,H]``, ``down_proj [E,H,I]``; each routed
+  expert adds its delta inside its activation; B starts at zero; the base is
+  frozen), §"Why it happens" (the LoRA term is
+  ``scaling * (x @ A[e].T) @ B[e].T``; the backward decodes the 4-bit base
+  again; the method's plain forward visits the experts one at a time),
+  §"Limitations" (the stock epilogue ``act(gate) * up``).
+* experts4bit-qlora package METADATA -- §"The package family" (the experts
+  are stored as packed 4-bit stacks, decoded in registers, with fp32 sums).
 * The NF4 code book itself is not printed on those pages; it is the
   NormalFloat-4 data type of Dettmers et al., "QLoRA: Efficient Finetuning of
   Quantized LLMs" (2023), whose construction ``nf4_table`` restates.

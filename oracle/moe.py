@@ -1,9 +1,9 @@
 """Routed-expert MoE block over a frozen NF4 fused stack with per-expert LoRA.
 
 TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  Plain float64 numpy,
-written as the per-expert loop the pages describe as the method's own
-reference forward ("How do I QLoRA-train the fused experts of a MoE",
-§"Why it happens": "The reference forward is a per-expert loop by design").
+written as a loop over the experts, one at a time, which is how the pages
+say the method's own plain forward is built ("How do I QLoRA-train the fused
+experts of a MoE", §"Why it happens").
 
 What is computed (same page, §"The abstraction that fails, and what replaces
 it" and §"Why it happens"; readings where the pages are silent are marked):
@@ -26,7 +26,7 @@ it" and §"Why it happens"; readings where the pages are silent are marked):
   gradients ``dB_gu[e] += s dgu (A_gu[e] x)^T``, ``dA_gu[e] += s (B_gu[e]^T dgu) x^T``,
   ``dB_d[e] += s dyw (A_d[e] a)^T``, ``dA_d[e] += s (B_d[e]^T dyw) a^T``.
   The base weights are dequantised again in the backward (§"Why it
-  happens": the base re-dequantises in backward).
+  happens": the backward decodes the 4-bit base again).
 
 Pins (tests/test_oracle_moe.py): B = 0 gives exactly the base-only block;
 a per-token, per-expert brute-force loop; dense-delta equivalence with

@@ -6,9 +6,9 @@ Format, as the pages fix it and as read where they are silent:
 
 * 4-bit packed fused expert stacks, two codes per byte, one float32 absmax
   per block of 64 consecutive elements of a row (package METADATA,
-  §"The package family": "4-bit-packed expert stacks with in-register decode
-  and fp32 accumulation"; block size 64 and float32 absmax are the standard
-  bitsandbytes NF4 defaults).
+  §"The package family": the experts are packed 4-bit stacks, decoded in
+  registers and summed in fp32; block size 64 and float32 absmax are the
+  standard bitsandbytes NF4 defaults).
 * Reading (pages silent): element ``2m`` of a row is the HIGH nibble of byte
   ``m`` and element ``2m+1`` the LOW nibble.
 * Reading (pages silent): a block is 64 consecutive elements of one row of an
