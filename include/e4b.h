@@ -62,7 +62,7 @@ typedef uint16_t e4b_bf16;                 /* bfloat16 bit pattern */
 typedef enum {
   E4B_OK = 0,
   E4B_ERR_INVALID_ARG = 1,          /* null/misaligned pointer, negative size, inconsistent dims */
-  E4B_ERR_UNSUPPORTED = 2,          /* a shape, rank, block size or epilogue this build refuses */
+  E4B_ERR_UNSUPPORTED = 2,          /* a shape, rank, block size or epilogue the library refuses */
   E4B_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes < e4b_sizes.workspace_bytes */
   E4B_ERR_CUDA = 4,                 /* a CUDA runtime/driver call or a launch failed */
   E4B_ERR_DEVICE_TIMEOUT = 5        /* a device-side wait ran out (see e4b_check_device_error) */
