@@ -28,7 +28,10 @@ it" and §"Why it happens"; readings where the pages are silent are marked):
   The base weights are dequantised again in the backward (§"Why it
   happens": the backward decodes the 4-bit base again).
 
-Pins (tests/test_oracle_moe.py): B = 0 gives exactly the base-only block;
+Pins (tests/test_oracle_moe.py): the adapter layout consumed here (one A/B
+pair on the fused gate_up stack, one on down) reproduces the trainable-
+parameter counts the pages print for a real model (section "Measured
+result"); B = 0 gives exactly the base-only block;
 a per-token, per-expert brute-force loop; dense-delta equivalence with
 ``W + s B A`` materialised; E = 1, k = 1 against torch's SiLU, matmul and
 autograd; central finite differences of every gradient; routing against

@@ -306,3 +306,39 @@ def test_topk_softmax_backward_against_torch_autograd():
     assert np.array_equal(got["ids"], idx.numpy())
     assert np.allclose(got["d_logits"], lt.grad.numpy(), rtol=1e-12, atol=1e-13)
     assert np.allclose(got["dw"], dw.detach().numpy(), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- adapter layout (printed counts)
+
+def _golden_ints(name):
+    from conftest import golden_path
+    out = {}
+    for line in open(golden_path(name)):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            key, val = line.split()
+            out[key] = int(val)
+    return out
+
+
+def test_adapter_layout_matches_the_printed_trainable_parameter_counts():
+    # The pages print the trainable-parameter count of the per-expert adapter on a real model. The
+    # oracle's layout -- one A/B pair on the fused gate_up stack (A_gu [r, H], B_gu [2I, r]) and one on
+    # down (A_d [r, I], B_d [H, r]) -- must reproduce it; the oracle is run on those shapes so that
+    # the count is of the arrays it consumes.
+    g = _golden_ints("granite_trainable_params.txt")
+    r, L, H, I, E = g["rank"], g["layers"], g["hidden"], g["intermediate"], g["experts"]
+    q_out, kv_out = g["heads"] * g["head_dim"], g["kv_heads"] * g["head_dim"]
+    attention = L * r * ((H + q_out) + 2 * (H + kv_out) + (q_out + H))  # q, k, v, o
+    assert attention == g["attention_only"]
+    cfg = inputs.Config("granite_layer", E=E, H=H, I=I, top_k=8, T=2, r=r, alpha=16.0, routing="normal", seed=7)
+    prob = inputs.make_problem(cfg)
+    ex = _experts(prob)
+    out = oracle.moe_forward(inputs.bits_to_f32(prob.x).astype(np.float64), prob.logits, ex, cfg.top_k,
+                             cfg.alpha, tokens=[0])
+    assert np.isfinite(out["y"][0]).all()
+    per_layer = ex.A_gu.size + ex.B_gu.size + ex.A_d.size + ex.B_d.size
+    assert attention + L * per_layer == g["attention_and_experts"]
+    # layouts the count rules out: adapter on gate_up alone; separate gate and up adapters
+    assert attention + L * E * r * (H + 2 * I) != g["attention_and_experts"]
+    assert attention + L * E * r * (2 * (H + I) + (I + H)) != g["attention_and_experts"]
