@@ -22,7 +22,9 @@ Format, as the pages fix it and as read where they are silent:
 Pins (tests/test_oracle_nf4.py): the table against the values printed in the
 QLoRA paper's NF4 appendix and against its invariants; bf16 rounding against
 torch's float32->bfloat16 conversion; nibble order on hand-built bytes;
-quantise/dequantise round trip, brute-force argmin and error bound.
+quantise/dequantise round trip, brute-force argmin and error bound; the
+storage's bytes per weight against the size of a frozen stack the pages print
+(16.31 GB for a real model's expert stacks).
 """
 
 from __future__ import annotations

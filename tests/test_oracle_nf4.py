@@ -135,3 +135,29 @@ def test_quantise_zero_block_and_tie():
 def test_dequant_rejects_bad_absmax_shape(K):
     with pytest.raises(ValueError):
         oracle.dequantize_nf4(np.zeros((1, K // 2), np.uint8), np.zeros((1, K // 64 + 1), np.float32))
+
+
+def _golden_ints(name):
+    from conftest import golden_path
+    out = {}
+    for line in open(golden_path(name)):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            key, val = line.split()
+            out[key] = int(val)
+    return out
+
+
+def test_storage_layout_matches_the_printed_stack_size():
+    # The oracle's storage -- two codes per byte, one float32 absmax per 64 weights of a row -- applied to
+    # a real model's expert stacks gives the byte count the pages print (16.31 GB). Double-quantised
+    # scales or another block size would not.
+    g = _golden_ints("qwen3_nf4_stack_bytes.txt")
+    rng = np.random.default_rng(0)
+    K = 256
+    packed, absmax = oracle.quantize_nf4(rng.standard_normal((3, K)).astype(np.float32))
+    bytes_per_weight = (packed.nbytes + absmax.nbytes) / (3 * K)
+    weights = g["layers"] * g["experts"] * (2 * g["intermediate"] * g["hidden"] + g["hidden"] * g["intermediate"])
+    assert round(weights * bytes_per_weight / 1e7) == g["hashed_gb_x100"]
+    for alt in (0.5 + 4 / 32, 0.5 + 4 / 128, 0.5 + 1 / 64 + 4 / (64 * 256)):  # block 32, block 128, 8-bit scales
+        assert round(weights * alt / 1e7) != g["hashed_gb_x100"]
