@@ -29,6 +29,9 @@ MUTATIONS = [
     ("moe.py", 'order = np.argsort(-logits, axis=1, kind="stable")', 'order = np.argsort(logits, axis=1, kind="stable")[:, ::-1]'),
     ("moe.py", "w[t] * (dw[t] - float(np.dot(w[t], dw[t])))", "w[t] * dw[t]"),     # router: no softmax mean
     ("moe.py", "w[t] * (dw[t] - float(np.dot(w[t], dw[t])))", "(dw[t] - float(np.dot(w[t], dw[t])))"),
+    ("nf4.py", "BLOCK = 64", "BLOCK = 128"),                                          # block size
+    ("nf4.py", "absmax = np.abs(blocks).max(axis=-1).astype(np.float32)",
+     "absmax = np.abs(blocks).max(axis=-1).astype(np.float64)"),                     # scale precision
 ]
 
 
