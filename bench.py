@@ -89,17 +89,28 @@ def profiled_traffic():
 
 
 def step_flops(cfg):
-    """Algorithmic FLOPs of one step: routed slots only, 2 FLOP per MAC."""
+    """Algorithmic FLOPs of one step of the workload's passes (forward, input gradient, LoRA weight
+    gradients): routed slots only, 2 FLOP per MAC."""
     N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
-    base = 12.0 * N * H * I                  # fwd gate_up + down, dgrad down + gate_up
-    lora = 3 * 2.0 * N * r * (2 * H + 3 * I)  # projections and K=r products, fwd + dgrad + wgrad
-    return base + lora
+    lora = 2.0 * N * r * (2 * H + 3 * I)     # one pass's LoRA products (projections and K=r terms)
+    flops = 6.0 * N * H * I + lora           # forward: gate_up + down
+    if "dgrad" in cfg.passes:
+        flops += 6.0 * N * H * I + lora      # dgrad down + gate_up
+    if "wgrad" in cfg.passes:
+        flops += lora                        # the four weight-gradient products
+    return flops
 
 
 def fwd_flops(cfg):
     """Algorithmic FLOPs of the forward alone (gate_up, down and the forward LoRA terms)."""
     N, H, I, r = cfg.N, cfg.H, cfg.I, cfg.r
     return 6.0 * N * H * I + 2.0 * N * r * (2 * H + 3 * I)
+
+
+def nf4_gemm_flop_total(gflops, kern):
+    """FLOPs of the grouped NF4 GEMM launches the profiler recorded (each mode's work per launch times
+    its launches): the modes a workload does not run count nothing."""
+    return sum(f * kern[n][0] for n, f in gflops.items() if n in kern)
 
 
 def stream_bytes(cfg, touched):
@@ -318,18 +329,20 @@ def main():
     base, lora = d.base(), d.lora()
     grads = (blk.lora_grads,)  # dA_gu, dB_gu, dA_d, dB_d are views of this one buffer: one all-reduce
 
-    fwd_only = cfg.passes == ("fwd",)  # decode-sized serving batch: the serving forward alone
+    fwd_only = cfg.passes == ("fwd",)  # a forward-only workload: the serving forward alone
+    do_wgrad = "wgrad" in cfg.passes
 
     def step():
         if fwd_only:  # routing + forward for inference, nothing kept for a backward
-            blk.e4b_moe_serve_fwd(d.logits, d.x, base, lora, keep_gu=False)
+            blk.e4b_moe_serve_fwd(d.logits, d.x, base, lora)
             return
         blk.e4b_route_permute(d.logits, d.x, gather=False)  # the forward gathers x with its first projection
         blk.e4b_grouped_nf4_lora_fwd(base, lora, x=d.x)
         blk.e4b_grouped_nf4_lora_dgrad(base, lora, d.dY)
-        blk.e4b_lora_wgrad()
-        if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
-            parallel.allreduce_lora_grads(grads)
+        if do_wgrad:
+            blk.e4b_lora_wgrad()
+            if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
+                parallel.allreduce_lora_grads(grads)
 
     def sync_all():
         torch.cuda.synchronize(dev)
@@ -390,7 +403,7 @@ def main():
         raise RuntimeError("device error in the timed region: %s" % e4b.STATUS.get(st, st))
     ms_per_step = total_ms / args.steps
     value = cfg.T * world * args.steps / (total_ms / 1e3)
-    flops = fwd_flops(cfg) if fwd_only else step_flops(cfg)
+    flops = step_flops(cfg)
 
     # ---- per-kernel device times over a second timed region (library profiler, events on the launch stream)
     e4b.e4b_profiler_enable(True)
@@ -401,10 +414,11 @@ def main():
     gflops = nf4_gemm_flops(cfg)
     nf4_ms = sum(kern.get(n, (0, 0.0))[1] for n in gflops)
     nf4_launches = sum(kern.get(n, (0, 0.0))[0] for n in gflops)
-    nf4_flop = sum(gflops.values()) * args.steps
+    nf4_flop = nf4_gemm_flop_total(gflops, kern)
     achieved = nf4_flop / (nf4_ms / 1e3) / 1e12 if nf4_ms > 0 else None
     kern_total = sum(v[1] for v in kern.values())
-    roofline = {"kernel": "nf4_gemm (fwd gate_up, fwd down, dgrad down, dgrad gate_up)", "bound": "tensor",
+    modes = [n[len("nf4_gemm_"):].replace("_", " ", 1) for n in gflops if n in kern]
+    roofline = {"kernel": "nf4_gemm (%s)" % ", ".join(modes), "bound": "tensor",
                 "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
                 "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long step)" % peak_src,
@@ -412,7 +426,7 @@ def main():
                 "traffic_unit": "DRAM bytes per step of the four nf4_gemm launches (ncu)",
                 "launches": nf4_launches,
                 "avg_launch_ms": nf4_ms / max(nf4_launches, 1),
-                "algorithmic_flop_per_step": sum(gflops.values())}
+                "algorithmic_flop_per_step": nf4_flop / args.steps}
     sbytes = stream_bytes(cfg, int((blk.counts > 0).sum().item()))
     st_ms = sum(kern.get(n, (0, 0.0))[1] for n in sbytes)
     if st_ms > 0:  # the weight-streaming forward ran: it is HBM-bound by design
@@ -434,7 +448,7 @@ def main():
     hx.copy_(d.x)
     hl.copy_(d.logits)
     hdy.copy_(d.dY)
-    outs = [blk.y] if fwd_only else [blk.y, blk.dx, blk.dA_gu, blk.dB_gu, blk.dA_d, blk.dB_d]
+    outs = [blk.y] if fwd_only else [blk.y, blk.dx] + ([blk.lora_grads] if do_wgrad else [])
     houts = [pin(t) for t in outs]
     ins = (hx, hl) if fwd_only else (hx, hl, hdy)
     h2d = sum(t.numel() * t.element_size() for t in ins)
@@ -492,7 +506,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(cfg, world, "flushed between timed steps by a 256 MiB write"),
                        cuda_graph=fwd_only, call=("e4b_moe_serve_fwd" if fwd_only else
-                                                  "route_permute + lora_fwd + lora_dgrad + lora_wgrad")),
+                                                  "route_permute + lora_fwd + lora_dgrad" +
+                                                  (" + lora_wgrad" if do_wgrad else ""))),
         "tflops": flops * world / (ms_per_step / 1e3) / 1e12,
         "step_flop_per_gpu": flops,
         "roofline": roofline,

@@ -406,9 +406,12 @@ class Block:
                                     _ptr(self.dB_gu), _ptr(self.dA_d), _ptr(self.dB_d), _ptr(self.ws),
                                     self.ws.numel(), _stream(stream)), "e4b_lora_wgrad")
 
-    def e4b_moe_serve_fwd(self, logits, x, base: Nf4Experts, lora: Lora, keep_gu=True, stream=None):
-        """Routing + forward for inference into ``self.y``.  ``keep_gu=False`` passes no gu buffer
-        (allowed for decode-sized batches only; larger ones are refused without it)."""
+    def e4b_moe_serve_fwd(self, logits, x, base: Nf4Experts, lora: Lora, keep_gu=None, stream=None):
+        """Routing + forward for inference into ``self.y``.  ``keep_gu=False`` passes no gu buffer,
+        which the call allows for decode-sized batches only (at most 16 * E routed slots; larger ones
+        run the training forward, which writes gu); ``None`` keeps gu exactly when it is required."""
+        if keep_gu is None:
+            keep_gu = self.T * self.dims.top_k > 16 * self.dims.E
         fwd = self._fwd if keep_gu else self._fwd_nogu
         pl = self._rows(logits, "f32", self.dims.E, "logits")
         px = self._rows(x, "bf16", self.dims.H, "x")

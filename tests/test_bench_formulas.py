@@ -11,7 +11,8 @@ _spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "benc
 bench = importlib.util.module_from_spec(_spec)
 _spec.loader.exec_module(bench)
 
-CFG = inputs.Config("count", E=4, H=64, I=192, top_k=2, T=5, r=8, alpha=16.0, routing="normal", seed=1)
+CFG = inputs.Config("count", E=4, H=64, I=192, top_k=2, T=5, r=8, alpha=16.0, routing="normal", seed=1,
+                    passes=("fwd", "dgrad", "wgrad"))
 
 
 def _matmuls():
@@ -30,6 +31,19 @@ def test_step_flops_is_the_sum_of_the_step_matmuls():
     macs = sum(a * b * c for a, b, c in fwd + dgrad + wgrad) * CFG.N
     assert bench.step_flops(CFG) == 2 * macs
     assert bench.fwd_flops(CFG) == 2 * CFG.N * sum(a * b * c for a, b, c in fwd)
+    # workloads without some passes count only the passes they run
+    import dataclasses
+    fd = dataclasses.replace(CFG, passes=("fwd", "dgrad"))
+    assert bench.step_flops(fd) == 2 * CFG.N * sum(a * b * c for a, b, c in fwd + dgrad)
+    assert bench.step_flops(dataclasses.replace(CFG, passes=("fwd",))) == bench.fwd_flops(CFG)
+
+
+def test_gemm_flop_total_counts_only_the_launched_modes():
+    g = bench.nf4_gemm_flops(CFG)
+    kern = {"nf4_gemm_fwd_gate_up": (3, 1.0), "nf4_gemm_fwd_down": (3, 1.0), "combine_y": (3, 1.0)}
+    assert bench.nf4_gemm_flop_total(g, kern) == 3 * (g["nf4_gemm_fwd_gate_up"] + g["nf4_gemm_fwd_down"])
+    kern.update({"nf4_gemm_dgrad_down": (3, 1.0), "nf4_gemm_dgrad_gate_up": (3, 1.0)})
+    assert bench.nf4_gemm_flop_total(g, kern) == 3 * sum(g.values())
 
 
 def test_gemm_flops_cover_the_base_products_and_their_k_r_terms():
