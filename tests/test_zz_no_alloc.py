@@ -10,7 +10,7 @@ offsets, permutation and the permuted rows must be identical, and the routing
 weights within the parity tests' tolerance (they come out bit-identical).
 A third call writes the routing tables only (no permuted rows), through the
 binding.  It also checks that a problem too large for the fixed array is refused.
-This file is named to be collected last.
+This file is named to be collected after the main parity tests.
 """
 
 import ctypes

@@ -22,6 +22,7 @@ def _built():
     build.build()
     e4b.lib()
 
+
 TRAIN = inputs.Config("max_experts", E=1024, H=64, I=64, top_k=8, T=600, r=8, alpha=16.0, routing="zipf",
                       seed=61)
 SERVE = inputs.Config("max_experts_decode", E=1024, H=128, I=64, top_k=8, T=16, r=16, alpha=32.0,
