@@ -42,9 +42,17 @@ def _worker(rank, world, port, out_q):
     import torch.distributed as dist
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        grads = [torch.from_numpy(g.copy()) for g in _rank_grads(rank)]
+        mine = _rank_grads(rank)
+        grads = [torch.from_numpy(g.copy()) for g in mine]
         parallel.allreduce_lora_grads(grads)
-        out_q.put((rank, [g.numpy() for g in grads]))
+        # as the training step does it: the four gradients as views of one flat buffer, one collective
+        flat = torch.cat([torch.from_numpy(g).reshape(-1) for g in mine])
+        views, o = [], 0
+        for g in mine:
+            views.append(flat[o:o + g.size].view(g.shape))
+            o += g.size
+        parallel.allreduce_lora_grads([flat])
+        out_q.put((rank, [g.numpy() for g in grads], [v.numpy().copy() for v in views]))
     finally:
         dist.destroy_process_group()
 
@@ -63,7 +71,10 @@ def test_two_rank_allreduce_equals_union_batch():
     procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    results = dict(q.get(timeout=240) for _ in range(world))
+    results, flat_results = {}, {}
+    for _ in range(world):
+        rank, per_tensor, flat_views = q.get(timeout=240)
+        results[rank], flat_results[rank] = per_tensor, flat_views
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -77,7 +88,8 @@ def test_two_rank_allreduce_equals_union_batch():
     dY = inputs.bits_to_f32(union.dY).astype(np.float64)
     bo = oracle.moe_backward(x, union.logits, dY, _experts(union), CFG.top_k, CFG.alpha)
     for r in range(world):
-        for k, got in zip(KEYS, results[r]):
+        for k, got, got_flat in zip(KEYS, results[r], flat_results[r]):
             np.testing.assert_allclose(got, bo[k], rtol=1e-10, atol=1e-12)
+            np.testing.assert_array_equal(got_flat, got)
     # the ranks really had different batches
     assert not np.array_equal(pa.x, pb.x)
