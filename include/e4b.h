@@ -147,7 +147,9 @@ const char *e4b_status_string(e4b_status s);
 /* Library version string. */
 const char *e4b_version(void);
 
-/* The 16 NF4 levels the library decodes with (float32, ascending). */
+/* The 16 NF4 levels the library decodes with (float32, ascending): the
+ * NormalFloat-4 code book of the QLoRA paper (Dettmers et al., 2023), which
+ * the pages name as the default base format without printing it. */
 void e4b_nf4_levels(float out[16]);
 
 /* Buffer sizes for `dims` and T tokens.  Host only; no CUDA call. */
@@ -287,7 +289,12 @@ e4b_status e4b_router_backward(const e4b_moe_dims *dims, int32_t T, const e4b_ro
 
 /* Dequantises n NF4 elements (n a multiple of 64): packed uint8 [n/2],
  * absmax float32 [n/64] -> bf16 [n], with the same device routine the
- * grouped GEMMs decode with.  For bit-exact testing of the decode. */
+ * grouped GEMMs decode with.  For bit-exact testing of the decode.  Device
+ * pointers owned by the caller (packed and out 16-byte aligned, absmax 4-byte
+ * aligned); invalid sizes or alignment -> E4B_ERR_INVALID_ARG, no launch.
+ * Pages: experts4bit-qlora package METADATA, section "The package family"
+ * (the 4-bit codes decoded in registers); the element layout is the one
+ * e4b_nf4_experts states. */
 e4b_status e4b_nf4_dequant(const uint8_t *packed, const float *absmax, int64_t n, e4b_bf16 *out,
                            e4b_stream_t stream);
 
