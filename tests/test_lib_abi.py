@@ -227,3 +227,16 @@ def test_binding_checks_struct_sizes_against_the_dims():
     with pytest.raises(ValueError, match="on cuda:0, the problem is on cuda:1"):
         e4b._check_struct(Fake(), {"A_gu": 1}, "cuda:1", "lora")
     e4b._check_struct(e4b.Lora(), {"A_gu": 10 ** 9}, "cuda:0", "lora")  # built field by field: not checked
+
+
+def test_binding_signatures_match_the_header_prototypes():
+    # every prototype in include/e4b.h has a ctypes signature with the same number of arguments
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(e4b.HEADER).read(), flags=re.S)
+    protos = re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(e4b_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.M | re.S)
+    assert len(protos) == len(e4b.header_symbols())
+    for name, args in protos:
+        a = args.strip()
+        n = 0 if a in ("", "void") else a.count(",") + 1
+        assert name in e4b._SIGNATURES, name
+        assert len(e4b._SIGNATURES[name][1]) == n, name
