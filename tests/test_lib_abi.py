@@ -240,3 +240,22 @@ def test_binding_signatures_match_the_header_prototypes():
         n = 0 if a in ("", "void") else a.count(",") + 1
         assert name in e4b._SIGNATURES, name
         assert len(e4b._SIGNATURES[name][1]) == n, name
+
+
+def test_binding_structs_match_the_header_structs_field_by_field():
+    # a field out of order would hand the library one buffer in place of another
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(e4b.HEADER).read(), flags=re.S)
+    structs = {}
+    for body, name in re.findall(r"typedef\s+struct\s*\{(.*?)\}\s*(\w+)\s*;", text, flags=re.S):
+        fields = []
+        for decl in filter(None, (d.strip() for d in body.split(";"))):
+            decl = re.sub(r"\[[^\]]*\]", "", decl)
+            fields += [re.findall(r"\w+", part)[-1] for part in decl.split(",")]
+        structs[name] = fields
+    pairs = {"e4b_moe_dims": e4b.MoeDims, "e4b_nf4_experts": e4b.Nf4Experts, "e4b_lora": e4b.Lora,
+             "e4b_routing": e4b.Routing, "e4b_fwd_buffers": e4b.FwdBuffers, "e4b_bwd_buffers": e4b.BwdBuffers,
+             "e4b_sizes": e4b.Sizes, "e4b_kernel_time": e4b.KernelTime}
+    assert set(structs) == set(pairs)
+    for cname, cls in pairs.items():
+        assert [f[0] for f in cls._fields_] == structs[cname], cname
