@@ -6,6 +6,7 @@ prototypes compile as C, the enum values and struct layouts are what the binding
 argument checks return their statuses through a plain C call.
 """
 
+import ctypes
 import os
 import shutil
 import subprocess
@@ -13,6 +14,7 @@ import subprocess
 import pytest
 
 from grouped_nf4_expert_b200 import build as e4b_build
+from grouped_nf4_expert_b200 import e4b
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 INCLUDE = os.path.join(ROOT, "include")
@@ -57,6 +59,9 @@ int main(void) {
   CHECK(sizeof(e4b_routing) == 7 * sizeof(void *) && sizeof(e4b_fwd_buffers) == 6 * sizeof(void *));
   CHECK(sizeof(e4b_bwd_buffers) == 5 * sizeof(void *) && sizeof(e4b_sizes) == 32);
   CHECK(sizeof(e4b_kernel_time) == 64);
+  printf("SIZES %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(e4b_moe_dims), sizeof(e4b_nf4_experts),
+         sizeof(e4b_lora), sizeof(e4b_routing), sizeof(e4b_fwd_buffers), sizeof(e4b_bwd_buffers),
+         sizeof(e4b_sizes), sizeof(e4b_kernel_time));
   printf("OK\n");
   return 0;
 }
@@ -75,7 +80,13 @@ def _compile_and_run(tmp_path, compiler, std, ext):
     r = subprocess.run(cmd, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(out)], capture_output=True, text=True, timeout=120)
-    assert r.returncode == 0 and r.stdout.strip() == "OK", r.stdout + r.stderr
+    lines = r.stdout.split("\n")
+    assert r.returncode == 0 and lines[-2] == "OK", r.stdout + r.stderr
+    # the ctypes binding lays the structs out as the C compiler does
+    sizes = [int(v) for v in lines[-3].split()[1:]]
+    classes = [e4b.MoeDims, e4b.Nf4Experts, e4b.Lora, e4b.Routing, e4b.FwdBuffers, e4b.BwdBuffers, e4b.Sizes,
+               e4b.KernelTime]
+    assert sizes == [ctypes.sizeof(c) for c in classes]
 
 
 @pytest.fixture(scope="module", autouse=True)
