@@ -259,3 +259,34 @@ def test_binding_structs_match_the_header_structs_field_by_field():
     assert set(structs) == set(pairs)
     for cname, cls in pairs.items():
         assert [f[0] for f in cls._fields_] == structs[cname], cname
+
+
+def test_buffer_capacities_hold_every_routing_outcome(so):
+    # rows_cap and tiles_cap (e4b_get_sizes) must hold the padded groups and the three device work lists
+    # for ANY split of the N slots over the E experts; the worst splits leave one slot over a tile edge
+    # in as many experts as possible.  Work-list layout: an 8-int header, 2 ints per 128-row m-tile,
+    # E ints of expert order, 3 per 256-row m-unit and 3 per 32-slot streaming tile, the m-unit and
+    # streaming regions sized 3 and 12 ints per m-tile of capacity.
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        E = int(rng.integers(1, 1025))
+        k = int(rng.integers(1, min(E, 32) + 1))
+        T = int(rng.integers(0, 5000))
+        N = T * k
+        d = e4b.Dims(E=E, H=64, I=64, top_k=k, r=8, alpha=16.0)
+        s = e4b.e4b_get_sizes(d, T)
+        mt_cap = (s.tiles_cap - 8 - E) // 17
+        assert s.tiles_cap == 8 + 17 * mt_cap + E
+        splits = [rng.multinomial(N, np.ones(E) / E)]
+        worst = np.zeros(E, dtype=np.int64)   # as many experts as possible hold 1 slot past an edge
+        m = min(E, N)
+        worst[:m] = 1
+        worst[0] += N - m
+        splits.append(worst)
+        for c in splits:
+            assert c.sum() == N
+            mt = int(((c + 127) // 128).sum())
+            mu = int((((c + 127) // 128 + 1) // 2).sum())
+            st = int(((c + 31) // 32).sum())
+            assert int(((c + 127) // 128 * 128).sum()) <= s.rows_cap
+            assert mt <= mt_cap and mu <= mt_cap and st <= 4 * mt_cap
