@@ -290,3 +290,13 @@ def test_buffer_capacities_hold_every_routing_outcome(so):
             st = int(((c + 31) // 32).sum())
             assert int(((c + 127) // 128 * 128).sum()) <= s.rows_cap
             assert mt <= mt_cap and mu <= mt_cap and st <= 4 * mt_cap
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch):
+    # no fallback: with libe4b.so absent the binding raises instead of computing anything elsewhere
+    monkeypatch.setattr(e4b, "_LIB", None)
+    monkeypatch.setattr(e4b, "LIB_PATH", e4b.LIB_PATH + ".missing")
+    with pytest.raises(RuntimeError, match="not built"):
+        e4b.lib()
+    with pytest.raises(RuntimeError, match="not built"):
+        e4b.e4b_get_sizes(e4b.Dims(E=4, H=64, I=64, top_k=2, r=8, alpha=16.0), 8)
