@@ -392,18 +392,85 @@ def _sample_tokens(T, n, seed):
     return np.sort(np.random.default_rng(seed).choice(T, size=n, replace=False))
 
 
-@pytest.mark.parametrize("name,ntok", [("finegrained", 24), ("train", 16)])
-def test_workload_fwd_dgrad_sampled_tokens(name, ntok):
+def _unit_covering_slots(prob, seed):
+    """Routed slots chosen so that every work unit of the GPU path holds one of them.
+
+    From the oracle's own routing: the slots of each expert in grouped
+    (stable) order, one random slot from each 128-row tile of the expert's
+    group (each 256-row unit of the grouped GEMM therefore holds two, a
+    128-row tail unit one) and the expert's last slot (the ragged end of its
+    group).  Every expert with a routed slot contributes.
+    """
+    cfg = prob.cfg
+    ids, _ = oracle.route_topk(prob.logits, cfg.top_k)
+    g = oracle.group_by_expert(ids, cfg.E)
+    rng = np.random.default_rng(seed)
+    chosen = set()
+    for e in range(cfg.E):
+        cnt = int(g["counts"][e])
+        if cnt == 0:
+            continue
+        members = g["slots"][g["starts"][e]:g["starts"][e] + cnt]
+        for lo in range(0, cnt, 128):
+            chosen.add(int(members[rng.integers(lo, min(cnt, lo + 128))]))
+        chosen.add(int(members[cnt - 1]))
+    return np.array(sorted(chosen), dtype=np.int64)
+
+
+def _per_row_err(gpu_rows, ref_rows):
+    """max over rows of max|gpu - oracle| / max|oracle| within the row (a row that is exactly zero in
+    the oracle must be exactly zero on the GPU)."""
+    gpu_rows = np.asarray(gpu_rows, np.float64)
+    ref_rows = np.asarray(ref_rows, np.float64)
+    assert gpu_rows.shape == ref_rows.shape
+    m = np.abs(ref_rows).max(axis=1)
+    d = np.abs(gpu_rows - ref_rows).max(axis=1)
+    err = np.where(m > 0, d / np.where(m > 0, m, 1.0), np.where(d == 0, 0.0, np.inf))
+    return float(err.max()), int(err.argmax())
+
+
+def _check_slots(blk, cfg, slots, fo, bo=None, dY=None):
+    """Per-slot intermediates of the sampled slots, row by row, and the block outputs of their tokens."""
+    ros = blk.row_of_slot.cpu().numpy().astype(np.int64)
+    rows = torch.from_numpy(ros[slots]).cuda()
+    s = cfg.alpha / cfg.r
+    toks = np.unique(slots // cfg.top_k)
+    errs = {}
+    pick = lambda buf: f64(buf[rows])  # noqa: E731
+    for key, buf, scale in [("gu", blk.gu, 1.0), ("act", blk.act, 1.0), ("p_gu", blk.p_gu, s),
+                            ("p_d", blk.p_d, s), ("y_perm", blk.y_perm, 1.0)]:
+        okey = "yd" if key == "y_perm" else key
+        errs[key] = _per_row_err(pick(buf), np.stack([fo[okey][int(f)] for f in slots]) * scale)
+    errs["y"] = _per_row_err(f64(blk.y)[toks], fo["y"][toks])
+    if bo is not None:
+        w = bo["w"].reshape(-1)
+        errs["dyw"] = _per_row_err(pick(blk.dyw), w[slots, None] * dY[slots // cfg.top_k])
+        for key, buf, scale in [("dgu", blk.dgu, 1.0), ("q_gu", blk.q_gu, s), ("q_d", blk.q_d, s),
+                                ("dx_perm", blk.dx_perm, 1.0)]:
+            okey = "dx_slot" if key == "dx_perm" else key
+            errs[key] = _per_row_err(pick(buf), np.stack([bo[okey][int(f)] for f in slots]) * scale)
+        errs["dx"] = _per_row_err(f64(blk.dx)[toks], bo["dx"][toks])
+    bad = {k: v for k, v in errs.items() if not v[0] <= TOL}
+    assert not bad, ("(max row error, sampled row index)", bad, errs)
+
+
+@pytest.mark.parametrize("name", ["finegrained", "train"])
+def test_workload_fwd_dgrad_every_unit_sampled(name):
+    # Full size (E128 H2048 I768 top-8, 8192 tokens, Zipf routing): one slot of every 128-row tile of
+    # every expert's group and each group's last slot, so a wrong work unit of any kernel (a heavy
+    # expert's 29th unit, a 128-row tail unit, the lightest expert) fails; checked row by row.
     cfg = inputs.CONFIGS[name]
     prob, _, blk = run(cfg, wgrad=False)
+    slots = _unit_covering_slots(prob, 100)
     ex = oracle_experts(prob)
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
     dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
-    toks = _sample_tokens(cfg.T, ntok, 100)
+    toks = np.unique(slots // cfg.top_k)
     fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=toks)
     bo = oracle.moe_backward(x, prob.logits, dY, ex, cfg.top_k, cfg.alpha, tokens=toks, grad_experts=[])
-    assert rel_err(f64(blk.y)[toks], fo["y"][toks]) <= TOL
-    assert rel_err(f64(blk.dx)[toks], bo["dx"][toks]) <= TOL
+    ids = oracle.route_topk(prob.logits, cfg.top_k)[0].reshape(-1)
+    assert set(ids[slots].tolist()) == set(np.flatnonzero(blk.counts.cpu().numpy()).tolist())
+    _check_slots(blk, cfg, slots, fo, bo, dY)
 
 
 def test_train_workload_wgrad_sampled_experts():
@@ -412,7 +479,10 @@ def test_train_workload_wgrad_sampled_experts():
     counts = blk.counts.cpu().numpy()
     order = np.argsort(-counts, kind="stable")
     nz = order[counts[order] > 0]
-    experts = sorted({int(nz[0]), int(nz[len(nz) // 2]), int(nz[-1])})
+    # the heaviest, the median and the lightest expert, and five more at random
+    rng = np.random.default_rng(104)
+    experts = sorted({int(nz[0]), int(nz[len(nz) // 2]), int(nz[-1])} |
+                     set(int(e) for e in rng.choice(nz, 5, replace=False)))
     ex = oracle_experts(prob)
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
     dY = inputs.bits_to_f32(prob.dY).astype(np.float64)
@@ -423,22 +493,26 @@ def test_train_workload_wgrad_sampled_experts():
 
 
 def test_decode_workload_full():
+    # every routed slot of the decode batch, row by row (the weight-streaming forward)
     cfg = inputs.CONFIGS["decode"]
     prob, _, blk = run(cfg, dgrad=False, wgrad=False)
     ex = oracle_experts(prob)
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
     fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha)
     assert rel_err(f64(blk.y), fo["y"]) <= TOL
+    _check_slots(blk, cfg, np.arange(cfg.T * cfg.top_k), fo)
 
 
-def test_mixtral_workload_forward_sampled_tokens():
+def test_mixtral_workload_forward_every_unit_sampled():
+    # E8 H4096 I14336 top-2, 4096 tokens (the largest groups): one slot of every 128-row tile of each
+    # expert's group and each group's last slot, checked row by row (gu, act, p, y_perm, y).
     cfg = inputs.CONFIGS["mixtral"]
     prob, _, blk = run(cfg, dgrad=False, wgrad=False)
-    toks = _sample_tokens(cfg.T, 6, 101)
+    slots = _unit_covering_slots(prob, 101)
     ex = oracle_experts(prob)
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
-    fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=toks)
-    assert rel_err(f64(blk.y)[toks], fo["y"][toks]) <= TOL
+    fo = oracle.moe_forward(x, prob.logits, ex, cfg.top_k, cfg.alpha, tokens=np.unique(slots // cfg.top_k))
+    _check_slots(blk, cfg, slots, fo)
 
 
 @pytest.mark.parametrize("name", ["finegrained", "train", "decode"])
