@@ -49,6 +49,8 @@ def parse_args():
                     help="tokens of the oracle's cpu_baseline sample")
     ap.add_argument("--ref-tokens", type=int, default=1, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sub-workloads", default=",".join(SUB_WORKLOADS),
+                    help="comma-separated workloads timed beside the headline one (1 GPU); '' for none")
     return ap.parse_args()
 
 
@@ -119,6 +121,12 @@ def stream_bytes(cfg, touched):
     per_weight = 0.5 + 4.0 / 64
     return {"nf4_stream_fwd_gate_up": touched * 2 * cfg.I * cfg.H * per_weight,
             "nf4_stream_fwd_down": touched * cfg.H * cfg.I * per_weight}
+
+
+def serve_bytes(cfg, touched):
+    """Algorithmic HBM bytes of the one-launch serving forward: the NF4 codes and fp32 block scales
+    of both stacks of every expert the batch routes to, each read once."""
+    return {"nf4_serve": sum(stream_bytes(cfg, touched).values())}
 
 
 def router_bwd_bytes(cfg):
@@ -297,32 +305,98 @@ def workload_config(cfg, world, l2_note):
 
 # --------------------------------------------------------------------------- GPU arm
 
-def main():
-    args = parse_args()
-    if args.impl == "reference":
-        return run_reference(args)
+# Workloads measured beside the headline one in the same run (each its own passes, timed the same way).
+SUB_WORKLOADS = ("mixtral", "finegrained", "decode", "tiny")
+# Oracle sample per workload for its cpu_baseline: tokens, chosen so each takes seconds on host cores.
+SUB_CPU_TOKENS = {"mixtral": 1, "finegrained": 2, "decode": 2, "tiny": 32, "train": 24, "tiny_b0": 32}
 
-    import numpy as np
+
+class Ctx:
+    """Device, ranks, peaks and the timing helpers shared by every workload of one run."""
+
+    def __init__(self, args, dev, world, rank):
+        import torch
+        import torch.distributed as dist
+        self.args, self.dev, self.world, self.rank = args, dev, world, rank
+        self.torch, self.dist = torch, dist
+        self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # 2x the 126 MB L2
+        self.peaks, self.peak_src = load_peaks()
+
+    def sync_all(self):
+        self.torch.cuda.synchronize(self.dev)
+        if self.world > 1:
+            self.dist.barrier()
+
+    def timed(self, K, body, flush_l2=True):
+        """Device time of K calls of body() (ms, summed over per-call CUDA events; max over ranks)."""
+        torch = self.torch
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        self.sync_all()
+        for i in range(K):
+            if flush_l2:
+                self.flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
+            evs[i][0].record()
+            body()
+            evs[i][1].record()
+        self.sync_all()
+        ms = sum(a.elapsed_time(b) for a, b in evs)
+        if self.world > 1:
+            t = torch.tensor([ms], dtype=torch.float64, device=self.dev)
+            self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    def capture(self, body):
+        """A CUDA graph of body() (the serving step: the library allocates and synchronises nothing),
+        and the number of library launches it holds."""
+        from grouped_nf4_expert_b200 import e4b
+        torch = self.torch
+        torch.cuda.synchronize(self.dev)
+        g = torch.cuda.CUDAGraph()
+        n0 = e4b.e4b_launch_count()
+        with torch.cuda.graph(g):
+            body()
+        n = e4b.e4b_launch_count() - n0
+        torch.cuda.synchronize(self.dev)
+        return g, n
+
+
+def tensor_roofline(ctx, kern, gflops, steps, traffic):
+    """The grouped NF4 GEMM launches against the dense bf16 tensor peak.  The timed regions are well
+    under a second at full clocks, so the fraction is taken against the measured burst GEMM peak;
+    the fraction of the sustained (power-capped, seconds-long) figure is given beside it."""
+    peaks = ctx.peaks
+    nf4_ms = sum(kern.get(n, (0, 0.0))[1] for n in gflops)
+    nf4_launches = sum(kern.get(n, (0, 0.0))[0] for n in gflops)
+    nf4_flop = nf4_gemm_flop_total(gflops, kern)
+    achieved = nf4_flop / (nf4_ms / 1e3) / 1e12 if nf4_ms > 0 else None
+    modes = [n[len("nf4_gemm_"):].replace("_", " ", 1) for n in gflops if n in kern]
+    per_mode = {}
+    for n, f in gflops.items():
+        if n in kern and kern[n][1] > 0:
+            a = f * kern[n][0] / (kern[n][1] / 1e3) / 1e12
+            per_mode[n] = {"achieved": a, "frac": a / peaks["bf16_tflops"],
+                           "avg_launch_ms": kern[n][1] / kern[n][0]}
+    return {"kernel": "nf4_gemm (%s)" % ", ".join(modes), "bound": "tensor",
+            "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": (achieved / peaks["bf16_tflops"]) if achieved else None,
+            "peak_source": "%s bf16_tflops (burst: the timed region is well under a second at full clocks)"
+                           % ctx.peak_src,
+            "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
+            "traffic": traffic,
+            "traffic_unit": "DRAM bytes per step of the nf4_gemm launches (ncu)",
+            "launches": nf4_launches, "avg_launch_ms": nf4_ms / max(nf4_launches, 1),
+            "algorithmic_flop_per_step": nf4_flop / steps, "per_mode": per_mode}
+
+
+def measure(ctx, cfg, headline):
+    """Times one workload's step (its own passes) and returns its record."""
     import torch
-    import torch.distributed as dist
-
-    from grouped_nf4_expert_b200 import build, e4b, inputs, parallel
+    from grouped_nf4_expert_b200 import e4b, inputs, parallel
     from grouped_nf4_expert_b200 import device as dv
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
-    if rank == 0:
-        build.build()
-    if world > 1:
-        dist.barrier()
-    e4b.lib()
-
-    cfg = inputs.CONFIGS[args.workload]
+    args, dev, world, rank = ctx.args, ctx.dev, ctx.world, ctx.rank
+    peaks, peak_src = ctx.peaks, ctx.peak_src
     prob = inputs.make_problem(cfg, data_rank=rank)
     d = dv.upload(prob, dev)
     blk = e4b.Block(dv.dims_of(cfg), cfg.T, dev)
@@ -344,59 +418,24 @@ def main():
             if world > 1:  # data parallel: sum the LoRA gradients of all ranks (NCCL over NVLink)
                 parallel.allreduce_lora_grads(grads)
 
-    def sync_all():
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # 2x the 126 MB L2
     for _ in range(max(args.warmup, 3)):
         step()
     st = blk.check_device_error()
     if st != e4b.E4B_OK:
         raise RuntimeError("device error after warm-up: %s" % e4b.STATUS.get(st, st))
 
-    def timed(K, body, flush_l2=True):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-        sync_all()
-        for i in range(K):
-            if flush_l2:
-                flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
-            evs[i][0].record()
-            body()
-            evs[i][1].record()
-        sync_all()
-        ms = sum(a.elapsed_time(b) for a, b in evs)
-        if world > 1:
-            t = torch.tensor([ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
-
-    def capture(body):
-        """A CUDA graph of body() (the serving step: the library allocates and synchronises nothing),
-        and the number of library launches it holds."""
-        torch.cuda.synchronize(dev)
-        g = torch.cuda.CUDAGraph()
-        n0 = e4b.e4b_launch_count()
-        with torch.cuda.graph(g):
-            body()
-        n = e4b.e4b_launch_count() - n0
-        torch.cuda.synchronize(dev)
-        return g, n
-
     # ---- main timed region (the serving step replays a CUDA graph of the call)
     graphs = []
     if fwd_only:
-        g_step, per_step = capture(step)
+        g_step, per_step = ctx.capture(step)
         graphs.append(g_step)
         with ClockSampler(dev) as clocks:
-            total_ms = timed(args.steps, g_step.replay)
+            total_ms = ctx.timed(args.steps, g_step.replay)
         launches = per_step * args.steps
     else:
         launches0 = e4b.e4b_launch_count()
         with ClockSampler(dev) as clocks:
-            total_ms = timed(args.steps, step)
+            total_ms = ctx.timed(args.steps, step)
         launches = e4b.e4b_launch_count() - launches0
     st = blk.check_device_error()
     if st != e4b.E4B_OK:
@@ -407,38 +446,37 @@ def main():
 
     # ---- per-kernel device times over a second timed region (library profiler, events on the launch stream)
     e4b.e4b_profiler_enable(True)
-    prof_ms = timed(args.steps, step)
+    prof_ms = ctx.timed(args.steps, step)
     e4b.e4b_profiler_enable(False)
     kern = e4b.e4b_profiler_read()
-    peaks, peak_src = load_peaks()
-    gflops = nf4_gemm_flops(cfg)
-    nf4_ms = sum(kern.get(n, (0, 0.0))[1] for n in gflops)
-    nf4_launches = sum(kern.get(n, (0, 0.0))[0] for n in gflops)
-    nf4_flop = nf4_gemm_flop_total(gflops, kern)
-    achieved = nf4_flop / (nf4_ms / 1e3) / 1e12 if nf4_ms > 0 else None
     kern_total = sum(v[1] for v in kern.values())
-    modes = [n[len("nf4_gemm_"):].replace("_", " ", 1) for n in gflops if n in kern]
-    roofline = {"kernel": "nf4_gemm (%s)" % ", ".join(modes), "bound": "tensor",
-                "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
-                "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long step)" % peak_src,
-                "traffic": (profiled_traffic() if args.workload == "train" else None),
-                "traffic_unit": "DRAM bytes per step of the four nf4_gemm launches (ncu)",
-                "launches": nf4_launches,
-                "avg_launch_ms": nf4_ms / max(nf4_launches, 1),
-                "algorithmic_flop_per_step": nf4_flop / args.steps}
-    sbytes = stream_bytes(cfg, int((blk.counts > 0).sum().item()))
+    roofline = tensor_roofline(ctx, kern, nf4_gemm_flops(cfg), args.steps,
+                               profiled_traffic() if cfg.name == "train" else None)
+    touched = int((blk.counts > 0).sum().item())
+    sbytes = serve_bytes(cfg, touched) if "nf4_serve" in kern else stream_bytes(cfg, touched)
     st_ms = sum(kern.get(n, (0, 0.0))[1] for n in sbytes)
     if st_ms > 0:  # the weight-streaming forward ran: it is HBM-bound by design
         st_launches = sum(kern.get(n, (0, 0.0))[0] for n in sbytes)
         st_bytes = sum(sbytes.values()) * args.steps
         ach = st_bytes / (st_ms / 1e3) / 1e9
-        roofline = {"kernel": "nf4_stream (fwd gate_up, fwd down)", "bound": "hbm", "achieved": ach,
+        per_mode = {}
+        for n in sbytes:
+            if n in kern and kern[n][0] > 0:
+                launch_ms = kern[n][1] / kern[n][0]  # one launch of each per step
+                per_mode[n] = {"achieved": sbytes[n] / (launch_ms / 1e3) / 1e9, "avg_launch_ms": launch_ms,
+                               "algorithmic_bytes": sbytes[n]}
+        for v in per_mode.values():
+            v["frac"] = v["achieved"] / peaks["hbm_gbs"]
+        name = ("nf4_serve (x scatter + p_gu, gate_up, p_d, down, combine in one launch)" if "nf4_serve" in sbytes
+                else "nf4_stream (fwd gate_up, fwd down)")
+        roofline = {"kernel": name, "bound": "hbm", "achieved": ach,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
                     "peak_source": "%s hbm_gbs" % peak_src, "traffic": None,
                     "traffic_unit": "DRAM bytes per launch (ncu), see profiles/",
                     "launches": st_launches, "avg_launch_ms": st_ms / max(st_launches, 1),
-                    "algorithmic_bytes_per_step": sum(sbytes.values())}
+                    "algorithmic_bytes_per_step": sum(sbytes.values()), "per_mode": per_mode}
+    if cfg.name.startswith("tiny"):
+        roofline = dict(roofline, note="latency-bound at this size (a few MFLOP per step): reported, not a target")
     per_kernel = {n: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
                       "share": v[1] / kern_total if kern_total else None} for n, v in kern.items()}
 
@@ -464,46 +502,16 @@ def main():
             h.copy_(t, non_blocking=True)
 
     if fwd_only:  # the whole serving step, copies included, as one graph
-        g_e2e, _ = capture(e2e_step)
+        g_e2e, _ = ctx.capture(e2e_step)
         graphs.append(g_e2e)
-        e2e_ms = timed(args.steps, g_e2e.replay)
+        e2e_ms = ctx.timed(args.steps, g_e2e.replay)
     else:
-        e2e_ms = timed(args.steps, e2e_step)
+        e2e_ms = ctx.timed(args.steps, e2e_step)
     e2e = {"value": cfg.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
-    # ---- the rows next to the path, each timed alone (HBM-bound by design).  Both read more than the
-    # 126 MB L2 per launch, so they are timed back to back without the flush (whose dirty lines would
-    # be written back during the next launch).
-    next_rows = {}
-    if not fwd_only:  # router backward (for a trained router) on this step's forward outputs
-        d_logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
-        rb_ms = timed(args.steps, lambda: blk.e4b_router_backward(d.dY, d_logits), flush_l2=False) / args.steps
-        rb_b = router_bwd_bytes(cfg)
-        next_rows["router_backward"] = {
-            "launch_ms": rb_ms, "algorithmic_bytes": rb_b, "achieved": rb_b / (rb_ms / 1e3) / 1e9,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rb_b / (rb_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "bound": "hbm", "l2": "not flushed: > 300 MB read per launch",
-            "note": "d(logits) [T,E] from dY and the forward's y_perm"}
-        del d_logits
-    nq = cfg.E * 2 * cfg.I * cfg.H  # the workload's gate_up stack, bf16 N(0, sigma_w)
-    gq = torch.Generator(device=dev).manual_seed(1234 + rank)
-    wq = (torch.randn(nq, generator=gq, device=dev) * cfg.sigma_w).to(torch.bfloat16)
-    pq = torch.empty(nq // 2, dtype=torch.uint8, device=dev)
-    aq = torch.empty(nq // 64, dtype=torch.float32, device=dev)
-    q_ms = timed(args.steps, lambda: e4b.e4b_nf4_quantize(wq, pq, aq), flush_l2=False) / args.steps
-    q_b = quantize_bytes(nq)
-    next_rows["nf4_quantize"] = {
-        "launch_ms": q_ms, "weights": nq, "algorithmic_bytes": q_b, "achieved": q_b / (q_ms / 1e3) / 1e9,
-        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_b / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-        "bound": "hbm", "l2": "not flushed: > 800 MB read per launch",
-        "note": "bf16 gate_up stack [E,2I,H] -> packed NF4 + fp32 absmax"}
-    del wq, pq, aq
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+    rec = {
+        "value": value, "unit": "tokens/s", "ms_per_step": ms_per_step,
         "config": dict(workload_config(cfg, world, "flushed between timed steps by a 256 MiB write"),
                        cuda_graph=fwd_only, call=("e4b_moe_serve_fwd" if fwd_only else
                                                   "route_permute + lora_fwd + lora_dgrad" +
@@ -515,12 +523,87 @@ def main():
         "profiled_ms_per_step": prof_ms / args.steps,
         "e2e": e2e,
         "gpu_launches": launches,
-        "next_rows": next_rows,
         "clocks": clocks.summary(),
     }
+    if "dgrad" in cfg.passes or fwd_only:
+        rec["routed_experts"] = int((blk.counts > 0).sum().item())
+
+    # ---- the rows next to the path, each timed alone (HBM-bound by design).  Both read more than the
+    # 126 MB L2 per launch, so they are timed back to back without the flush (whose dirty lines would
+    # be written back during the next launch).
+    if headline:
+        next_rows = {}
+        if not fwd_only:  # router backward (for a trained router) on this step's forward outputs
+            d_logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
+            rb_ms = ctx.timed(args.steps, lambda: blk.e4b_router_backward(d.dY, d_logits),
+                              flush_l2=False) / args.steps
+            rb_b = router_bwd_bytes(cfg)
+            next_rows["router_backward"] = {
+                "launch_ms": rb_ms, "algorithmic_bytes": rb_b, "achieved": rb_b / (rb_ms / 1e3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": rb_b / (rb_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "bound": "hbm", "l2": "not flushed: > 300 MB read per launch",
+                "note": "d(logits) [T,E] from dY and the forward's y_perm"}
+            del d_logits
+        nq = cfg.E * 2 * cfg.I * cfg.H  # the workload's gate_up stack, bf16 N(0, sigma_w)
+        gq = torch.Generator(device=dev).manual_seed(1234 + rank)
+        wq = (torch.randn(nq, generator=gq, device=dev) * cfg.sigma_w).to(torch.bfloat16)
+        pq = torch.empty(nq // 2, dtype=torch.uint8, device=dev)
+        aq = torch.empty(nq // 64, dtype=torch.float32, device=dev)
+        q_ms = ctx.timed(args.steps, lambda: e4b.e4b_nf4_quantize(wq, pq, aq), flush_l2=False) / args.steps
+        q_b = quantize_bytes(nq)
+        next_rows["nf4_quantize"] = {
+            "launch_ms": q_ms, "weights": nq, "algorithmic_bytes": q_b, "achieved": q_b / (q_ms / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_b / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "bound": "hbm", "l2": "not flushed: > 800 MB read per launch",
+            "note": "bf16 gate_up stack [E,2I,H] -> packed NF4 + fp32 absmax"}
+        del wq, pq, aq
+        rec["next_rows"] = next_rows
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(prob, args.cpu_sample_tokens)
-    del graphs
+        n_tok = args.cpu_sample_tokens if headline else SUB_CPU_TOKENS.get(cfg.name, 1)
+        rec["cpu_baseline"] = cpu_baseline(prob, n_tok)
+    del graphs, blk, d
+    torch.cuda.empty_cache()
+    return rec
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from grouped_nf4_expert_b200 import build, e4b, inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    e4b.lib()
+
+    ctx = Ctx(args, dev, world, rank)
+    cfg = inputs.CONFIGS[args.workload]
+    head = measure(ctx, cfg, headline=True)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+    }
+    line.update({k: v for k, v in head.items() if k not in line and k not in ("unit",)})
+    # The other workloads, each timed the same way in the same run (one GPU: a data-parallel run times
+    # the headline step only, since every rank would hold its GPU for them).
+    subs = [w for w in (args.sub_workloads.split(",") if args.sub_workloads else []) if w and w != args.workload]
+    if world == 1 and subs:
+        line["workloads"] = {w: measure(ctx, inputs.CONFIGS[w], headline=False) for w in subs}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
