@@ -95,6 +95,8 @@ constexpr int kEpiTileBytes = 32 * 16 * 2;
 constexpr int kEpiStepBytes = 3 * kEpiTileBytes;
 constexpr int kEpiWarpBytes = 2 * kEpiStepBytes;
 static_assert(kEpiWarpBytes >= 3 * 2 * kEpiTileBytes, "three 2-tile buffers for the plain epilogue");
+constexpr int kDgAhead = 3;  // down dgrad epilogue: gate/up copies in flight, 2 KB per step per warp
+static_assert(kEpiWarpBytes >= kDgAhead * 4 * 512, "down dgrad gate/up ring");
 constexpr int EPI_OFF = LB_OFF + LB_BYTES;
 constexpr int BAR_OFF = EPI_OFF + 4 * kEpiWarpBytes;
 constexpr int BAR_BYTES = 1024;
@@ -447,6 +449,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
         const uint4 q0 = *reinterpret_cast<const uint4*>(slot + raw_off);
         const uint4 q1 = *reinterpret_cast<const uint4*>(slot + raw_off + 16);
         const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        // The codes are in registers: hand the code slot back before decoding, so the producer refills it
+        // a whole decode earlier (the proxy fence orders these generic reads before the next TMA write).
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_empty[r]);
         // Rows past the end of the matrix decode with a zero scale: all zeros.
         const Nf4Planes pl = nf4_block_planes(valid ? amax : 0.0f);
         uint32_t v[32];
@@ -459,16 +466,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           st_shared_v4(dbase + ((c ^ (drow & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-        // One proxy fence orders both this thread's reads of the code slot
-        // before the next TMA write into it (generic reads, then an async-proxy
-        // write: released through raw_empty) and its tile stores before the
-        // UMMA reads them.
+        // The proxy fence orders the tile stores before the UMMA reads them.
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bdone[s]);
-          mbar_arrive(&raw_empty[r]);
-        }
+        if (lane == 0) mbar_arrive(&bdone[s]);
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -545,41 +546,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
           ++step;
         }
       } else if (MODE == kDgradDown) {
-        // SwiGLU backward; the forward gate/up values of the next step are
-        // loaded while this step's are used.
+        // SwiGLU backward.  The forward gate/up values of a row are copied
+        // with cp.async into a per-warp ring in the (here unused) staging
+        // area, kDgAhead steps ahead of their use, so that the step loop waits
+        // for none of them: one step ahead left this epilogue longer than the
+        // unit's UMMAs.  Ring slot layout [step % kDgAhead][piece][lane] x 16
+        // bytes: a warp's reads of one piece are 512 contiguous bytes.
         const int I2 = 2 * p.I, c0 = nt * 256;
         const int ncol = min(256, p.I - c0);  // a multiple of 64
         const uint16_t* grow = p.aux + row * I2 + c0;
         if (store) {
           // The unit's gate/up values of this row (2 x ncol bf16, from HBM: the
-          // buffer is larger than L2) are pulled into L2 up front, so the step
-          // loads below wait for L2, not for DRAM.
+          // buffer is larger than L2) are pulled into L2 up front.
           for (int off = 0; off < ncol; off += 64) {
             asm volatile("prefetch.global.L2 [%0];" ::"l"(grow + off));
             asm volatile("prefetch.global.L2 [%0];" ::"l"(grow + p.I + off));
           }
         }
-        // 16-column steps: every load and store covers whole 32-byte sectors.
-        uint4 gq[2], uq[2];
+        uint8_t* ring = smem + EPI_OFF + qrt * kEpiWarpBytes + lane * 16;
+        // copies of 16-column step js (gate: pieces 0-1, up: pieces 2-3); past the row's end nothing is read
+        auto issue = [&](int js) {
+          const int col = js * 16;
+          const uint32_t n = (store && col < ncol) ? 16u : 0u;
+          const uint16_t* g = n ? grow + col : grow;
+          uint8_t* dst = ring + (js % kDgAhead) * 4 * 512;
+          cp_async_16_zfill(dst, g, n);
+          cp_async_16_zfill(dst + 512, g + 8, n);
+          cp_async_16_zfill(dst + 1024, n ? g + p.I : grow, n);
+          cp_async_16_zfill(dst + 1536, n ? g + p.I + 8 : grow, n);
+          cp_async_commit();
+        };
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          gq[h] = store ? __ldg(reinterpret_cast<const uint4*>(grow) + h) : make_uint4(0, 0, 0, 0);
-          uq[h] = store ? __ldg(reinterpret_cast<const uint4*>(grow + p.I) + h) : make_uint4(0, 0, 0, 0);
-        }
+        for (int js = 0; js < kDgAhead - 1; ++js) issue(js);
 #pragma unroll 1
         for (int jj = 0; jj < ncol; jj += 16) {
-          uint4 gn[2], un[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const bool more = store && jj + 16 < ncol;
-            gn[h] = more ? __ldg(reinterpret_cast<const uint4*>(grow + jj + 16) + h) : make_uint4(0, 0, 0, 0);
-            un[h] = more ? __ldg(reinterpret_cast<const uint4*>(grow + p.I + jj + 16) + h) : make_uint4(0, 0, 0, 0);
-          }
+          issue(jj / 16 + kDgAhead - 1);
+          cp_async_wait_group<kDgAhead - 1>();  // this thread's copies of step jj/16 have landed
           float da[16];
           tmem_ld16(tl + jj, da);
           if (store) {
-            const uint32_t gw[8] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w};
-            const uint32_t uw[8] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w};
+            const uint8_t* src = ring + ((jj / 16) % kDgAhead) * 4 * 512;
+            const uint4 g0 = *reinterpret_cast<const uint4*>(src);
+            const uint4 g1 = *reinterpret_cast<const uint4*>(src + 512);
+            const uint4 u0 = *reinterpret_cast<const uint4*>(src + 1024);
+            const uint4 u1 = *reinterpret_cast<const uint4*>(src + 1536);
+            const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            const uint32_t uw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
             uint32_t dgw[8], duw[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -600,11 +612,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
             // unit's UMMAs, and the staging hand-off would lengthen it.
             store_row16(p.out0 + row * I2 + c0 + jj, dgw, p.v8);
             store_row16(p.out0 + row * I2 + p.I + c0 + jj, duw, p.v8);
-          }
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            gq[h] = gn[h];
-            uq[h] = un[h];
           }
         }
       } else {
@@ -652,8 +659,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       }
     }
     // Every bulk store of this warp has written global memory (and stopped
-    // reading its staging buffer) before the CTA goes away.
+    // reading its staging buffer), and every cp.async has landed, before the CTA goes away.
     if (lane == 0) bulk_wait<0>();
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncwarp();
   }
 
