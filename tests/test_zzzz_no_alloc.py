@@ -12,7 +12,7 @@ The work lists in ``tiles`` are compared up to the counts in their header:
 entries past the counts are not defined by a routing call.
 A third call writes the routing tables only (no permuted rows), through the
 binding.  It also checks that a problem too large for the fixed array is refused.
-This file is named to be collected after the main parity tests.
+This file is named to be collected after every other test file.
 """
 
 import ctypes
