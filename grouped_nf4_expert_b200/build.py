@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libe4b.so")
-SOURCES = ["api.cu", "route.cu", "gemm.cu", "stream.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "route.cu", "gemm.cu", "stream.cu", "serve.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-DNDEBUG"]

@@ -61,8 +61,15 @@ e4b_status check_dims(const e4b_moe_dims* d, int32_t T) {
 
 size_t workspace_bytes(const e4b_moe_dims* d, int32_t T) {
   const int64_t nblk = ((int64_t)T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock;
-  const size_t route = (size_t)2 * nblk * d->E * sizeof(int32_t);
-  return sizeof(DeviceError) + ((route + 255) / 256) * 256;
+  size_t ints = (size_t)2 * nblk * d->E;  // routing: per-block histograms and scatter bases
+  const int64_t N = (int64_t)T * d->top_k;
+  if (use_streaming_forward(N, d->E)) {  // the one-launch serving forward's counters and shares (after routing)
+    const int64_t st_cap = stiles_cap(N, d->E);
+    const size_t serve = ((size_t)serve_counters(d->E, st_cap, T, d->H) + 63) / 64 * 64 +
+                         (size_t)serve_part_floats(st_cap, d->I, d->r);
+    if (serve > ints) ints = serve;
+  }
+  return sizeof(DeviceError) + ((ints * sizeof(int32_t) + 255) / 256) * 256;
 }
 
 e4b_status check_ws(const e4b_moe_dims* d, int32_t T, const void* ws, size_t ws_bytes) {
@@ -397,55 +404,52 @@ e4b_status e4b_moe_serve_fwd(const e4b_moe_dims* dims, int32_t T, const float* l
   const int E = dims->E, H = dims->H, I = dims->I, r = dims->r, k = dims->top_k;
   const float s = dims->alpha / (float)r;
   int32_t* scratch = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sizeof(DeviceError));
+  const int64_t st_cap = stiles_cap(N, E);
+  // routing (one CTA for up to 64 tokens), which also zeroes the counters of the launch after it
   E4B_CUDA(launch_route_serve(logits, T, E, H, k, routing->topk_ids, routing->topk_w, routing->counts,
                               routing->offsets, routing->row_of_slot, routing->slot_of_row, routing->tiles,
-                              mtiles_cap(N, E), rows_cap(N, E), scratch, sms, st));
-  // x_perm[row] = x[token]; p_gu[row] = s * x A_gu[e]^T
-  E4B_CUDA(launch_lora_rows(reinterpret_cast<const uint16_t*>(x), true, routing->topk_ids, routing->row_of_slot,
-                            (int)N, k, H, lora->A_gu, r, s, fwd->x_perm, fwd->p_gu, sms, st));
-  Nf4GemmHost g{};
-  g.E = E;
-  g.H = H;
-  g.I = I;
-  g.r = r;
-  g.r_pad = r_padded(r);
-  g.tiles = routing->tiles;
-  g.rows_cap = rows_cap(N, E);
-  g.mt_cap = mtiles_cap(N, E);
-  g.err = static_cast<DeviceError*>(ws);
-  g.timeout_ns = kDefaultTimeoutNs;
-  // act = silu(gate) * up of W_gu x + p_gu B_gu^T (gu itself only when a buffer is given)
-  g.mode = kFwdGateUp;
-  g.nf4 = base->gate_up_nf4;
-  g.absmax = base->gate_up_absmax;
-  g.stored_rows = 2 * I;
-  g.stored_cols = H;
-  g.act_in = fwd->x_perm;
-  g.K = H;
-  g.n_dim = 2 * I;
-  g.lora_a_rows = fwd->p_gu;
-  g.lora_w = lora->B_gu;
-  g.out0 = fwd->gu;
-  g.out1 = fwd->act;
-  E4B_CUDA(launch_nf4_stream(g, sms, st));
-  // p_d[row] = s * act A_d[e]^T
-  E4B_CUDA(launch_lora_rows(fwd->act, false, routing->topk_ids, routing->row_of_slot, (int)N, k, I, lora->A_d, r,
-                            s, nullptr, fwd->p_d, sms, st));
-  // y_perm = W_d act + p_d B_d^T
-  g.mode = kFwdDown;
-  g.nf4 = base->down_nf4;
-  g.absmax = base->down_absmax;
-  g.stored_rows = H;
-  g.stored_cols = I;
-  g.act_in = fwd->act;
-  g.K = I;
-  g.n_dim = H;
-  g.lora_a_rows = fwd->p_d;
-  g.lora_w = lora->B_d;
-  g.out0 = fwd->y_perm;
-  g.out1 = nullptr;
-  E4B_CUDA(launch_nf4_stream(g, sms, st));
-  E4B_CUDA(launch_combine(fwd->y_perm, routing->row_of_slot, routing->topk_w, T, k, H, y, sms, st));
+                              mtiles_cap(N, E), rows_cap(N, E), scratch, sms, st, scratch,
+                              serve_counters(E, st_cap, T, H)));
+  // everything else in one launch: x scatter + p_gu, gate_up + SiLU gate, p_d, down, weighted combine
+  ServeHost h{};
+  h.T = T;
+  h.k = k;
+  h.E = E;
+  h.H = H;
+  h.I = I;
+  h.r = r;
+  h.r_pad = r_padded(r);
+  h.s = s;
+  h.gate_up_nf4 = base->gate_up_nf4;
+  h.gate_up_absmax = base->gate_up_absmax;
+  h.down_nf4 = base->down_nf4;
+  h.down_absmax = base->down_absmax;
+  h.A_gu = lora->A_gu;
+  h.B_gu = lora->B_gu;
+  h.A_d = lora->A_d;
+  h.B_d = lora->B_d;
+  h.x = reinterpret_cast<const uint16_t*>(x);
+  h.x_perm = fwd->x_perm;
+  h.p_gu = fwd->p_gu;
+  h.gu = fwd->gu;
+  h.act = fwd->act;
+  h.p_d = fwd->p_d;
+  h.y_perm = fwd->y_perm;
+  h.y = reinterpret_cast<uint16_t*>(y);
+  h.topk_ids = routing->topk_ids;
+  h.topk_w = routing->topk_w;
+  h.row_of_slot = routing->row_of_slot;
+  h.slot_of_row = routing->slot_of_row;
+  h.counts = routing->counts;
+  h.tiles = routing->tiles;
+  h.counters = scratch;
+  h.pd_part = reinterpret_cast<float*>(scratch + (serve_counters(E, st_cap, T, H) + 63) / 64 * 64);
+  h.rows_cap = rows_cap(N, E);
+  h.mt_cap = mtiles_cap(N, E);
+  h.st_cap = st_cap;
+  h.err = static_cast<DeviceError*>(ws);
+  h.timeout_ns = kDefaultTimeoutNs;
+  E4B_CUDA(launch_nf4_serve(h, sms, st));
   return E4B_OK;
 }
 

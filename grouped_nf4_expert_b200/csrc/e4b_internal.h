@@ -31,6 +31,25 @@ inline int64_t tiles_cap(int64_t N, int E) { return stiles_offset(mtiles_cap(N, 
 // slots per expert (decode-sized), the 2-SM training tiles otherwise.
 inline bool use_streaming_forward(int64_t N, int E) { return N <= 16 * (int64_t)E; }
 inline int64_t rows_cap(int64_t N, int E) { return ((N + (int64_t)E * 127) + 127) / 128 * 128; }
+// Upper bound of the 32-slot streaming tiles of N slots over E experts.
+inline int64_t stiles_cap(int64_t N, int E) { return (N + 31) / 32 + E; }
+
+// Device counters of the one-launch serving forward (int32, in the workspace after
+// the error word, zeroed by the routing launch before it): slots prepped per
+// expert [E], gate_up units done per slot tile [st_cap], LoRA-down projection
+// done per slot tile [st_cap], slots of a token whose y_perm piece is written
+// [T * ceil(H/128)].
+inline int64_t serve_cnt_a_offset(int E) { return E; }
+inline int64_t serve_pd_offset(int E, int64_t st_cap) { return E + st_cap; }
+inline int64_t serve_comb_offset(int E, int64_t st_cap) { return E + 2 * st_cap; }
+inline int64_t serve_claim_offset(int E, int64_t st_cap, int T, int H) {
+  return E + 2 * st_cap + (int64_t)T * ((H + 127) / 128);
+}
+// ... and the unit-claim counter.
+inline int64_t serve_counters(int E, int64_t st_cap, int T, int H) { return serve_claim_offset(E, st_cap, T, H) + 1; }
+// Then (256-byte aligned) float32 shares of the LoRA down projection, one [32, r]
+// block per (slot tile, 64-feature gate/up tile).
+inline int64_t serve_part_floats(int64_t st_cap, int I, int r) { return st_cap * (I / 64) * 32 * (int64_t)r; }
 
 struct DeviceError;
 
@@ -56,10 +75,12 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
 
 // Routing tables for the serving forward (no x gather, no padding markers for
 // batches of at most kRouteTokensPerBlock tokens, which take one launch).
+// `zero`/`n_zero` (optional): int32 counters that the same launch sets to 0 (the
+// one-launch serving forward's counters).
 cudaError_t launch_route_serve(const float* logits, int T, int E, int H, int k, int32_t* topk_ids, float* topk_w,
                                int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* slot_of_row,
                                int32_t* tiles, int64_t mt_cap, int64_t rows_cap, int32_t* scratch, int num_sms,
-                               cudaStream_t stream);
+                               cudaStream_t stream, int32_t* zero = nullptr, int64_t n_zero = 0);
 // out[row(f)] = bf16(s * src_row(f) . A[e(f)]^T) per routed slot f on the CUDA cores; src_row is the token's
 // row (by_token) or the permuted row; copy_dst (optional) receives the source row at the permuted row.
 cudaError_t launch_lora_rows(const uint16_t* src, bool by_token, const int32_t* topk_ids, const int32_t* row_of_slot,
@@ -110,6 +131,28 @@ struct Nf4GemmHost {
 cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stream);
 // Weight-streaming forward (kFwdGateUp / kFwdDown only) for decode-sized batches.
 cudaError_t launch_nf4_stream(const Nf4GemmHost& h, int num_sms, cudaStream_t stream);
+
+// The serving forward of a decode-sized batch in one launch (serve.cu): x
+// scatter + p_gu, gate_up, p_d, down and the weighted combine.
+struct ServeHost {
+  int T, k, E, H, I, r, r_pad;
+  float s;
+  const uint8_t* gate_up_nf4;
+  const float* gate_up_absmax;
+  const uint8_t* down_nf4;
+  const float* down_absmax;
+  const uint16_t *A_gu, *B_gu, *A_d, *B_d;
+  const uint16_t* x;
+  uint16_t *x_perm, *p_gu, *gu, *act, *p_d, *y_perm, *y;
+  const int32_t *topk_ids, *row_of_slot, *slot_of_row, *counts, *tiles;
+  const float* topk_w;
+  int32_t* counters;  // serve_counters(E, st_cap, T, H) ints, zero on entry
+  float* pd_part;     // serve_part_floats(st_cap, I, r) floats (no initial contents needed)
+  int64_t rows_cap, mt_cap, st_cap;
+  DeviceError* err;
+  long long timeout_ns;
+};
+cudaError_t launch_nf4_serve(const ServeHost& h, int num_sms, cudaStream_t stream);
 
 struct LoraProjHost {
   const uint16_t* act_in;  // [rows_cap, K]

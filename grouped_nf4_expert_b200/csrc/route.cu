@@ -263,9 +263,11 @@ __global__ void __launch_bounds__(32) route_rank_kernel(const int32_t* __restric
 // Routing of a batch of at most kRouteTokensPerBlock tokens in one CTA, for
 // the serving forward: top-k + softmax per token (as route_topk_kernel), the
 // expert counts, 128-aligned group offsets, the weight-streaming tile list
-// and the stable slot ranks (as route_scan_kernel and route_rank_kernel), in
-// one launch.  No padding markers and no m-tile lists: the serving forward
-// reads neither.
+// and the stable slot ranks (row_of_slot, and slot_of_row for the routed
+// rows), as route_scan_kernel and route_rank_kernel do, in one launch.  No
+// padding markers and no m-tile lists: the serving forward reads neither.  The
+// launch also sets `n_zero` ints at `zero` to 0 (the counters of the serving
+// launch that follows it).
 template <int EPL>
 __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                           int32_t* __restrict__ topk_ids,
@@ -273,7 +275,10 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
                                                           int32_t* __restrict__ counts,
                                                           int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ row_of_slot,
-                                                          int32_t* __restrict__ tiles, int64_t st_offset) {
+                                                          int32_t* __restrict__ slot_of_row,
+                                                          int32_t* __restrict__ tiles, int64_t st_offset,
+                                                          int32_t* __restrict__ zero, int64_t n_zero) {
+  for (int64_t z = threadIdx.x; z < n_zero; z += blockDim.x) zero[z] = 0;
   __shared__ int s_cnt[E4B_MAX_EXPERTS];
   __shared__ int s_run[E4B_MAX_EXPERTS];
   __shared__ int s_warp[32];
@@ -357,7 +362,10 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
       const unsigned peers = __match_any_sync(0xffffffffu, ex);
       const int rank = __popc(peers & ((1u << lane) - 1u));
       const int leader = __ffs(peers) - 1;
-      if (ex >= 0) row_of_slot[f] = s_run[ex] + rank;
+      if (ex >= 0) {
+        row_of_slot[f] = s_run[ex] + rank;
+        slot_of_row[s_run[ex] + rank] = f;
+      }
       __syncwarp();
       if (ex >= 0 && lane == leader) s_run[ex] += __popc(peers);
       __syncwarp();
@@ -879,16 +887,19 @@ cudaError_t launch_route(const float* logits, const uint16_t* x, int T, int E, i
 cudaError_t launch_route_serve(const float* logits, int T, int E, int H, int k, int32_t* topk_ids, float* topk_w,
                                int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* slot_of_row,
                                int32_t* tiles, int64_t mt_cap, int64_t rows_cap, int32_t* scratch, int num_sms,
-                               cudaStream_t stream) {
-  if (T > kRouteTokensPerBlock)
-    return launch_route(logits, nullptr, T, E, H, k, topk_ids, topk_w, counts, offsets, row_of_slot, slot_of_row,
-                        tiles, mt_cap, nullptr, rows_cap, scratch, num_sms, stream);
+                               cudaStream_t stream, int32_t* zero, int64_t n_zero) {
+  if (T > kRouteTokensPerBlock) {
+    cudaError_t err = launch_route(logits, nullptr, T, E, H, k, topk_ids, topk_w, counts, offsets, row_of_slot,
+                                   slot_of_row, tiles, mt_cap, nullptr, rows_cap, scratch, num_sms, stream);
+    if (err != cudaSuccess || zero == nullptr || n_zero == 0) return err;
+    return cudaMemsetAsync(zero, 0, (size_t)n_zero * sizeof(int32_t), stream);
+  }
   const int64_t st_off = stiles_offset(mt_cap, E);
   const int epl = (E + 31) / 32;
   LaunchScope scope("route_small", stream);
 #define E4B_ROUTE_SMALL(P)                                                                                   \
   route_small_kernel<P><<<1, 1024, 0, stream>>>(logits, T, E, k, topk_ids, topk_w, counts, offsets, row_of_slot, \
-                                                tiles, st_off)
+                                                slot_of_row, tiles, st_off, zero, n_zero)
   if (epl <= 1)
     E4B_ROUTE_SMALL(1);
   else if (epl <= 2)

@@ -220,15 +220,20 @@ e4b_status e4b_grouped_nf4_lora_fwd(const e4b_moe_dims *dims, int32_t T,
  * (decode-sized batches above all): y = the block's output for x (bf16
  * [T, H]) and logits (float32 [T, E]), the same arithmetic as
  * e4b_route_permute + e4b_grouped_nf4_lora_fwd.  Batches with at most
- * 16 * E routed slots take the serving pipeline: routing tables in one
- * launch (T <= 64) or three, the x scatter fused with the LoRA projection
- * s * x A_gu^T on the CUDA cores, the weight-streaming gate_up, the
- * projection s * act A_d^T, the weight-streaming down and the weighted
- * combine -- six launches, nothing kept for a backward: fwd->gu may be NULL
- * (then not written), padding rows of the permuted buffers and
- * routing->slot_of_row are left unspecified, and the m-tile lists in
- * routing->tiles are not built, so the routing and buffers of a serving call
- * must not be passed to e4b_grouped_nf4_lora_dgrad or e4b_lora_wgrad.
+ * 16 * E routed slots take the serving pipeline: the routing tables in one
+ * launch (T <= 64) or three, then ONE persistent launch for everything else
+ * -- the x scatter with the LoRA projection s * x A_gu^T, the weight-
+ * streaming gate_up GEMM with the SiLU-gated epilogue, the projection
+ * s * act A_d^T, the weight-streaming down GEMM and the router-weighted
+ * combine, its work units ordered so that each waits (device-side, bounded:
+ * a wait that runs out records E4B_ERR_DEVICE_TIMEOUT in the workspace) only
+ * for units before it.  Nothing is kept for a backward: fwd->gu may be NULL
+ * (then not written), padding rows of the permuted buffers are left
+ * unspecified and the m-tile lists in routing->tiles are not built, so the
+ * routing and buffers of a serving call must not be passed to
+ * e4b_grouped_nf4_lora_dgrad or e4b_lora_wgrad.  The launch keeps its
+ * counters and partial sums in ws (e4b_get_sizes accounts for them), so two
+ * serving calls that share a workspace must not overlap on the GPU.
  * Larger batches run e4b_route_permute + e4b_grouped_nf4_lora_fwd (fwd->gu
  * is then required).  Argument checks, ownership and errors as for those two
  * calls; the call allocates nothing and never synchronises, so it can be

@@ -4,7 +4,8 @@ The pages ask for the fast path's engagement to be asserted, not just its
 results: here the library's own launch record (the per-kernel profiler and the
 launch counter) shows, per call, which kernels ran and how often -- the grouped
 tensor-core GEMMs for training-sized batches, the weight-streaming kernels for
-decode-sized ones, the fused row gathers, the six-launch serving call.
+decode-sized ones, the fused row gathers, and the serving call of a decode-sized
+batch: routing plus one persistent launch for everything else.
 Collected after the parity tests.
 """
 
@@ -66,11 +67,21 @@ def test_decode_sized_batch_forward_runs_the_weight_streaming_kernels():
     _training_calls(gp.SMALL["stream_r24"], streaming=True)
 
 
-def test_serving_call_is_six_launches_for_a_decode_batch():
+def test_serving_call_is_routing_plus_one_launch_for_a_decode_batch():
     cfg = inputs.CONFIGS["decode"]
     d = dv.upload(inputs.make_problem(cfg))
     blk = e4b.Block(dv.dims_of(cfg), cfg.T)
     assert _launched(lambda: blk.e4b_moe_serve_fwd(d.logits, d.x, d.base(), d.lora())) == {
-        "route_small": 1, "scatter_lora_rows": 1, "nf4_stream_fwd_gate_up": 1, "lora_rows": 1,
-        "nf4_stream_fwd_down": 1, "combine_y": 1}
+        "route_small": 1, "nf4_serve": 1}
+    assert blk.check_device_error() == e4b.E4B_OK
+
+
+def test_serving_call_above_64_tokens_routes_in_three_launches_then_one():
+    # more than one routing block of tokens: the multi-block routing kernels, then the same single launch
+    cfg = gp.SMALL["stream_zipf_r64"]
+    assert cfg.T > 64 and cfg.N <= 16 * cfg.E
+    d = dv.upload(inputs.make_problem(cfg))
+    blk = e4b.Block(dv.dims_of(cfg), cfg.T)
+    assert _launched(lambda: blk.e4b_moe_serve_fwd(d.logits, d.x, d.base(), d.lora())) == {
+        "route_topk": 1, "route_scan": 1, "route_rank": 1, "nf4_serve": 1}
     assert blk.check_device_error() == e4b.E4B_OK
