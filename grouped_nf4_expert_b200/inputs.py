@@ -171,6 +171,16 @@ def make_problem(cfg: Config, T: int = None, data_rank: int = 0) -> Problem:
                    A_gu, B_gu, A_d, B_d, dY)
 
 
+def dense_expert_weights(cfg: Config):
+    """Dense bf16 expert stacks drawn ~ N(0, sigma_w): ``gate_up`` [E, 2I, H] and ``down`` [E, H, I]
+    (bf16 bit patterns), the weights the workloads describe before NF4 quantisation.  Random draws only:
+    quantising them is the caller's step."""
+    E, H, I = cfg.E, cfg.H, cfg.I
+    gu = _normal_bf16(_rng(cfg.seed, 13), (E, 2 * I, H), cfg.sigma_w)
+    dn = _normal_bf16(_rng(cfg.seed, 14), (E, H, I), cfg.sigma_w)
+    return gu, dn
+
+
 def bits_to_f32(b: np.ndarray) -> np.ndarray:
     """bfloat16 bit patterns -> float32 values (exact widening)."""
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)

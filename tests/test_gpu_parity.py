@@ -305,7 +305,11 @@ def test_block_parity_small(name, fused):
 
 
 def _check_block(cfg, fused):
-    prob, _, blk = run(cfg, fused_gather=fused)
+    _check_block_prob(cfg, None, fused)
+
+
+def _check_block_prob(cfg, prob, fused=True):
+    prob, _, blk = run(cfg, fused_gather=fused, prob=prob)
     ros = check_routing(prob, blk)
     ex = oracle_experts(prob)
     x = inputs.bits_to_f32(prob.x).astype(np.float64)
@@ -330,6 +334,29 @@ def _check_block(cfg, fused):
         errs[key] = rel_err(f64(buf), bo[key])
     bad = {k: v for k, v in errs.items() if not v <= TOL}
     assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("name", ["tiny", "medium", "stream_r24"])
+def test_block_parity_on_quantised_normal_stacks(name):
+    # The workloads' recipe for the frozen base: dense weights ~ N(0, 0.02), NF4-quantised (64-element
+    # blocks, fp32 absmax).  The GPU quantiser must produce the oracle quantiser's bytes exactly; the
+    # block then runs on those bytes and is compared with the oracle element by element.
+    cfg = SMALL[name] if name in SMALL else inputs.CONFIGS[name]
+    prob = inputs.make_problem(cfg)
+    gu_w, dn_w = inputs.dense_expert_weights(cfg)
+    want = {}
+    for key, wbits in (("gate_up", gu_w), ("down", dn_w)):
+        packed, absmax = oracle.quantize_nf4(inputs.bits_to_f32(wbits))
+        got_p, got_a = _quantize_gpu(wbits.reshape(-1))
+        assert np.array_equal(got_p, packed.reshape(-1)), key
+        assert np.array_equal(got_a.view(np.uint32), absmax.reshape(-1).view(np.uint32)), key
+        want[key] = (packed, absmax)
+    prob.gate_up_nf4, prob.gate_up_absmax = want["gate_up"]
+    prob.down_nf4, prob.down_absmax = want["down"]
+    # every code occurs (quantised normals, not a narrow subset)
+    codes = np.concatenate([prob.gate_up_nf4.reshape(-1) >> 4, prob.gate_up_nf4.reshape(-1) & 15])
+    assert np.unique(codes).size == 16
+    _check_block_prob(cfg, prob)
 
 
 def test_b_zero_delta_is_exactly_zero_on_gpu():
