@@ -57,39 +57,50 @@ __device__ __forceinline__ void store_row16(uint16_t* dst, const uint32_t (&w)[8
 // activation tile and decodes weight rows (output columns) [128c, 128c+128)
 // of the tile; its TMEM receives its 128 rows x 256 columns.  Each CTA loads
 // only its own tiles (no multicast loads).
-// Roles per CTA: warp 0 = NF4 codes + block scales into a ring of their own
-// (one slot per decode group, filled far ahead), warp 1 = TMEM owner (both
-// CTAs) and UMMA issuer (even CTA only), warp 2 = relay (odd CTA), warp 3 =
-// activation tiles and LoRA operands, warps 4-19 = four decode groups taking
-// the k-chunks round robin, warps 20-23 = epilogue.  A stage slot holds one
-// k-chunk's activation tile and decoded weight tile; decoders decode into
-// registers from the code ring and only wait for the slot to be free to store,
-// so a slot's round trip is the activation load plus a store.
-// The UMMA issuer (even CTA) learns of its own CTA's readiness through local
-// barriers (bdone, xfull, lfull) and of the odd CTA's through bfull / lready,
-// which the odd CTA's relay signals with st.async stores whose mbarrier
+// Roles per CTA: warp 0 = NF4 codes into a ring of their own (one TMA per
+// k-chunk, filled far ahead), warp 1 = TMEM owner (both CTAs) and UMMA issuer
+// (even CTA only), warp 2 = relay (odd CTA), warp 3 = activation tiles and
+// LoRA operands, warps 4-19 = three decode groups taking the k-chunks round
+// robin (warps 5, 9, 13, 17, which share the issuer's scheduler partition,
+// idle), warps 20-23 = epilogue.  A stage slot holds one k-chunk's activation
+// tile and decoded weight tile, or, once per unit ahead of its k-chunks, the
+// unit's LoRA operands (so the LoRA step needs no buffers of its own and the
+// ring is five slots deep).  Decoders decode into registers from the code ring
+// (block scales: their own loads, a chunk ahead) and only wait for the slot to
+// be free to store (a counter the activation loader advances as it sees each
+// use's slot emptied), so a slot's round trip is the activation load plus a
+// store.
+// Each CTA's relay (warp 2) waits for its own half of a stage use (bdone,
+// xfull) and signals the even CTA's full[s], the one barrier the UMMA issuer
+// tests per stage use: the even CTA's relay with an arrive that also arms 4
+// transaction bytes, the odd CTA's with a 4-byte st.async whose mbarrier
 // complete_tx carries the cluster-scope release (a release-arrive would stall
-// the signalling warp for about a microsecond).  bfull / lready expect 4 bytes
-// per phase and are re-armed by the issuer as soon as it has observed a phase.
-// The issuer's commits arrive on both CTAs' empty / lempty / accfull barriers.
+// the signalling warp for about a microsecond).  The issuer's instruction
+// stream is one dependent chain per k-chunk sharing its scheduler with four
+// decode warps, so it is kept short.  The issuer's commits arrive on both
+// CTAs' empty / accfull barriers.
 namespace nf4g {
 constexpr int BM = 128;   // activation rows per CTA (256 per pair)
 constexpr int BN = 128;   // weight rows decoded per CTA (256 output columns per pair)
-constexpr int BK = 64, STAGES = 4;
+constexpr int BK = 64, STAGES = 5;
 constexpr int A_BYTES = BM * BK * 2;                 // activation tile, K-major SW128
 constexpr int B_BYTES = BN * BK * 2;                 // dequantised weight tile
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
-constexpr int kGroups = 4;          // decode groups; group g decodes the k-chunks j with j % 4 == g
+// Decode groups; group g decodes the k-chunks j with j % kGroups == g.  With three groups the
+// decode warps stay out of the scheduler partition of the UMMA issuer (warps with warp % 4 == 1,
+// which then idle): the issuer's per-k-chunk instructions form one dependent chain, and beside
+// four ALU-bound decode warps each of them waited ~10 cycles for an issue slot.
+constexpr int kGroups = 4;
 constexpr int kGroupWarps = 4;      // warps per decode group (one per 32 weight rows)
-constexpr int RAW_STAGES = 2 * kGroups;  // code slot r always belongs to group r % 4 (no phase aliasing)
+constexpr bool kDecodeSkipsIssuerPartition = (kGroups == 3);
+constexpr int RAW_STAGES = 2 * kGroups;  // code slot r always belongs to group r % kGroups (no phase aliasing)
 constexpr int RAW_BYTES = BN * BK / 2;               // NF4 codes as loaded
-constexpr int AMAX_BYTES = BN * 4;                   // one absmax per decode thread
-constexpr int RAW_SLOT = RAW_BYTES + AMAX_BYTES;     // 4608
+constexpr int RAW_SLOT = RAW_BYTES;
 constexpr int RAW_OFF = STAGES * STAGE_BYTES;
-constexpr int LA_OFF = RAW_OFF + RAW_STAGES * RAW_SLOT;
-constexpr int LA_BYTES = BM * E4B_MAX_RANK * 2;      // p or q rows of this CTA
-constexpr int LB_BYTES = BN * E4B_MAX_RANK * 2;      // LoRA weight rows of this CTA
-constexpr int LB_OFF = LA_OFF + LA_BYTES;
+// A unit's LoRA operands (p or q rows of this CTA, 128 x r_pad; its LoRA weight
+// rows, 128 x r_pad) take the A and B halves of the stage slot before the unit's
+// first k-chunk.
+static_assert(BM * E4B_MAX_RANK * 2 <= A_BYTES && BN * E4B_MAX_RANK * 2 <= B_BYTES, "LoRA operands fit a stage");
 // Epilogue staging: per epilogue warp, two steps x up to three 32-row x 16-column output tiles.
 constexpr int kEpiTileBytes = 32 * 16 * 2;
 constexpr int kEpiStepBytes = 3 * kEpiTileBytes;
@@ -97,20 +108,25 @@ constexpr int kEpiWarpBytes = 2 * kEpiStepBytes;
 static_assert(kEpiWarpBytes >= 3 * 2 * kEpiTileBytes, "three 2-tile buffers for the plain epilogue");
 constexpr int kDgAhead = 3;  // down dgrad epilogue: gate/up copies in flight, 2 KB per step per warp
 static_assert(kEpiWarpBytes >= kDgAhead * 4 * 512, "down dgrad gate/up ring");
-constexpr int EPI_OFF = LB_OFF + LB_BYTES;
+constexpr int EPI_OFF = RAW_OFF + RAW_STAGES * RAW_SLOT;
 constexpr int BAR_OFF = EPI_OFF + 4 * kEpiWarpBytes;
 constexpr int BAR_BYTES = 1024;
 constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;
-constexpr int kEpiWarp0 = 4 + kGroups * kGroupWarps;
+constexpr int kEpiWarp0 = 20;  // warps 4..19: decode warps (and, with three groups, the idle warps 5, 9, 13, 17)
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+static_assert(kGroups * kGroupWarps == (kDecodeSkipsIssuerPartition ? 12 : 16), "decode warps among 4..19");
+// Index of decode warp `warp` (0 .. kGroups * kGroupWarps - 1), or -1 for an idle warp.
+__device__ __forceinline__ int decode_index(int warp) {
+  if (!kDecodeSkipsIssuerPartition) return warp - 4;
+  const int q = warp & 3;
+  return q == 1 ? -1 : 3 * ((warp - 4) >> 2) + (q == 0 ? 0 : q - 1);
+}
 constexpr int kTmemCols = 512;      // 2 accumulator buffers x 256 columns
-constexpr int kRawFullCount = 1 + 32;  // the producer's expect_tx arrival + 32 absmax cp.async arrivals
-static_assert(LA_OFF % 1024 == 0 && LB_OFF % 1024 == 0, "swizzle atom alignment");
+static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atom alignment");
 static_assert(RAW_STAGES % kGroups == 0, "code slots are owned by one decode group each");
-// A decode group waits for stage slot j % STAGES after its previous chunk j - kGroups
-// waited for the commit of chunk j - kGroups - STAGES; the barrier cannot be two
-// phases behind as long as STAGES >= kGroups.
-static_assert(STAGES >= kGroups, "stage-slot waits cannot alias");
+// Decode groups learn that their stage slot is free from a monotonic counter (bfree);
+// the activation loader, the relay and the issuer wait for every stage use in order,
+// so their parity waits cannot alias.
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace nf4g
 
@@ -141,48 +157,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   uint8_t* smem = align1024(smem_dyn);
   uint8_t* stages = smem;
   uint8_t* rawbuf = smem + RAW_OFF;
-  uint8_t* la = smem + LA_OFF;
-  uint8_t* lb = smem + LB_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* raw_full = bars;                   // [RAW_STAGES] codes + block scales landed
+  uint64_t* raw_full = bars;                   // [RAW_STAGES] codes landed
   uint64_t* raw_empty = raw_full + RAW_STAGES; // [RAW_STAGES] codes read into registers (group's 4 warps)
   uint64_t* xfull = raw_empty + RAW_STAGES;    // [STAGES] activation tile landed
-  uint64_t* bfull = xfull + STAGES;            // [STAGES] (even CTA) the odd CTA's stage complete (relay)
-  uint64_t* empty = bfull + STAGES;            // [STAGES] stage consumed by the UMMAs
+  uint64_t* full = xfull + STAGES;             // [STAGES] (even CTA) both CTAs' halves of the stage in place
+  uint64_t* empty = full + STAGES;             // [STAGES] stage consumed by the UMMAs
   uint64_t* bdone = empty + STAGES;            // [STAGES] this CTA's decoded tile written (group's 4 warps)
-  uint64_t* lfull = bdone + STAGES;            // local LoRA operands landed
-  uint64_t* lready = lfull + 1;          // (even CTA) the odd CTA's LoRA operands landed
-  uint64_t* lempty = lfull + 2;          // LoRA operands consumed
-  uint64_t* accfull = lfull + 3;         // [2] accumulator buffer complete
-  uint64_t* accempty = lfull + 5;        // [2] (even CTA) accumulator buffer drained in both CTAs
-  uint64_t* drain = lfull + 7;           // (even CTA) all issued UMMAs finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + 8);
-  CtaControl* ctl = reinterpret_cast<CtaControl*>(lfull + 9);
-  uint32_t* sig = reinterpret_cast<uint32_t*>(lfull + 10);  // target word of the st.async signals
+  uint64_t* accfull = bdone + STAGES;          // [2] accumulator buffer complete
+  uint64_t* accempty = accfull + 2;            // [2] (even CTA) accumulator buffer drained in both CTAs
+  uint64_t* drain = accfull + 4;               // (even CTA) all issued UMMAs finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 5);
+  CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 6);
+  uint32_t* sig = reinterpret_cast<uint32_t*>(accfull + 7);  // target word of the st.async signals
+  // Stage uses whose slot is free (the activation loader's count of empty phases it has waited for): a decode
+  // group skips the uses of the other groups and the units' LoRA uses, so it cannot wait on empty's parity.
+  uint32_t* bfree = reinterpret_cast<uint32_t*>(accfull + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   if (threadIdx.x == 0) {
     for (int r = 0; r < RAW_STAGES; ++r) {
-      mbar_init(&raw_full[r], kRawFullCount);
+      mbar_init(&raw_full[r], 1);
       mbar_init(&raw_empty[r], kGroupWarps);
     }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&xfull[s], 1);
-      mbar_init(&bfull[s], 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&bdone[s], kGroupWarps);
     }
-    mbar_init(lfull, 1);
-    mbar_init(lready, 1);
-    for (int s = 0; s < STAGES; ++s) mbar_arrive_expect_tx(&bfull[s], 4);  // arm phase 0
-    mbar_arrive_expect_tx(lready, 4);
-    mbar_init(lempty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 8);
     }
     mbar_init(drain, 1);
+    *bfree = 0;
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -201,15 +211,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   const int blocks_per_row = p.stored_cols / 64;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
-  // Stored rows of this CTA's weight tile (K-major modes): two 64-row halves.
-  auto kmajor_rows = [&](int nt, int& rA, int& rB) {
-    if (MODE == kFwdGateUp) {  // even CTA: gate rows, odd CTA: the matching up rows
-      rA = (rank ? p.I : 0) + nt * 128;
-      rB = rA + 64;
-    } else {
-      rA = nt * 256 + rank * 128;
-      rB = rA + 64;
-    }
+  // First of the 128 consecutive stored rows of this CTA's weight tile (K-major modes).
+  auto kmajor_row0 = [&](int nt) -> int {
+    if (MODE == kFwdGateUp) return (rank ? p.I : 0) + nt * 128;  // even CTA: gate rows, odd CTA: up rows
+    return nt * 256 + rank * 128;
   };
   // Decoded tile row t of this CTA is valid (exists in the stored matrix / output).
   auto row_valid = [&](int nt, int t) -> bool {
@@ -221,88 +226,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------ NF4 codes + block scales into the code ring (whole warp)
-    if (lane == 0) tma_prefetch_desc(&map_raw);
-    uint32_t j = 0, issued = 0, last_par = 0;  // issued/last_par: per code slot
-    bool ok = true;
-    int e_next = (pair < n_units) ? units[3 * (pair / p.n_nt)] : 0;
-    for (int u = pair; u < n_units && ok; u += n_pairs) {
-      const int nt = u % p.n_nt;
-      const int e = e_next;
-      if (u + n_pairs < n_units) e_next = units[3 * ((u + n_pairs) / p.n_nt)];
-      int rA = 0, rB = 0;
-      if (!kMN) kmajor_rows(nt, rA, rB);
-      for (int kc = 0; kc < kchunks; ++kc, ++j) {
-        const uint32_t r = j % RAW_STAGES, ph = (j / RAW_STAGES) & 1;
-        ok = __all_sync(kFull, mbar_wait_lazy(&raw_empty[r], ph ^ 1, ctl, p.err, p.timeout_ns, 11, 64));
-        if (!ok) break;
-        uint8_t* slot = rawbuf + r * RAW_SLOT;
-        if (lane == 0) {
+    // ------------------------------------------------ NF4 codes into the code ring (one lane)
+    // One TMA per k-chunk: the 128 weight rows x 64 codes of this CTA (K-major: 128 consecutive stored rows;
+    // N-contiguous: 64 stored rows x 128 codes).  The block scales are read by the decoders themselves, a
+    // chunk ahead: gathered here they made this role slower than the k-chunk rate.
+    if (lane == 0) {
+      tma_prefetch_desc(&map_raw);
+      uint32_t j = 0, issued = 0, last_par = 0;  // issued/last_par: per code slot
+      bool ok = true;
+      int e_next = (pair < n_units) ? units[3 * (pair / p.n_nt)] : 0;
+      for (int u = pair; u < n_units && ok; u += n_pairs) {
+        const int nt = u % p.n_nt;
+        const int e = e_next;
+        if (u + n_pairs < n_units) e_next = units[3 * ((u + n_pairs) / p.n_nt)];
+        const int rA = kMN ? 0 : kmajor_row0(nt);
+        for (int kc = 0; kc < kchunks; ++kc, ++j) {
+          const uint32_t r = j % RAW_STAGES, ph = (j / RAW_STAGES) & 1;
+          if (!(ok = mbar_wait_lazy(&raw_empty[r], ph ^ 1, ctl, p.err, p.timeout_ns, 11, 64))) break;
+          uint8_t* slot = rawbuf + r * RAW_SLOT;
           mbar_arrive_expect_tx(&raw_full[r], (uint32_t)RAW_BYTES);
-          if (!kMN) {
+          if (!kMN)
             tma_load_3d(slot, &map_raw, &raw_full[r], kc * (BK / 2), rA, e);
-            tma_load_3d(slot + RAW_BYTES / 2, &map_raw, &raw_full[r], kc * (BK / 2), rB, e);
-          } else {
+          else
             tma_load_3d(slot, &map_raw, &raw_full[r], (nt * 256 + rank * 128) / 2, kc * BK, e);
-          }
+          issued |= 1u << r;
+          last_par = (last_par & ~(1u << r)) | (ph << r);
         }
-        // absmax of the block each decode thread t will decode -> amax[t]
-        float* amax = reinterpret_cast<float*>(slot + RAW_BYTES);
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int t = lane + 32 * qq;
-          int srow, sblk;
-          if (!kMN) {
-            srow = (t < 64) ? rA + t : rB + (t - 64);
-            sblk = kc;
-          } else {
-            srow = kc * BK + (t & 63);
-            sblk = nt * 4 + rank * 2 + (t >> 6);
+      }
+      if (!ok) {
+        // Let copies already issued land before the CTA's shared memory goes away.
+        for (int i = 0; i < RAW_STAGES; ++i)
+          if (issued & (1u << i)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&raw_full[i], (last_par >> i) & 1u) &&
+                   (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
+            }
           }
-          if (row_valid(nt, t))
-            cp_async_4(amax + t, p.absmax + ((size_t)e * p.stored_rows + srow) * blocks_per_row + sblk);
-        }
-        cp_async_arrive_noinc(&raw_full[r]);
-        issued |= 1u << r;
-        last_par = (last_par & ~(1u << r)) | (ph << r);
       }
     }
-    if (!ok && lane == 0) {
-      // Let copies already issued land before the CTA's shared memory goes away.
-      for (int i = 0; i < RAW_STAGES; ++i)
-        if (issued & (1u << i)) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&raw_full[i], (last_par >> i) & 1u) &&
-                 (long long)(globaltimer_ns() - t0) < p.timeout_ns) {
-          }
-        }
-    }
+    __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------ activation tiles + LoRA operands (one lane)
     if (lane == 0) {
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_la);
       tma_prefetch_desc(&map_lb);
-      uint32_t ti = 0, s = 0, ph = 0, issued = 0, last_par = 0;  // issued/last_par: per stage slot
+      uint32_t s = 0, ph = 0, issued = 0, last_par = 0;  // issued/last_par: per stage slot
+      uint32_t js = 0;                                       // stage uses whose slot was free
       bool ok = true;
-      for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
+      for (int u = pair; u < n_units && ok; u += n_pairs) {
         const int nt = u % p.n_nt;
         const int e = units[3 * (u / p.n_nt)], row0 = units[3 * (u / p.n_nt) + 1] + (int)rank * 128;
-        int rA = 0, rB = 0;
-        if (!kMN) kmajor_rows(nt, rA, rB);
-        if (!(ok = mbar_wait_lazy(lempty, (ti & 1) ^ 1, ctl, p.err, p.timeout_ns, 10, 64))) break;
-        mbar_arrive_expect_tx(lfull, (uint32_t)(512 * p.r_pad));
-        tma_load_2d(la, &map_la, lfull, 0, row0);
-        if (!kMN) {
-          tma_load_3d(lb, &map_lb, lfull, 0, rA, e);
-          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, 0, rB, e);
-        } else {
-          const int c0 = nt * 256 + rank * 128;
-          tma_load_3d(lb, &map_lb, lfull, c0, 0, e);
-          tma_load_3d(lb + 128 * p.r_pad, &map_lb, lfull, c0 + 64, 0, e);
+        const int rA = kMN ? 0 : kmajor_row0(nt);
+        // The unit's LoRA operands take one stage use ahead of its k-chunks; nothing is decoded into it,
+        // so this lane also stands in for the decode group's four bdone arrivals.
+        if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 10))) break;
+        st_release_shared(bfree, ++js);
+        {
+          uint8_t* la = stages + s * STAGE_BYTES;
+          uint8_t* lb = la + A_BYTES;
+          mbar_arrive_expect_tx(&xfull[s], (uint32_t)(512 * p.r_pad));
+          tma_load_2d(la, &map_la, &xfull[s], 0, row0);
+          if (!kMN) {
+            tma_load_3d(lb, &map_lb, &xfull[s], 0, rA, e);
+            tma_load_3d(lb + 128 * p.r_pad, &map_lb, &xfull[s], 0, rA + 64, e);
+          } else {
+            const int c0 = nt * 256 + rank * 128;
+            tma_load_3d(lb, &map_lb, &xfull[s], c0, 0, e);
+            tma_load_3d(lb + 128 * p.r_pad, &map_lb, &xfull[s], c0 + 64, 0, e);
+          }
+          for (int w = 0; w < kGroupWarps; ++w) mbar_arrive(&bdone[s]);
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
         }
         for (int kc = 0; kc < kchunks; ++kc) {
           if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 12))) break;
+          st_release_shared(bfree, ++js);  // the decode group of this use may store its tile
           mbar_arrive_expect_tx(&xfull[s], (uint32_t)A_BYTES);
           tma_load_2d(stages + s * STAGE_BYTES, &map_a, &xfull[s], kc * BK, row0);
           issued |= 1u << s;
@@ -334,60 +337,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     if (elect_one_sync()) {
       const uint32_t idesc = make_idesc_bf16(256, 256, false, kMN);
       const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
-      const uint32_t la_u = smem_u32(la), lb_u = smem_u32(lb);
       const uint32_t st_u = smem_u32(stages);
       const uint32_t bstep = kMN ? 128u : 2u;  // K16 step of B in the descriptor address field
-      uint32_t ti = 0, s = 0, ph = 0;          // unit counter; k-chunk stage slot and parity
+      // Descriptors of slot 0's tiles; slot s adds s * STAGE_BYTES to the address field (bits 0-13,
+      // address / 16: shared memory stays below 256 KB, so the sum cannot carry out of it).
+      const uint64_t adesc0 = make_sdesc(st_u, 16, 1024, kSw128);
+      const uint64_t bdesc0 = kMN ? make_sdesc(st_u + A_BYTES, 8192, 1024, kSw128)
+                                  : make_sdesc(st_u + A_BYTES, 16, 1024, kSw128);
+      uint32_t ti = 0, s = 0, ph = 0;  // unit counter; stage slot and parity
       bool ok = true;
-      // Both CTAs' halves of the k-chunk in slot s (activation tile and decoded
-      // weight tile) are in place; arms bfull[s] for its next use.
+      // Both CTAs' halves of the stage use in slot s are in place (one barrier, signalled by the
+      // two relays).
       auto wait_chunk = [&](uint32_t ss, uint32_t pp) -> bool {
-        if (!mbar_wait(&bdone[ss], pp, ctl, p.err, p.timeout_ns, 24)) return false;
-        if (!mbar_wait(&xfull[ss], pp, ctl, p.err, p.timeout_ns, 25)) return false;
-        if (!mbar_wait_cluster(&bfull[ss], pp, ctl, p.err, p.timeout_ns, 23)) return false;
-        mbar_arrive_expect_tx(&bfull[ss], 4);
-        return true;
+        return mbar_wait_cluster(&full[ss], pp, ctl, p.err, p.timeout_ns, 23);
       };
       for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
         const uint32_t b = ti & 1, use = ti >> 1;
         const uint32_t d = tmem + b * 256;
         if (!(ok = mbar_wait_cluster(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
         tc_fence_after();
-        if (!(ok = mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 21))) break;
-        if (!(ok = mbar_wait_cluster(lready, ti & 1, ctl, p.err, p.timeout_ns, 21))) break;
-        mbar_arrive_expect_tx(lready, 4);  // arm the next phase
+        // LoRA step first, from the unit's first stage use: acc = (s*p) . B_lora^T over K = r
+        // (overwrites the accumulator).
+        if (!(ok = wait_chunk(s, ph))) break;
         tc_fence_after();
-        // LoRA step first: acc = (s*p) . B_lora^T over K = r (overwrites the accumulator).
-        for (int ks = 0; ks < p.r_pad / 16; ++ks) {
-          const uint64_t bd = kMN ? make_sdesc(lb_u + 2048 * ks, 128 * p.r_pad, 1024, kSw128)
-                                  : make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz);
-          umma_bf16_2sm(d, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
+        {
+          const uint32_t la_u = st_u + s * STAGE_BYTES, lb_u = la_u + A_BYTES;
+          for (int ks = 0; ks < p.r_pad / 16; ++ks) {
+            const uint64_t bd = kMN ? make_sdesc(lb_u + 2048 * ks, 128 * p.r_pad, 1024, kSw128)
+                                    : make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz);
+            umma_bf16_2sm(d, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
+          }
+          umma_commit_2sm(&empty[s], 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
         }
-        umma_commit_2sm(lempty, 0x3);
         if (!(ok = wait_chunk(s, ph))) break;
         tc_fence_after();
         for (int kc = 0; kc < kchunks; ++kc) {
-          const uint32_t a0 = st_u + s * STAGE_BYTES;
-          const uint64_t adesc = make_sdesc(a0, 16, 1024, kSw128);
-          const uint64_t bdesc = kMN ? make_sdesc(a0 + A_BYTES, 8192, 1024, kSw128)
-                                     : make_sdesc(a0 + A_BYTES, 16, 1024, kSw128);
+          const uint64_t soff = (uint64_t)(s * (STAGE_BYTES >> 4));
+          const uint64_t adesc = adesc0 + soff, bdesc = bdesc0 + soff;
           const uint32_t s1 = (s + 1 == STAGES) ? 0 : s + 1, ph1 = (s + 1 == STAGES) ? ph ^ 1 : ph;
           const bool more = kc + 1 < kchunks;
 #pragma unroll
           for (int kk = 0; kk < BK / 16 - 1; ++kk)  // K16 step: +32 bytes of A; +32 (K-major) / +2048 bytes of B
             umma_bf16_2sm(d, adesc + 2 * kk, bdesc + bstep * kk, idesc, 1u);
           // Peek at the next k-chunk while the UMMAs above execute.
-          const bool next_ready = more && mbar_test_wait(&bdone[s1], ph1) && mbar_test_wait(&xfull[s1], ph1) &&
-                                  mbar_test_wait_cluster(&bfull[s1], ph1);
+          const bool next_ready = more && mbar_test_wait_cluster(&full[s1], ph1);
           umma_bf16_2sm(d, adesc + 2 * (BK / 16 - 1), bdesc + bstep * (BK / 16 - 1), idesc, 1u);
           umma_commit_2sm(&empty[s], 0x3);
           s = s1;
           ph = ph1;
           if (more) {
-            if (next_ready)
-              mbar_arrive_expect_tx(&bfull[s], 4);
-            else if (!(ok = wait_chunk(s, ph)))
-              break;
+            if (!next_ready && !(ok = wait_chunk(s, ph))) break;
             tc_fence_after();
           }
         }
@@ -400,77 +403,119 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 2 && rank == 1) {
-    // ------------------------------------------------ relay (odd CTA): its LoRA operands and each k-chunk's
-    // activation + decoded tiles are in place -> even CTA (one 4-byte st.async per event)
-    const uint32_t lready_even = mapa_shared(smem_u32(lready), 0);
-    const uint32_t bfull_even = mapa_shared(smem_u32(bfull), 0);
+  } else if (warp == 2) {
+    // ------------------------------------------------ relays: this CTA's half of each stage use (LoRA
+    // operands, or activation + decoded tiles) is in place -> the even CTA's full[s].  The odd CTA
+    // signals with one 4-byte st.async; the even CTA's relay arrives locally and arms the 4 bytes
+    // (which may land first: the transaction count goes negative until then).  Off the issuer's
+    // scheduler partition, so that the issuer tests one barrier per stage use.
+    const uint32_t full_even = mapa_shared(smem_u32(full), 0);
     const uint32_t sig_even = mapa_shared(smem_u32(sig), 0);
-    uint32_t ti = 0, s = 0, ph = 0;
+    uint32_t s = 0, ph = 0;
     bool ok = true;
-    for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
-      if (!(ok = __all_sync(kFull, mbar_wait(lfull, ti & 1, ctl, p.err, p.timeout_ns, 50)))) break;
-      if (lane == 0) st_async_signal(sig_even, lready_even, 1u);
-      for (int kc = 0; kc < kchunks; ++kc) {
+    for (int u = pair; u < n_units && ok; u += n_pairs) {
+      for (int kc = 0; kc <= kchunks; ++kc) {  // the unit's LoRA stage use, then its k-chunks
         ok = __all_sync(kFull, mbar_wait(&bdone[s], ph, ctl, p.err, p.timeout_ns, 51));
         if (ok) ok = __all_sync(kFull, mbar_wait(&xfull[s], ph, ctl, p.err, p.timeout_ns, 52));
         if (!ok) break;
-        if (lane == 0) st_async_signal(sig_even, bfull_even + 8 * s, 1u);
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive_expect_tx(&full[s], 4);
+          else
+            st_async_signal(sig_even, full_even + 8 * s, 1u);
+        }
         if (++s == STAGES) {
           s = 0;
           ph ^= 1;
         }
       }
     }
-  } else if (warp >= 4 && warp < kEpiWarp0) {
+  } else if (warp >= 4 && warp < kEpiWarp0 && decode_index(warp) >= 0) {
     // ------------------------------------------------ NF4 decode, groups take the k-chunks round robin
-    // Group g decodes chunk j (j % 4 == g) from code slot j % RAW_STAGES into
-    // registers, then waits for stage slot j % STAGES to be free and stores the tile.
-    const uint32_t grp = (warp - 4) >> 2;
-    const int t = (threadIdx.x - 128) & 127;
+    // Group g decodes the pair's k-chunks jj with jj % kGroups == g (chunk jj: unit jj / kchunks of the
+    // pair, k-chunk jj % kchunks) from code slot jj % RAW_STAGES into registers, then waits for its stage
+    // use (jj plus the LoRA uses of the units so far, plus one) to find its slot free and stores the tile.
+    // Each thread loads the block scale of its row for its group's next chunk while decoding the current one.
+    const int dix = decode_index(warp);
+    const uint32_t grp = (uint32_t)(dix / kGroupWarps);
+    const int t = 32 * (dix % kGroupWarps) + lane;  // the weight row (K-major) / code column pair this thread decodes
     const Nf4Shift ks = nf4_shift_consts();
     const int raw_off = kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32;
     // Row `drow` of the decoded 128B-swizzled tile: 16-byte chunk c at c ^ (drow % 8).
     const int drow = kMN ? (t & 63) : t;
     const uint32_t drow_off = (kMN ? (t >> 6) * 8192 : 0) + (drow >> 3) * 1024 + (drow & 7) * 128;
     const uint32_t b_u = smem_u32(stages) + A_BYTES;
-    uint32_t j = 0;  // chunk counter at the unit's start
-    bool ok = true;
-    for (int u = pair; u < n_units && ok; u += n_pairs, j += kchunks) {
-      const int nt = u % p.n_nt;
-      const bool valid = row_valid(nt, t);
-      for (int kc = (int)((grp + kGroups - j % kGroups) % kGroups); kc < kchunks; kc += kGroups) {
-        const uint32_t jj = j + kc;
-        const uint32_t r = jj % RAW_STAGES, rph = (jj / RAW_STAGES) & 1;
-        ok = __all_sync(kFull, mbar_wait(&raw_full[r], rph, ctl, p.err, p.timeout_ns, 30));
-        if (!ok) break;
-        const uint8_t* slot = rawbuf + r * RAW_SLOT;
-        const float amax = reinterpret_cast<const float*>(slot + RAW_BYTES)[t];
-        const uint4 q0 = *reinterpret_cast<const uint4*>(slot + raw_off);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(slot + raw_off + 16);
-        const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        // The codes are in registers: hand the code slot back before decoding, so the producer refills it
-        // a whole decode earlier (the proxy fence orders these generic reads before the next TMA write).
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&raw_empty[r]);
-        // Rows past the end of the matrix decode with a zero scale: all zeros.
-        const Nf4Planes pl = nf4_block_planes(valid ? amax : 0.0f);
-        uint32_t v[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) nf4_decode_word(codes[c], pl, ks, &v[4 * c]);
-        const uint32_t s = jj % STAGES, sph = (jj / STAGES) & 1;
-        ok = __all_sync(kFull, mbar_wait(&empty[s], sph ^ 1, ctl, p.err, p.timeout_ns, 31));
-        if (!ok) break;
-        const uint32_t dbase = b_u + s * STAGE_BYTES + drow_off;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(dbase + ((c ^ (drow & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-        // The proxy fence orders the tile stores before the UMMA reads them.
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bdone[s]);
+    // A cursor over this group's chunks, kept one chunk ahead of the decode: unit index ui of the pair,
+    // its k-chunk kc, unit u, its n-tile nt and expert e.  The block scale of this thread's row for the
+    // cursor's chunk is loaded a group iteration before it is used, with no division and no dependent
+    // load on the way (the expert of the unit after the cursor's is loaded a unit ahead): a stall there
+    // would hold up the decode that follows it in this warp's instruction stream.
+    const uint32_t n_chunks = (uint32_t)((n_units - pair + n_pairs - 1) / n_pairs) * (uint32_t)kchunks;
+    auto unit_expert = [&](int u) -> int { return u < n_units ? units[3 * (u / p.n_nt)] : 0; };
+    int c_ui = 0, c_kc = (int)grp, c_u = pair;
+    while (c_kc >= kchunks) {
+      c_kc -= kchunks;
+      ++c_ui;
+      c_u += n_pairs;
+    }
+    int c_nt = c_u % p.n_nt, c_e = unit_expert(c_u), e_after = unit_expert(c_u + n_pairs);
+    auto advance = [&]() {
+      c_kc += kGroups;
+      while (c_kc >= kchunks) {
+        c_kc -= kchunks;
+        ++c_ui;
+        c_u += n_pairs;
+        c_nt = c_u % p.n_nt;
+        c_e = e_after;
+        e_after = unit_expert(c_u + n_pairs);
       }
+    };
+    // Block scale of this thread's row for the cursor's chunk (0 for rows past the end of the matrix:
+    // all-zero decode).
+    auto block_scale = [&]() -> float {
+      if (c_u >= n_units || !row_valid(c_nt, t)) return 0.0f;
+      size_t idx;
+      if (!kMN)
+        idx = ((size_t)c_e * p.stored_rows + kmajor_row0(c_nt) + t) * blocks_per_row + c_kc;
+      else
+        idx = ((size_t)c_e * p.stored_rows + c_kc * BK + (t & 63)) * blocks_per_row + c_nt * 4 + rank * 2 + (t >> 6);
+      return __ldg(p.absmax + idx);
+    };
+    float amax_next = block_scale();
+    bool ok = true;
+    for (uint32_t jj = grp; jj < n_chunks && ok; jj += kGroups) {
+      const float amax = amax_next;
+      const uint32_t ui = (uint32_t)c_ui;  // the cursor is at chunk jj here
+      advance();
+      const uint32_t r = jj % RAW_STAGES, rph = (jj / RAW_STAGES) & 1;
+      ok = __all_sync(kFull, mbar_wait(&raw_full[r], rph, ctl, p.err, p.timeout_ns, 30));
+      if (!ok) break;
+      const uint8_t* slot = rawbuf + r * RAW_SLOT;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(slot + raw_off);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(slot + raw_off + 16);
+      const uint32_t codes[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      // The codes are in registers: hand the code slot back before decoding, so the producer refills it
+      // a whole decode earlier (the proxy fence orders these generic reads before the next TMA write).
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[r]);
+      amax_next = block_scale();
+      const Nf4Planes pl = nf4_block_planes(amax);
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) nf4_decode_word(codes[c], pl, ks, &v[4 * c]);
+      const uint32_t js = jj + ui + 1;  // stage use: one LoRA use ahead of each unit
+      const uint32_t s = js % STAGES;
+      ok = __all_sync(kFull, count_wait(bfree, js + 1, ctl, p.err, p.timeout_ns, 31));
+      if (!ok) break;
+      const uint32_t dbase = b_u + s * STAGE_BYTES + drow_off;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(dbase + ((c ^ (drow & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      // The proxy fence orders the tile stores before the UMMA reads them.
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bdone[s]);
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ epilogue
@@ -1437,7 +1482,7 @@ cudaError_t launch_nf4_gemm(const Nf4GemmHost& h, int num_sms, cudaStream_t stre
     mo1 = mo0;
   if (err != cudaSuccess) return err;
   if (!mn)
-    err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 32, 64);
+    err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 32, 128);
   else
     err = map_u8_3d(&mraw, h.nf4, h.stored_cols / 2, h.stored_rows, h.E, 64, 64);
   if (err != cudaSuccess) return err;
