@@ -131,34 +131,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, CtaCon
   }
 }
 
-// A monotonic shared-memory counter written by one thread with release
-// semantics and waited on by others (no phase aliasing however far the
-// waiters skip ahead, unlike an mbarrier's parity).
-__device__ __forceinline__ void st_release_shared(uint32_t* ctr, uint32_t v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(ctr)), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t* ctr) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(ctr)) : "memory");
-  return v;
-}
-// Waits until *ctr >= target, bounded like mbar_wait.
-__device__ __forceinline__ bool count_wait(const uint32_t* ctr, uint32_t target, CtaControl* ctl, DeviceError* err,
-                                           long long timeout_ns, int site) {
-  if ((int32_t)(ld_acquire_shared(ctr) - target) >= 0) return true;
-  const long long c0 = clock64(), limit = wait_limit_cycles(timeout_ns);
-  while (true) {
-    __nanosleep(32);
-    if ((int32_t)(ld_acquire_shared(ctr) - target) >= 0) return true;
-    if (ctl->abort) return false;
-    if (clock64() - c0 > limit) {
-      ctl->abort = 1;
-      record_error(err, E4B_ERR_DEVICE_TIMEOUT, site);
-      return false;
-    }
-  }
-}
-
 // Bounded wait for roles off the critical path (producers far ahead of their
 // consumers, epilogues waiting for a whole tile): sleeps `sleep_ns` between
 // polls so that the decoding warps get the issue slots.

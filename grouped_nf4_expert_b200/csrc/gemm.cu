@@ -59,48 +59,43 @@ __device__ __forceinline__ void store_row16(uint16_t* dst, const uint32_t (&w)[8
 // only its own tiles (no multicast loads).
 // Roles per CTA: warp 0 = NF4 codes into a ring of their own (one TMA per
 // k-chunk, filled far ahead), warp 1 = TMEM owner (both CTAs) and UMMA issuer
-// (even CTA only), warp 2 = relay (odd CTA), warp 3 = activation tiles and
-// LoRA operands, warps 4-19 = three decode groups taking the k-chunks round
-// robin (warps 5, 9, 13, 17, which share the issuer's scheduler partition,
-// idle), warps 20-23 = epilogue.  A stage slot holds one k-chunk's activation
-// tile and decoded weight tile, or, once per unit ahead of its k-chunks, the
-// unit's LoRA operands (so the LoRA step needs no buffers of its own and the
-// ring is five slots deep).  Decoders decode into registers from the code ring
-// (block scales: their own loads, a chunk ahead) and only wait for the slot to
-// be free to store (a counter the activation loader advances as it sees each
-// use's slot emptied), so a slot's round trip is the activation load plus a
-// store.
-// Each CTA's relay (warp 2) waits for its own half of a stage use (bdone,
-// xfull) and signals the even CTA's full[s], the one barrier the UMMA issuer
-// tests per stage use: the even CTA's relay with an arrive that also arms 4
+// (even CTA only), warp 2 = relay, warp 3 = activation tiles and LoRA
+// operands, warps 4-19 = four decode groups taking the k-chunks round robin,
+// warps 20-23 = epilogue.  Operands are staged in two rings: activation slots
+// (six; a unit's LoRA operands take two of them ahead of its k-chunks, so the
+// LoRA step needs no buffers of its own) and decoded-tile slots (one per decode
+// group).  The activation tile is the operand that arrives last (a TMA load of
+// ~1000+ cycles), so its ring is the deeper one; decoders decode into registers
+// from the code ring (block scales: their own loads, a chunk ahead) and only
+// wait for their own slot to be free to store.
+// Each CTA's relay (warp 2) waits for its own operands of an MMA step (xfull,
+// bdone) and signals the even CTA's full[], the one barrier the UMMA issuer
+// tests per step: the even CTA's relay with an arrive that also arms 4
 // transaction bytes, the odd CTA's with a 4-byte st.async whose mbarrier
 // complete_tx carries the cluster-scope release (a release-arrive would stall
 // the signalling warp for about a microsecond).  The issuer's instruction
 // stream is one dependent chain per k-chunk sharing its scheduler with four
 // decode warps, so it is kept short.  The issuer's commits arrive on both
-// CTAs' empty / accfull barriers.
+// CTAs' aempty / bempty / accfull barriers.
 namespace nf4g {
 constexpr int BM = 128;   // activation rows per CTA (256 per pair)
 constexpr int BN = 128;   // weight rows decoded per CTA (256 output columns per pair)
-constexpr int BK = 64, STAGES = 5;
+constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;                 // activation tile, K-major SW128
 constexpr int B_BYTES = BN * BK * 2;                 // dequantised weight tile
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
-// Decode groups; group g decodes the k-chunks j with j % kGroups == g.  With three groups the
-// decode warps stay out of the scheduler partition of the UMMA issuer (warps with warp % 4 == 1,
-// which then idle): the issuer's per-k-chunk instructions form one dependent chain, and beside
-// four ALU-bound decode warps each of them waited ~10 cycles for an issue slot.
-constexpr int kGroups = 4;
+constexpr int kGroups = 4;          // decode groups; group g decodes the k-chunks j with j % 4 == g
 constexpr int kGroupWarps = 4;      // warps per decode group (one per 32 weight rows)
-constexpr bool kDecodeSkipsIssuerPartition = (kGroups == 3);
-constexpr int RAW_STAGES = 2 * kGroups;  // code slot r always belongs to group r % kGroups (no phase aliasing)
+// Activation ring: SA slots.  A unit takes two activation uses for its LoRA operands (its p or q
+// rows, 128 x r_pad, and its LoRA weight rows, 128 x r_pad), then one per k-chunk.
+constexpr int SA = 6;
+// Decoded-tile ring: one slot per decode group (group g's chunks always use slot g).
+constexpr int SB = kGroups;
+constexpr int RAW_STAGES = 2 * kGroups;  // code slot r always belongs to group r % 4 (no phase aliasing)
 constexpr int RAW_BYTES = BN * BK / 2;               // NF4 codes as loaded
 constexpr int RAW_SLOT = RAW_BYTES;
-constexpr int RAW_OFF = STAGES * STAGE_BYTES;
-// A unit's LoRA operands (p or q rows of this CTA, 128 x r_pad; its LoRA weight
-// rows, 128 x r_pad) take the A and B halves of the stage slot before the unit's
-// first k-chunk.
-static_assert(BM * E4B_MAX_RANK * 2 <= A_BYTES && BN * E4B_MAX_RANK * 2 <= B_BYTES, "LoRA operands fit a stage");
+constexpr int B_OFF = SA * A_BYTES;
+constexpr int RAW_OFF = B_OFF + SB * B_BYTES;
+static_assert(BM * E4B_MAX_RANK * 2 <= A_BYTES && BN * E4B_MAX_RANK * 2 <= A_BYTES, "LoRA operands fit a slot");
 // Epilogue staging: per epilogue warp, two steps x up to three 32-row x 16-column output tiles.
 constexpr int kEpiTileBytes = 32 * 16 * 2;
 constexpr int kEpiStepBytes = 3 * kEpiTileBytes;
@@ -112,21 +107,14 @@ constexpr int EPI_OFF = RAW_OFF + RAW_STAGES * RAW_SLOT;
 constexpr int BAR_OFF = EPI_OFF + 4 * kEpiWarpBytes;
 constexpr int BAR_BYTES = 1024;
 constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;
-constexpr int kEpiWarp0 = 20;  // warps 4..19: decode warps (and, with three groups, the idle warps 5, 9, 13, 17)
+constexpr int kEpiWarp0 = 4 + kGroups * kGroupWarps;
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
-static_assert(kGroups * kGroupWarps == (kDecodeSkipsIssuerPartition ? 12 : 16), "decode warps among 4..19");
-// Index of decode warp `warp` (0 .. kGroups * kGroupWarps - 1), or -1 for an idle warp.
-__device__ __forceinline__ int decode_index(int warp) {
-  if (!kDecodeSkipsIssuerPartition) return warp - 4;
-  const int q = warp & 3;
-  return q == 1 ? -1 : 3 * ((warp - 4) >> 2) + (q == 0 ? 0 : q - 1);
-}
 constexpr int kTmemCols = 512;      // 2 accumulator buffers x 256 columns
-static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atom alignment");
+static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "swizzle atom alignment");
 static_assert(RAW_STAGES % kGroups == 0, "code slots are owned by one decode group each");
-// Decode groups learn that their stage slot is free from a monotonic counter (bfree);
-// the activation loader, the relay and the issuer wait for every stage use in order,
-// so their parity waits cannot alias.
+// Every barrier is waited on phase by phase by the roles that use it: the activation loader,
+// relays and issuer go through all activation uses and MMA steps in order, and a decode group
+// owns its decoded-tile slot and code slots, so no parity wait can alias.
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace nf4g
 
@@ -155,24 +143,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
   constexpr bool kMN = (MODE == kDgradDown || MODE == kDgradGateUp);  // B operand N-contiguous
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align1024(smem_dyn);
-  uint8_t* stages = smem;
+  uint8_t* aring = smem;          // [SA] activation tiles / LoRA operands
+  uint8_t* bring = smem + B_OFF;  // [SB] decoded weight tiles
   uint8_t* rawbuf = smem + RAW_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* raw_full = bars;                   // [RAW_STAGES] codes landed
   uint64_t* raw_empty = raw_full + RAW_STAGES; // [RAW_STAGES] codes read into registers (group's 4 warps)
-  uint64_t* xfull = raw_empty + RAW_STAGES;    // [STAGES] activation tile landed
-  uint64_t* full = xfull + STAGES;             // [STAGES] (even CTA) both CTAs' halves of the stage in place
-  uint64_t* empty = full + STAGES;             // [STAGES] stage consumed by the UMMAs
-  uint64_t* bdone = empty + STAGES;            // [STAGES] this CTA's decoded tile written (group's 4 warps)
-  uint64_t* accfull = bdone + STAGES;          // [2] accumulator buffer complete
+  uint64_t* xfull = raw_empty + RAW_STAGES;    // [SA] activation use landed
+  uint64_t* aempty = xfull + SA;               // [SA] activation slot consumed by the UMMAs
+  uint64_t* full = aempty + SA;                // [SA] (even CTA) both CTAs' operands of an MMA step in place
+  uint64_t* bdone = full + SA;                 // [SB] this CTA's decoded tile written (group's 4 warps)
+  uint64_t* bempty = bdone + SB;               // [SB] decoded-tile slot consumed by the UMMAs
+  uint64_t* accfull = bempty + SB;             // [2] accumulator buffer complete
   uint64_t* accempty = accfull + 2;            // [2] (even CTA) accumulator buffer drained in both CTAs
   uint64_t* drain = accfull + 4;               // (even CTA) all issued UMMAs finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 5);
   CtaControl* ctl = reinterpret_cast<CtaControl*>(accfull + 6);
   uint32_t* sig = reinterpret_cast<uint32_t*>(accfull + 7);  // target word of the st.async signals
-  // Stage uses whose slot is free (the activation loader's count of empty phases it has waited for): a decode
-  // group skips the uses of the other groups and the units' LoRA uses, so it cannot wait on empty's parity.
-  uint32_t* bfree = reinterpret_cast<uint32_t*>(accfull + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -181,18 +168,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       mbar_init(&raw_full[r], 1);
       mbar_init(&raw_empty[r], kGroupWarps);
     }
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < SA; ++s) {
       mbar_init(&xfull[s], 1);
+      mbar_init(&aempty[s], 1);
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < SB; ++s) {
       mbar_init(&bdone[s], kGroupWarps);
+      mbar_init(&bempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 8);
     }
     mbar_init(drain, 1);
-    *bfree = 0;
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -267,24 +256,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------ activation tiles + LoRA operands (one lane)
+    // Activation uses in order: per unit two for its LoRA operands (p or q rows into slot a, LoRA weight
+    // rows into slot a + 1, both copies completing on xfull[a]; xfull[a + 1] gets a plain arrival), then
+    // one per k-chunk.
     if (lane == 0) {
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_la);
       tma_prefetch_desc(&map_lb);
-      uint32_t s = 0, ph = 0, issued = 0, last_par = 0;  // issued/last_par: per stage slot
-      uint32_t js = 0;                                       // stage uses whose slot was free
+      uint32_t s = 0, ph = 0, issued = 0, last_par = 0;  // issued/last_par: per activation slot
+      auto issued_next = [&]() {
+        issued |= 1u << s;
+        last_par = (last_par & ~(1u << s)) | (ph << s);
+        if (++s == SA) {
+          s = 0;
+          ph ^= 1;
+        }
+      };
       bool ok = true;
       for (int u = pair; u < n_units && ok; u += n_pairs) {
         const int nt = u % p.n_nt;
         const int e = units[3 * (u / p.n_nt)], row0 = units[3 * (u / p.n_nt) + 1] + (int)rank * 128;
         const int rA = kMN ? 0 : kmajor_row0(nt);
-        // The unit's LoRA operands take one stage use ahead of its k-chunks; nothing is decoded into it,
-        // so this lane also stands in for the decode group's four bdone arrivals.
-        if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 10))) break;
-        st_release_shared(bfree, ++js);
+        const uint32_t s1 = (s + 1 == SA) ? 0 : s + 1, ph1 = (s + 1 == SA) ? ph ^ 1 : ph;
+        if (!(ok = mbar_wait(&aempty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 10))) break;
+        if (!(ok = mbar_wait(&aempty[s1], ph1 ^ 1, ctl, p.err, p.timeout_ns, 10))) break;
         {
-          uint8_t* la = stages + s * STAGE_BYTES;
-          uint8_t* lb = la + A_BYTES;
+          uint8_t* la = aring + s * A_BYTES;
+          uint8_t* lb = aring + s1 * A_BYTES;
           mbar_arrive_expect_tx(&xfull[s], (uint32_t)(512 * p.r_pad));
           tma_load_2d(la, &map_la, &xfull[s], 0, row0);
           if (!kMN) {
@@ -295,29 +293,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
             tma_load_3d(lb, &map_lb, &xfull[s], c0, 0, e);
             tma_load_3d(lb + 128 * p.r_pad, &map_lb, &xfull[s], c0 + 64, 0, e);
           }
-          for (int w = 0; w < kGroupWarps; ++w) mbar_arrive(&bdone[s]);
-          issued |= 1u << s;
-          last_par = (last_par & ~(1u << s)) | (ph << s);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
+          mbar_arrive(&xfull[s1]);
+          issued_next();
+          issued_next();
         }
         for (int kc = 0; kc < kchunks; ++kc) {
-          if (!(ok = mbar_wait(&empty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 12))) break;
-          st_release_shared(bfree, ++js);  // the decode group of this use may store its tile
+          if (!(ok = mbar_wait(&aempty[s], ph ^ 1, ctl, p.err, p.timeout_ns, 12))) break;
           mbar_arrive_expect_tx(&xfull[s], (uint32_t)A_BYTES);
-          tma_load_2d(stages + s * STAGE_BYTES, &map_a, &xfull[s], kc * BK, row0);
-          issued |= 1u << s;
-          last_par = (last_par & ~(1u << s)) | (ph << s);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
+          tma_load_2d(aring + s * A_BYTES, &map_a, &xfull[s], kc * BK, row0);
+          issued_next();
         }
       }
       if (!ok) {
-        for (int i = 0; i < STAGES; ++i)
+        for (int i = 0; i < SA; ++i)
           if (issued & (1u << i)) {
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&xfull[i], (last_par >> i) & 1u) &&
@@ -337,60 +325,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     if (elect_one_sync()) {
       const uint32_t idesc = make_idesc_bf16(256, 256, false, kMN);
       const uint32_t lswz = swz_for_row_bytes(2 * p.r_pad);
-      const uint32_t st_u = smem_u32(stages);
+      const uint32_t a_u = smem_u32(aring), b_u = smem_u32(bring);
       const uint32_t bstep = kMN ? 128u : 2u;  // K16 step of B in the descriptor address field
-      // Descriptors of slot 0's tiles; slot s adds s * STAGE_BYTES to the address field (bits 0-13,
+      // Descriptors of slot 0 of each ring; slot s adds s * slot bytes to the address field (bits 0-13,
       // address / 16: shared memory stays below 256 KB, so the sum cannot carry out of it).
-      const uint64_t adesc0 = make_sdesc(st_u, 16, 1024, kSw128);
-      const uint64_t bdesc0 = kMN ? make_sdesc(st_u + A_BYTES, 8192, 1024, kSw128)
-                                  : make_sdesc(st_u + A_BYTES, 16, 1024, kSw128);
-      uint32_t ti = 0, s = 0, ph = 0;  // unit counter; stage slot and parity
+      const uint64_t adesc0 = make_sdesc(a_u, 16, 1024, kSw128);
+      const uint64_t bdesc0 = kMN ? make_sdesc(b_u, 8192, 1024, kSw128) : make_sdesc(b_u, 16, 1024, kSw128);
+      uint32_t ti = 0;            // unit counter
+      uint32_t sa = 0, sb = 0;    // activation slot, decoded-tile slot
+      uint32_t fs = 0, fph = 0;   // MMA step: full[] slot and parity
       bool ok = true;
-      // Both CTAs' halves of the stage use in slot s are in place (one barrier, signalled by the
-      // two relays).
-      auto wait_chunk = [&](uint32_t ss, uint32_t pp) -> bool {
-        return mbar_wait_cluster(&full[ss], pp, ctl, p.err, p.timeout_ns, 23);
+      auto next_a = [&]() { sa = (sa + 1 == SA) ? 0 : sa + 1; };
+      auto next_f = [&]() {
+        if (++fs == SA) {
+          fs = 0;
+          fph ^= 1;
+        }
       };
+      // Both CTAs' operands of the MMA step are in place (one barrier, signalled by the two relays).
+      auto wait_step = [&]() -> bool { return mbar_wait_cluster(&full[fs], fph, ctl, p.err, p.timeout_ns, 23); };
       for (int u = pair; u < n_units && ok; u += n_pairs, ++ti) {
         const uint32_t b = ti & 1, use = ti >> 1;
         const uint32_t d = tmem + b * 256;
         if (!(ok = mbar_wait_cluster(&accempty[b], (use & 1) ^ 1, ctl, p.err, p.timeout_ns, 20))) break;
         tc_fence_after();
-        // LoRA step first, from the unit's first stage use: acc = (s*p) . B_lora^T over K = r
-        // (overwrites the accumulator).
-        if (!(ok = wait_chunk(s, ph))) break;
+        // LoRA step first: acc = (s*p) . B_lora^T over K = r (overwrites the accumulator), from the unit's
+        // two activation uses (p or q rows, then the LoRA weight rows).
+        if (!(ok = wait_step())) break;
         tc_fence_after();
         {
-          const uint32_t la_u = st_u + s * STAGE_BYTES, lb_u = la_u + A_BYTES;
+          const uint32_t sa1 = (sa + 1 == SA) ? 0 : sa + 1;
+          const uint32_t la_u = a_u + sa * A_BYTES, lb_u = a_u + sa1 * A_BYTES;
           for (int ks = 0; ks < p.r_pad / 16; ++ks) {
             const uint64_t bd = kMN ? make_sdesc(lb_u + 2048 * ks, 128 * p.r_pad, 1024, kSw128)
                                     : make_sdesc(lb_u + 32 * ks, 16, 16 * p.r_pad, lswz);
             umma_bf16_2sm(d, make_sdesc(la_u + 32 * ks, 16, 16 * p.r_pad, lswz), bd, idesc, ks > 0 ? 1u : 0u);
           }
-          umma_commit_2sm(&empty[s], 0x3);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
+          umma_commit_2sm(&aempty[sa], 0x3);
+          umma_commit_2sm(&aempty[sa1], 0x3);
+          next_a();
+          next_a();
+          next_f();
         }
-        if (!(ok = wait_chunk(s, ph))) break;
+        if (!(ok = wait_step())) break;
         tc_fence_after();
         for (int kc = 0; kc < kchunks; ++kc) {
-          const uint64_t soff = (uint64_t)(s * (STAGE_BYTES >> 4));
-          const uint64_t adesc = adesc0 + soff, bdesc = bdesc0 + soff;
-          const uint32_t s1 = (s + 1 == STAGES) ? 0 : s + 1, ph1 = (s + 1 == STAGES) ? ph ^ 1 : ph;
+          const uint64_t adesc = adesc0 + (uint64_t)(sa * (A_BYTES >> 4));
+          const uint64_t bdesc = bdesc0 + (uint64_t)(sb * (B_BYTES >> 4));
+          const uint32_t fs1 = (fs + 1 == SA) ? 0 : fs + 1, fph1 = (fs + 1 == SA) ? fph ^ 1 : fph;
           const bool more = kc + 1 < kchunks;
 #pragma unroll
           for (int kk = 0; kk < BK / 16 - 1; ++kk)  // K16 step: +32 bytes of A; +32 (K-major) / +2048 bytes of B
             umma_bf16_2sm(d, adesc + 2 * kk, bdesc + bstep * kk, idesc, 1u);
           // Peek at the next k-chunk while the UMMAs above execute.
-          const bool next_ready = more && mbar_test_wait_cluster(&full[s1], ph1);
+          const bool next_ready = more && mbar_test_wait_cluster(&full[fs1], fph1);
           umma_bf16_2sm(d, adesc + 2 * (BK / 16 - 1), bdesc + bstep * (BK / 16 - 1), idesc, 1u);
-          umma_commit_2sm(&empty[s], 0x3);
-          s = s1;
-          ph = ph1;
+          umma_commit_2sm(&aempty[sa], 0x3);
+          umma_commit_2sm(&bempty[sb], 0x3);
+          next_a();
+          sb = (sb + 1 == SB) ? 0 : sb + 1;
+          fs = fs1;
+          fph = fph1;
           if (more) {
-            if (!next_ready && !(ok = wait_chunk(s, ph))) break;
+            if (!next_ready && !(ok = wait_step())) break;
             tc_fence_after();
           }
         }
@@ -404,58 +401,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ------------------------------------------------ relays: this CTA's half of each stage use (LoRA
-    // operands, or activation + decoded tiles) is in place -> the even CTA's full[s].  The odd CTA
-    // signals with one 4-byte st.async; the even CTA's relay arrives locally and arms the 4 bytes
-    // (which may land first: the transaction count goes negative until then).  Off the issuer's
-    // scheduler partition, so that the issuer tests one barrier per stage use.
+    // ------------------------------------------------ relays: this CTA's operands of each MMA step (a
+    // unit's LoRA operands, or a k-chunk's activation and decoded tiles) are in place -> the even CTA's
+    // full[].  The odd CTA signals with one 4-byte st.async; the even CTA's relay arrives locally and
+    // arms the 4 bytes (which may land first: the transaction count goes negative until then).  Off the
+    // issuer's scheduler partition, so that the issuer tests one barrier per MMA step.
     const uint32_t full_even = mapa_shared(smem_u32(full), 0);
     const uint32_t sig_even = mapa_shared(smem_u32(sig), 0);
-    uint32_t s = 0, ph = 0;
+    uint32_t sa = 0, pha = 0, jb = 0, fs = 0;
     bool ok = true;
+    auto wait_a = [&]() -> bool {
+      const bool r = __all_sync(kFull, mbar_wait(&xfull[sa], pha, ctl, p.err, p.timeout_ns, 52));
+      if (++sa == SA) {
+        sa = 0;
+        pha ^= 1;
+      }
+      return r;
+    };
+    auto signal = [&]() {
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive_expect_tx(&full[fs], 4);
+        else
+          st_async_signal(sig_even, full_even + 8 * fs, 1u);
+      }
+      fs = (fs + 1 == SA) ? 0 : fs + 1;
+    };
     for (int u = pair; u < n_units && ok; u += n_pairs) {
-      for (int kc = 0; kc <= kchunks; ++kc) {  // the unit's LoRA stage use, then its k-chunks
-        ok = __all_sync(kFull, mbar_wait(&bdone[s], ph, ctl, p.err, p.timeout_ns, 51));
-        if (ok) ok = __all_sync(kFull, mbar_wait(&xfull[s], ph, ctl, p.err, p.timeout_ns, 52));
-        if (!ok) break;
-        if (lane == 0) {
-          if (rank == 0)
-            mbar_arrive_expect_tx(&full[s], 4);
-          else
-            st_async_signal(sig_even, full_even + 8 * s, 1u);
-        }
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1;
-        }
+      if (!(ok = wait_a()) || !(ok = wait_a())) break;  // the unit's two LoRA operand uses
+      signal();
+      for (int kc = 0; kc < kchunks; ++kc, ++jb) {
+        ok = __all_sync(kFull, mbar_wait(&bdone[jb % SB], (jb / SB) & 1, ctl, p.err, p.timeout_ns, 51));
+        if (!ok || !(ok = wait_a())) break;
+        signal();
       }
     }
-  } else if (warp >= 4 && warp < kEpiWarp0 && decode_index(warp) >= 0) {
+  } else if (warp >= 4 && warp < kEpiWarp0) {
     // ------------------------------------------------ NF4 decode, groups take the k-chunks round robin
-    // Group g decodes the pair's k-chunks jj with jj % kGroups == g (chunk jj: unit jj / kchunks of the
-    // pair, k-chunk jj % kchunks) from code slot jj % RAW_STAGES into registers, then waits for its stage
-    // use (jj plus the LoRA uses of the units so far, plus one) to find its slot free and stores the tile.
-    // Each thread loads the block scale of its row for its group's next chunk while decoding the current one.
-    const int dix = decode_index(warp);
-    const uint32_t grp = (uint32_t)(dix / kGroupWarps);
-    const int t = 32 * (dix % kGroupWarps) + lane;  // the weight row (K-major) / code column pair this thread decodes
+    // Group g decodes the pair's k-chunks jj with jj % 4 == g (chunk jj: unit jj / kchunks of the pair,
+    // k-chunk jj % kchunks) from code slot jj % RAW_STAGES into registers, then waits for its decoded-tile
+    // slot g to be free and stores the tile.  Each thread loads the block scale of its row for its
+    // group's next chunk while decoding the current one.
+    const uint32_t grp = (warp - 4) >> 2;
+    const int t = (threadIdx.x - 128) & 127;  // the weight row (K-major) / code column pair this thread decodes
     const Nf4Shift ks = nf4_shift_consts();
     const int raw_off = kMN ? (t & 63) * 64 + (t >> 6) * 32 : t * 32;
     // Row `drow` of the decoded 128B-swizzled tile: 16-byte chunk c at c ^ (drow % 8).
     const int drow = kMN ? (t & 63) : t;
     const uint32_t drow_off = (kMN ? (t >> 6) * 8192 : 0) + (drow >> 3) * 1024 + (drow & 7) * 128;
-    const uint32_t b_u = smem_u32(stages) + A_BYTES;
-    // A cursor over this group's chunks, kept one chunk ahead of the decode: unit index ui of the pair,
-    // its k-chunk kc, unit u, its n-tile nt and expert e.  The block scale of this thread's row for the
+    const uint32_t b_u = smem_u32(bring) + grp * B_BYTES;
+    // A cursor over this group's chunks, kept one chunk ahead of the decode: its k-chunk kc, unit u,
+    // the unit's n-tile nt and expert e.  The block scale of this thread's row for the
     // cursor's chunk is loaded a group iteration before it is used, with no division and no dependent
     // load on the way (the expert of the unit after the cursor's is loaded a unit ahead): a stall there
     // would hold up the decode that follows it in this warp's instruction stream.
     const uint32_t n_chunks = (uint32_t)((n_units - pair + n_pairs - 1) / n_pairs) * (uint32_t)kchunks;
     auto unit_expert = [&](int u) -> int { return u < n_units ? units[3 * (u / p.n_nt)] : 0; };
-    int c_ui = 0, c_kc = (int)grp, c_u = pair;
+    int c_kc = (int)grp, c_u = pair;
     while (c_kc >= kchunks) {
       c_kc -= kchunks;
-      ++c_ui;
       c_u += n_pairs;
     }
     int c_nt = c_u % p.n_nt, c_e = unit_expert(c_u), e_after = unit_expert(c_u + n_pairs);
@@ -463,7 +467,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       c_kc += kGroups;
       while (c_kc >= kchunks) {
         c_kc -= kchunks;
-        ++c_ui;
         c_u += n_pairs;
         c_nt = c_u % p.n_nt;
         c_e = e_after;
@@ -485,8 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
     bool ok = true;
     for (uint32_t jj = grp; jj < n_chunks && ok; jj += kGroups) {
       const float amax = amax_next;
-      const uint32_t ui = (uint32_t)c_ui;  // the cursor is at chunk jj here
-      advance();
+      advance();  // the cursor moves to this group's next chunk
       const uint32_t r = jj % RAW_STAGES, rph = (jj / RAW_STAGES) & 1;
       ok = __all_sync(kFull, mbar_wait(&raw_full[r], rph, ctl, p.err, p.timeout_ns, 30));
       if (!ok) break;
@@ -504,18 +506,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(nf4g::kThreads, 1)
       uint32_t v[32];
 #pragma unroll
       for (int c = 0; c < 8; ++c) nf4_decode_word(codes[c], pl, ks, &v[4 * c]);
-      const uint32_t js = jj + ui + 1;  // stage use: one LoRA use ahead of each unit
-      const uint32_t s = js % STAGES;
-      ok = __all_sync(kFull, count_wait(bfree, js + 1, ctl, p.err, p.timeout_ns, 31));
+      // slot grp's previous use (this group's chunk jj - 4) consumed by its UMMAs
+      ok = __all_sync(kFull, mbar_wait(&bempty[grp], ((jj / kGroups) & 1) ^ 1, ctl, p.err, p.timeout_ns, 31));
       if (!ok) break;
-      const uint32_t dbase = b_u + s * STAGE_BYTES + drow_off;
+      const uint32_t dbase = b_u + drow_off;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         st_shared_v4(dbase + ((c ^ (drow & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
       // The proxy fence orders the tile stores before the UMMA reads them.
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bdone[s]);
+      if (lane == 0) mbar_arrive(&bdone[grp]);
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ epilogue
