@@ -483,21 +483,41 @@ __global__ void __launch_bounds__(nf4v::kThreads, 1)
       for (int f = blockIdx.x; f < N; f += gridDim.x) {
         const int e = __ldg(p.topk_ids + f), row = __ldg(p.row_of_slot + f), t = f / p.k;
         const uint4* xs = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H);
+        // Each lane keeps kPrepBatch 16-byte pieces of a row in flight at once: a loop that waited for
+        // each piece in turn made this phase ~8 us long, and the first gate_up units wait for it.
+        constexpr int kPrepBatch = 4;
         if (pw == 0) {
           uint4* dst = reinterpret_cast<uint4*>(p.x_perm + (size_t)row * p.H);
-          for (int c = lane; c < vec; c += 32) dst[c] = __ldg(xs + c);
+          for (int c0 = lane; c0 < vec; c0 += 32 * kPrepBatch) {
+            uint4 xq[kPrepBatch];
+#pragma unroll
+            for (int i = 0; i < kPrepBatch; ++i)
+              if (c0 + 32 * i < vec) xq[i] = __ldg(xs + c0 + 32 * i);
+#pragma unroll
+            for (int i = 0; i < kPrepBatch; ++i)
+              if (c0 + 32 * i < vec) dst[c0 + 32 * i] = xq[i];
+          }
         }
         for (int jr = pw; jr < p.r; jr += kPrepWarps) {
           const uint4* ap = reinterpret_cast<const uint4*>(p.A_gu + ((size_t)e * p.r + jr) * p.H);
           float acc = 0.0f;
-          for (int c = lane; c < vec; c += 32) {
-            const uint4 xq = __ldg(xs + c), aq = __ldg(ap + c);
-            const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq);
-            const uint32_t* aw = reinterpret_cast<const uint32_t*>(&aq);
+          for (int c0 = lane; c0 < vec; c0 += 32 * kPrepBatch) {
+            uint4 xq[kPrepBatch], aq[kPrepBatch];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              acc = fmaf(bf16lo_to_f32(xw[i]), bf16lo_to_f32(aw[i]), acc);
-              acc = fmaf(bf16hi_to_f32(xw[i]), bf16hi_to_f32(aw[i]), acc);
+            for (int i = 0; i < kPrepBatch; ++i) {
+              const bool in = c0 + 32 * i < vec;
+              xq[i] = in ? __ldg(xs + c0 + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
+              aq[i] = in ? __ldg(ap + c0 + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int q = 0; q < kPrepBatch; ++q) {
+              const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq[q]);
+              const uint32_t* aw = reinterpret_cast<const uint32_t*>(&aq[q]);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                acc = fmaf(bf16lo_to_f32(xw[i]), bf16lo_to_f32(aw[i]), acc);
+                acc = fmaf(bf16hi_to_f32(xw[i]), bf16hi_to_f32(aw[i]), acc);
+              }
             }
           }
 #pragma unroll
