@@ -288,7 +288,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(cfg, args.gpus, "host memory"),
+        "config": workload_config(cfg, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -296,11 +296,14 @@ def run_reference(args):
     return 0
 
 
-def workload_config(cfg, world, l2_note):
+def workload_config(cfg, world):
+    """The workload's identity, the same dict in both arms' lines (the GPU arm's call sequence and graph
+    use are top-level keys of its own record)."""
     return {"workload": "%s: %s" % (cfg.name, cfg.note), "E": cfg.E, "H": cfg.H, "I": cfg.I,
             "top_k": cfg.top_k, "tokens_per_gpu": cfg.T, "global_batch": cfg.T * world, "r": cfg.r,
             "alpha": cfg.alpha, "routing": cfg.routing, "nf4_blocksize": 64, "parallelism": "dp%d" % world,
-            "passes": list(cfg.passes), "l2": l2_note}
+            "passes": list(cfg.passes),
+            "l2": "GPU arm: flushed between timed steps by a 256 MiB write; reference arm: host memory"}
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -512,10 +515,10 @@ def measure(ctx, cfg, headline):
 
     rec = {
         "value": value, "unit": "tokens/s", "ms_per_step": ms_per_step,
-        "config": dict(workload_config(cfg, world, "flushed between timed steps by a 256 MiB write"),
-                       cuda_graph=fwd_only, call=("e4b_moe_serve_fwd" if fwd_only else
-                                                  "route_permute + lora_fwd + lora_dgrad" +
-                                                  (" + lora_wgrad" if do_wgrad else ""))),
+        "config": workload_config(cfg, world),
+        "call": ("e4b_moe_serve_fwd" if fwd_only else
+                 "route_permute + lora_fwd + lora_dgrad" + (" + lora_wgrad" if do_wgrad else "")),
+        "cuda_graph": fwd_only,
         "tflops": flops * world / (ms_per_step / 1e3) / 1e12,
         "step_flop_per_gpu": flops,
         "roofline": roofline,
