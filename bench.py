@@ -392,6 +392,67 @@ def tensor_roofline(ctx, kern, gflops, steps, traffic):
             "algorithmic_flop_per_step": nf4_flop / steps, "per_mode": per_mode}
 
 
+def pipelined_e2e(ctx, K, blk, base, lora, d, ins, outs, houts, do_wgrad, grads):
+    """Device time (ms, max over ranks) of K training steps end to end through the public calls: every
+    step's inputs come from pinned host memory (`ins`) and its results (`outs`) go back to pinned host
+    memory, on two copy streams, so that step i+1's copy-in and step i's copy-out overlap the compute
+    of their neighbours.  Timed from the first copy-in to the last copy-out."""
+    import torch
+    from grouped_nf4_expert_b200 import parallel
+    dev = ctx.dev
+    cs = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    dins = [(d.x, d.logits, d.dY), tuple(t.clone() for t in (d.x, d.logits, d.dY))]
+    stage = [[torch.empty_like(t) for t in outs] for _ in range(2)]
+    hsets = [houts, [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]]
+    in_ready = [torch.cuda.Event() for _ in range(K)]
+    done = [torch.cuda.Event() for _ in range(K)]
+    out_done = [torch.cuda.Event() for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def copy_in(i):
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(done[i - 2])  # step i-2 used this input set
+            for dst, src in zip(dins[i % 2], ins):
+                dst.copy_(src, non_blocking=True)
+            in_ready[i].record(s_in)
+
+    ctx.sync_all()
+    t0.record(s_in)
+    copy_in(0)
+    for i in range(K):
+        if i + 1 < K:
+            copy_in(i + 1)
+        cs.wait_event(in_ready[i])
+        x, logits, dy = dins[i % 2]
+        blk.e4b_route_permute(logits, x, gather=False)
+        blk.e4b_grouped_nf4_lora_fwd(base, lora, x=x)
+        blk.e4b_grouped_nf4_lora_dgrad(base, lora, dy)
+        if do_wgrad:
+            blk.e4b_lora_wgrad()
+            if ctx.world > 1:
+                parallel.allreduce_lora_grads(grads)
+        if i >= 2:
+            cs.wait_event(out_done[i - 2])  # step i-2's results have left this staging set
+        for dst, src in zip(stage[i % 2], outs):
+            dst.copy_(src, non_blocking=True)
+        done[i].record(cs)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[i])
+            for dst, src in zip(hsets[i % 2], stage[i % 2]):
+                dst.copy_(src, non_blocking=True)
+            out_done[i].record(s_out)
+    t1.record(s_out)
+    ctx.sync_all()
+    ms = t0.elapsed_time(t1)
+    if ctx.world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        ctx.dist.all_reduce(t, op=ctx.dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
 def measure(ctx, cfg, headline):
     """Times one workload's step (its own passes) and returns its record."""
     import torch
@@ -508,10 +569,15 @@ def measure(ctx, cfg, headline):
         g_e2e, _ = ctx.capture(e2e_step)
         graphs.append(g_e2e)
         e2e_ms = ctx.timed(args.steps, g_e2e.replay)
+        e2e_how = "each step: copy-in, the serving call, copy-out, one CUDA graph"
     else:
-        e2e_ms = ctx.timed(args.steps, e2e_step)
+        e2e_ms = pipelined_e2e(ctx, args.steps, blk, base, lora, d, ins, outs, houts, do_wgrad, grads)
+        e2e_how = ("training loop: step i+1's inputs are copied in and step i's results copied out on two copy "
+                   "streams while the compute stream runs (inputs and results double-buffered on the device; "
+                   "each step's results are first copied to a device staging buffer on the compute stream)")
     e2e = {"value": cfg.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
+           "schedule": e2e_how}
 
     rec = {
         "value": value, "unit": "tokens/s", "ms_per_step": ms_per_step,
